@@ -1,0 +1,152 @@
+"""Named synthetic workloads shaped like the MiMo-V2 attention layers.
+
+Every workload is drawn by :mod:`global_attention_moe_b200.synth` with seed 0
+unless a caller passes another seed.  Q/K/V are i.i.d. N(0,1) rounded to BF16;
+the sink (sliding-window layers only) is N(0,1) per query head in FP32.
+
+Layer facts (miles docs "MiMo-V2.6-Flash", section 1 Model Introduction and
+section 5.4 Notable quirks; miles PR #3648 "add MiMo-V2.6-Flash-RL support",
+Design Notes): sliding-window layers attend the query plus 128 previous keys
+with a learnable sink, 8 KV heads and RoPE base 1e4; global layers are causal
+with 4 KV heads, RoPE base 1e7 and no sink; Q/K are 192-dim, V is 128-dim and
+scaled by 0.707; RoPE covers 64 of the 192 Q/K dims.  The 64 query heads are a
+choice of this build (the pages do not state the query-head count).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import synth
+
+LAYER_SWA = 0
+LAYER_GLOBAL = 1
+HEAD_DIM_QK = 192
+HEAD_DIM_V = 128
+ROPE_DIMS = 64
+V_SCALE = 0.707
+SWA_WINDOW = 128
+ROPE_BASE_SWA = 1e4
+ROPE_BASE_GLOBAL = 1e7
+
+
+@dataclass
+class Workload:
+    name: str
+    layer_kind: int
+    lengths: list
+    num_q_heads: int
+    num_kv_heads: int
+    window: int  # -1 for the global (causal) layer
+    rope_base: float
+    has_sink: bool
+    seed: int = 0
+    head_dim_qk: int = HEAD_DIM_QK
+    head_dim_v: int = HEAD_DIM_V
+    rope_dims: int = ROPE_DIMS
+    v_scale: float = V_SCALE
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def total_tokens(self) -> int:
+        return int(sum(self.lengths))
+
+    @property
+    def num_seqs(self) -> int:
+        return len(self.lengths)
+
+    @property
+    def max_seqlen(self) -> int:
+        return int(max(self.lengths)) if self.lengths else 0
+
+    def describe(self) -> dict:
+        return {
+            "workload": self.name,
+            "layer": "swa_sink" if self.layer_kind == LAYER_SWA else "global_causal",
+            "num_seqs": self.num_seqs,
+            "total_tokens": self.total_tokens,
+            "max_seqlen": self.max_seqlen,
+            "q_heads": self.num_q_heads,
+            "kv_heads": self.num_kv_heads,
+            "head_dim_qk": self.head_dim_qk,
+            "head_dim_v": self.head_dim_v,
+            "window": self.window,
+            "rope_base": self.rope_base,
+            "rope_dims": self.rope_dims,
+            "v_scale": self.v_scale,
+            "sink": self.has_sink,
+            "seed": self.seed,
+        }
+
+
+def attended_pairs(lengths, window: int, num_q_heads: int) -> int:
+    """(query head, query, key) triples attended: sum over queries of min(p+1, W+1)."""
+    total = 0
+    for L in lengths:
+        L = int(L)
+        if window < 0:
+            total += L * (L + 1) // 2
+        else:
+            w1 = window + 1
+            if L <= w1:
+                total += L * (L + 1) // 2
+            else:
+                total += w1 * (w1 + 1) // 2 + (L - w1) * w1
+    return total * num_q_heads
+
+
+def tiny_swa(seed: int = 0) -> Workload:
+    return Workload("tiny_swa_sink_T512_h4_kv1", LAYER_SWA, [512], 4, 1, SWA_WINDOW, ROPE_BASE_SWA, True, seed)
+
+
+def swa_4096(seed: int = 0) -> Workload:
+    return Workload("swa_sink_T4096_h64_kv8", LAYER_SWA, [4096], 64, 8, SWA_WINDOW, ROPE_BASE_SWA, True, seed)
+
+
+def swa_varlen(seed: int = 0) -> Workload:
+    lengths = synth.seq_lengths(seed, 16, 256, 2048).tolist()
+    return Workload("swa_sink_varlen_B16_U256_2048_h64_kv8", LAYER_SWA, lengths, 64, 8, SWA_WINDOW,
+                    ROPE_BASE_SWA, True, seed)
+
+
+def global_2x8192(seed: int = 0) -> Workload:
+    return Workload("global_causal_B2_L8192_h64_kv4", LAYER_GLOBAL, [8192, 8192], 64, 4, -1,
+                    ROPE_BASE_GLOBAL, False, seed)
+
+
+def swa_131072(seed: int = 0) -> Workload:
+    return Workload("swa_sink_T131072_h64_kv8", LAYER_SWA, [131072], 64, 8, SWA_WINDOW, ROPE_BASE_SWA, True, seed)
+
+
+WORKLOADS = {
+    "tiny": tiny_swa,
+    "swa4096": swa_4096,
+    "swa_varlen": swa_varlen,
+    "global": global_2x8192,
+    "swa_long": swa_131072,
+}
+
+
+@dataclass
+class Inputs:
+    q: np.ndarray          # uint16 BF16 bits [T, Hq, 192]
+    k: np.ndarray          # uint16 BF16 bits [T, Hkv, 192]
+    v: np.ndarray          # uint16 BF16 bits [T, Hkv, 128]
+    sink: np.ndarray | None  # float32 [Hq] or None
+    cu_seqlens: np.ndarray  # int32 [B+1]
+
+
+def make_inputs(w: Workload, threads: int | None = None) -> Inputs:
+    """Draw the workload's tensors in the order q, k, v, sink (separate streams)."""
+    T = w.total_tokens
+    q = synth.normal_bf16(w.seed, synth.STREAM_Q, (T, w.num_q_heads, w.head_dim_qk), threads)
+    k = synth.normal_bf16(w.seed, synth.STREAM_K, (T, w.num_kv_heads, w.head_dim_qk), threads)
+    v = synth.normal_bf16(w.seed, synth.STREAM_V, (T, w.num_kv_heads, w.head_dim_v), threads)
+    sink = synth.normal_f32(w.seed, synth.STREAM_SINK, w.num_q_heads) if w.has_sink else None
+    cu = synth.cu_seqlens_from_lengths(w.lengths)
+    return Inputs(q, k, v, sink, cu)
+
+
+def custom(name, layer_kind, lengths, hq, hkv, window, rope_base, has_sink, seed=0, v_scale=V_SCALE) -> Workload:
+    return Workload(name, layer_kind, list(lengths), hq, hkv, window, rope_base, has_sink, seed, v_scale=v_scale)
