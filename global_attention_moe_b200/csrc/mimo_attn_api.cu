@@ -1,0 +1,255 @@
+// mimo_attn_api.cu -- host side of the C ABI declared in include/mimo_attn.h:
+// argument validation (before any CUDA call), TMA tensor-map encoding, kernel
+// launch, the device error word and the host-buffer end-to-end entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mimo_attn.h"
+#include "attn_fwd_simple.cuh"
+#include "params.cuh"
+
+using namespace mimo;
+
+namespace {
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s bound on any single wait
+
+PFN_cuTensorMapEncodeTiled_v12000 tensormap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 view [rows, inner] (row-major) with a {64, 128} box and 128-byte swizzle.
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  auto enc = tensormap_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate(const void* q, const void* k, const void* v, const float* sink, const int32_t* cu,
+             const mimo_attn_dims* d, int layer_kind, int window, double rope_base, int rope_dims, float v_scale,
+             const void* out, const float* lse) {
+  if (!d) return MIMO_ERR_INVALID_ARG;
+  if (layer_kind != MIMO_LAYER_SWA && layer_kind != MIMO_LAYER_GLOBAL) return MIMO_ERR_INVALID_ARG;
+  if (d->num_seqs < 1 || d->total_tokens < 0 || d->max_seqlen < 0 || d->num_q_heads < 1 || d->num_kv_heads < 1)
+    return MIMO_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads != 0) return MIMO_ERR_INVALID_ARG;
+  if (d->max_seqlen > d->total_tokens) return MIMO_ERR_INVALID_ARG;
+  if (d->head_dim_qk < 1 || d->head_dim_v < 1) return MIMO_ERR_INVALID_ARG;
+  if (d->head_dim_qk != kHeadDimQK || d->head_dim_v != kHeadDimV) return MIMO_ERR_UNSUPPORTED;
+  if (rope_dims < 0 || rope_dims % 2 != 0 || rope_dims > d->head_dim_qk) return MIMO_ERR_INVALID_ARG;
+  if (rope_dims != kRopeDims) return MIMO_ERR_UNSUPPORTED;
+  if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return MIMO_ERR_INVALID_ARG;
+  if (!std::isfinite(v_scale)) return MIMO_ERR_INVALID_ARG;
+  if (layer_kind == MIMO_LAYER_SWA && window < 0) return MIMO_ERR_INVALID_ARG;
+  if (layer_kind == MIMO_LAYER_GLOBAL && sink != nullptr) return MIMO_ERR_INVALID_ARG;
+  if ((int64_t)d->num_q_heads * d->total_tokens > INT32_MAX) return MIMO_ERR_UNSUPPORTED;
+  if (!cu) return MIMO_ERR_INVALID_ARG;
+  if (d->total_tokens > 0) {
+    if (!q || !k || !v || !out || !lse) return MIMO_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+      return MIMO_ERR_INVALID_ARG;
+  }
+  if (sink && (reinterpret_cast<uintptr_t>(sink) & 3u)) return MIMO_ERR_INVALID_ARG;
+  return MIMO_OK;
+}
+
+void fill_params(FwdParams& P, const float* sink, const int32_t* cu, const mimo_attn_dims* d, int layer_kind,
+                 int window, double rope_base, float v_scale, void* out, float* lse) {
+  std::memset(&P, 0, sizeof P);
+  P.cu_seqlens = cu;
+  P.sink = sink;
+  P.out = static_cast<uint16_t*>(out);
+  P.lse = lse;
+  P.num_seqs = d->num_seqs;
+  P.total_tokens = d->total_tokens;
+  P.max_seqlen = d->max_seqlen;
+  P.hq = d->num_q_heads;
+  P.hkv = d->num_kv_heads;
+  P.group = d->num_q_heads / d->num_kv_heads;
+  P.window = (layer_kind == MIMO_LAYER_GLOBAL) ? -1 : window;
+  P.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDimQK)));
+  P.v_scale = v_scale;
+  P.wait_limit_ns = kDefaultWaitLimitNs;
+  for (int i = 0; i < kRopeDims / 2; ++i) P.theta[i] = std::pow(rope_base, -2.0 * i / kRopeDims);
+}
+
+int launch_simple(const void* q, const void* k, const void* v, const FwdParams& P, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!encode_2d(&tq, q, (uint64_t)P.hq * kHeadDimQK, P.total_tokens) ||
+      !encode_2d(&tk, k, (uint64_t)P.hkv * kHeadDimQK, P.total_tokens) ||
+      !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, P.total_tokens))
+    return MIMO_ERR_CUDA;
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
+  if (configured_device != dev) {
+    if (cudaFuncSetAttribute(attn_fwd_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             simple::kSmemBytes) != cudaSuccess)
+      return MIMO_ERR_CUDA;
+    configured_device = dev;
+  }
+  if (P.max_seqlen == 0) return MIMO_OK;
+  dim3 grid((P.max_seqlen + kBlockM - 1) / kBlockM, P.num_seqs, P.hq);
+  attn_fwd_simple_kernel<<<grid, simple::kThreads, simple::kSmemBytes, stream>>>(tq, tk, tv, P);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the bounded wait must give up.
+  const bool ok = mbar_wait(&bar, 0, limit_ns);
+  if (!ok && threadIdx.x == 0) atomicOr(&g_mimo_error, kErrTimeout);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+int mimo_attn_fwd(const void* q, const void* k, const void* v, const float* sink, const int32_t* cu_seqlens,
+                  const mimo_attn_dims* dims, int layer_kind, int window, double rope_base, int rope_dims,
+                  float v_scale, void* out, float* lse, void* stream) {
+  int st = validate(q, k, v, sink, cu_seqlens, dims, layer_kind, window, rope_base, rope_dims, v_scale, out, lse);
+  if (st != MIMO_OK) return st;
+  if (dims->total_tokens == 0) return MIMO_OK;
+  FwdParams P;
+  fill_params(P, sink, cu_seqlens, dims, layer_kind, window, rope_base, v_scale, out, lse);
+  return launch_simple(q, k, v, P, static_cast<cudaStream_t>(stream));
+}
+
+size_t mimo_attn_host_workspace_size(const mimo_attn_dims* d, int has_sink) {
+  if (!d || d->num_seqs < 1 || d->total_tokens < 0 || d->num_q_heads < 1 || d->num_kv_heads < 1 ||
+      d->head_dim_qk < 1 || d->head_dim_v < 1)
+    return 0;
+  const size_t T = d->total_tokens, hq = d->num_q_heads, hkv = d->num_kv_heads;
+  size_t n = 0;
+  n += align256(T * hq * d->head_dim_qk * 2);   // q
+  n += align256(T * hkv * d->head_dim_qk * 2);  // k
+  n += align256(T * hkv * d->head_dim_v * 2);   // v
+  n += has_sink ? align256(hq * 4) : 0;         // sink
+  n += align256((d->num_seqs + 1) * 4);         // cu_seqlens
+  n += align256(T * hq * d->head_dim_v * 2);    // out
+  n += align256(hq * T * 4);                    // lse
+  return n;
+}
+
+int mimo_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, const float* sink_host,
+                       const int32_t* cu_host, const mimo_attn_dims* d, int layer_kind, int window,
+                       double rope_base, int rope_dims, float v_scale, void* out_host, float* lse_host,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!d || !cu_host || !workspace) return MIMO_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return MIMO_ERR_INVALID_ARG;
+  const size_t need = mimo_attn_host_workspace_size(d, sink_host != nullptr);
+  if (need == 0 || workspace_bytes < need) return MIMO_ERR_INVALID_ARG;
+  // cu_seqlens is in host memory here, so it is checked in full before any copy.
+  if (cu_host[0] != 0 || cu_host[d->num_seqs] != d->total_tokens) return MIMO_ERR_INVALID_ARG;
+  for (int b = 0; b < d->num_seqs; ++b) {
+    const int64_t len = (int64_t)cu_host[b + 1] - cu_host[b];
+    if (len < 0 || len > d->max_seqlen) return MIMO_ERR_INVALID_ARG;
+  }
+  const size_t T = d->total_tokens, hq = d->num_q_heads, hkv = d->num_kv_heads;
+  const size_t bq = T * hq * d->head_dim_qk * 2, bk = T * hkv * d->head_dim_qk * 2, bv = T * hkv * d->head_dim_v * 2;
+  const size_t bs = sink_host ? hq * 4 : 0, bc = (d->num_seqs + 1) * 4, bo = T * hq * d->head_dim_v * 2,
+               bl = hq * T * 4;
+  char* w = static_cast<char*>(workspace);
+  char* dq = w;
+  char* dk = dq + align256(bq);
+  char* dv = dk + align256(bk);
+  char* ds = dv + align256(bv);
+  char* dc = ds + (sink_host ? align256(bs) : 0);
+  char* dout = dc + align256(bc);
+  char* dl = dout + align256(bo);
+  int st = validate(T ? dq : nullptr, T ? dk : nullptr, T ? dv : nullptr, sink_host ? (const float*)ds : nullptr,
+                    (const int32_t*)dc, d, layer_kind, window, rope_base, rope_dims, v_scale, T ? dout : nullptr,
+                    T ? (const float*)dl : nullptr);
+  if (st != MIMO_OK) return st;
+  if (T > 0 && (!q_host || !k_host || !v_host || !out_host || !lse_host)) return MIMO_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  bool ok = true;
+  if (T > 0) {
+    ok = ok && cudaMemcpyAsync(dq, q_host, bq, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dk, k_host, bk, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dv, v_host, bv, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  }
+  if (sink_host) ok = ok && cudaMemcpyAsync(ds, sink_host, bs, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  ok = ok && cudaMemcpyAsync(dc, cu_host, bc, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  if (!ok) return MIMO_ERR_CUDA;
+  if (T > 0) {
+    st = mimo_attn_fwd(dq, dk, dv, sink_host ? (const float*)ds : nullptr, (const int32_t*)dc, d, layer_kind,
+                       window, rope_base, rope_dims, v_scale, dout, (float*)dl, stream);
+    if (st != MIMO_OK) return st;
+    ok = ok && cudaMemcpyAsync(out_host, dout, bo, cudaMemcpyDeviceToHost, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(lse_host, dl, bl, cudaMemcpyDeviceToHost, s) == cudaSuccess;
+  }
+  ok = ok && cudaStreamSynchronize(s) == cudaSuccess;
+  return ok ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
+int mimo_attn_check(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MIMO_ERR_CUDA;
+  unsigned int e = 0;
+  if (cudaMemcpyFromSymbol(&e, g_mimo_error, sizeof e) != cudaSuccess) return MIMO_ERR_CUDA;
+  if (e) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_mimo_error, &zero, sizeof zero) != cudaSuccess) return MIMO_ERR_CUDA;
+  }
+  if (e & kErrTimeout) return MIMO_ERR_TIMEOUT;
+  if (e & kErrRange) return MIMO_ERR_RANGE;
+  if (e & kErrSeqlens) return MIMO_ERR_BAD_SEQLENS;
+  return MIMO_OK;
+}
+
+int mimo_attn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000ull || limit_ns > 10000000000ull) return MIMO_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(limit_ns);
+  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  return mimo_attn_check(stream);
+}
+
+const char* mimo_attn_status_string(int status) {
+  switch (status) {
+    case MIMO_OK: return "ok";
+    case MIMO_ERR_INVALID_ARG: return "invalid argument";
+    case MIMO_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MIMO_ERR_CUDA: return "CUDA error";
+    case MIMO_ERR_TIMEOUT: return "bounded wait timed out in a kernel";
+    case MIMO_ERR_RANGE: return "rotated Q/K value outside the FP16 range";
+    case MIMO_ERR_BAD_SEQLENS: return "cu_seqlens inconsistent with dims";
+    default: return "unknown status";
+  }
+}
+
+int mimo_attn_version(void) { return (1 << 16) | 0; }
+
+}  // extern "C"

@@ -1,0 +1,135 @@
+"""Python binding of the C-ABI library ``libmimo_attn.so`` (include/mimo_attn.h).
+
+Argument marshalling only: torch tensors supply device memory and the current
+CUDA stream; every step of the attention forward runs in the library's CUDA
+kernels.  There is no CPU or eager fallback -- if the library is missing the
+import of this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "_build", "libmimo_attn.so")
+
+LAYER_SWA = 0
+LAYER_GLOBAL = 1
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BAD_SEQLENS = range(7)
+
+# Every symbol include/mimo_attn.h declares.
+SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host", "mimo_attn_check",
+           "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_version")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("total_tokens", ctypes.c_int32), ("max_seqlen", ctypes.c_int32),
+                ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim_qk", ctypes.c_int32), ("head_dim_v", ctypes.c_int32)]
+
+
+class MimoAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m global_attention_moe_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, D, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_float
+    lib.mimo_attn_fwd.restype = I
+    lib.mimo_attn_fwd.argtypes = [P, P, P, P, P, ctypes.POINTER(Dims), I, I, D, I, F, P, P, P]
+    lib.mimo_attn_host_workspace_size.restype = ctypes.c_size_t
+    lib.mimo_attn_host_workspace_size.argtypes = [ctypes.POINTER(Dims), I]
+    lib.mimo_attn_fwd_host.restype = I
+    lib.mimo_attn_fwd_host.argtypes = [P, P, P, P, P, ctypes.POINTER(Dims), I, I, D, I, F, P, P, P,
+                                       ctypes.c_size_t, P]
+    lib.mimo_attn_check.restype = I
+    lib.mimo_attn_check.argtypes = [P]
+    lib.mimo_attn_selftest_wait_timeout.restype = I
+    lib.mimo_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
+    lib.mimo_attn_status_string.restype = ctypes.c_char_p
+    lib.mimo_attn_status_string.argtypes = [I]
+    lib.mimo_attn_version.restype = I
+    lib.mimo_attn_version.argtypes = []
+    return lib
+
+
+LIB = _load()
+
+
+def status_string(status: int) -> str:
+    return LIB.mimo_attn_status_string(int(status)).decode()
+
+
+def version() -> tuple[int, int]:
+    v = LIB.mimo_attn_version()
+    return v >> 16, v & 0xFFFF
+
+
+def make_dims(num_seqs, total_tokens, max_seqlen, hq, hkv, dqk=192, dv=128) -> Dims:
+    return Dims(int(num_seqs), int(total_tokens), int(max_seqlen), int(hq), int(hkv), int(dqk), int(dv))
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def fwd_raw(q_ptr, k_ptr, v_ptr, sink_ptr, cu_ptr, dims: Dims, layer_kind, window, rope_base, rope_dims, v_scale,
+            out_ptr, lse_ptr, stream_handle) -> int:
+    """Direct C-ABI call with integer device pointers; returns the status code."""
+    return LIB.mimo_attn_fwd(q_ptr, k_ptr, v_ptr, sink_ptr, cu_ptr, ctypes.byref(dims), int(layer_kind),
+                             int(window), float(rope_base), int(rope_dims), float(v_scale), out_ptr, lse_ptr,
+                             stream_handle)
+
+
+def fwd(q, k, v, sink, cu_seqlens, max_seqlen, layer_kind, window, rope_base, rope_dims=64, v_scale=0.707,
+        out=None, lse=None, stream=None):
+    """Attention forward on CUDA tensors (bf16 q/k/v in THD layout, int32 cu_seqlens,
+    fp32 sink or None).  Returns (out bf16 [T, Hq, 128], lse fp32 [Hq, T])."""
+    import torch
+    T, hq, dqk = q.shape
+    hkv, dv = k.shape[1], v.shape[2]
+    for t in (q, k, v):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("q/k/v must be contiguous bf16 CUDA tensors")
+    if out is None:
+        out = torch.empty((T, hq, dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=q.device)
+    dims = make_dims(cu_seqlens.numel() - 1, T, max_seqlen, hq, hkv, dqk, dv)
+    st = fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), sink.data_ptr() if sink is not None else None,
+                 cu_seqlens.data_ptr(), dims, layer_kind, window, rope_base, rope_dims, v_scale, out.data_ptr(),
+                 lse.data_ptr(), _stream_handle(stream))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_attn_fwd")
+    return out, lse
+
+
+def host_workspace_size(dims: Dims, has_sink: bool) -> int:
+    return LIB.mimo_attn_host_workspace_size(ctypes.byref(dims), int(bool(has_sink)))
+
+
+def fwd_host(q_host, k_host, v_host, sink_host, cu_host, dims: Dims, layer_kind, window, rope_base, rope_dims,
+             v_scale, out_host, lse_host, workspace, stream=None):
+    """End-to-end call from (pinned) host tensors through a caller-provided device workspace."""
+    st = LIB.mimo_attn_fwd_host(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
+                                sink_host.data_ptr() if sink_host is not None else None, cu_host.data_ptr(),
+                                ctypes.byref(dims), int(layer_kind), int(window), float(rope_base), int(rope_dims),
+                                float(v_scale), out_host.data_ptr(), lse_host.data_ptr(), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_attn_fwd_host")
+
+
+def check(stream=None) -> int:
+    """Sync the stream and return (and clear) the device error status."""
+    return LIB.mimo_attn_check(_stream_handle(stream))
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> int:
+    return LIB.mimo_attn_selftest_wait_timeout(int(limit_ns), _stream_handle(stream))

@@ -1,0 +1,161 @@
+/*
+ * mimo_attn.h -- C ABI of the B200 (sm_100a) attention forward for the
+ * MiMo-V2 text decoder: the sliding-window layer with a learnable per-head
+ * sink and the global causal layer.
+ *
+ * The operation (miles PR #3648 "add MiMo-V2.6-Flash-RL support", Motivation
+ * and Design Notes; miles docs "MiMo-V2.6-Flash", section 1 Model Introduction
+ * and section 5.4 Notable quirks; Megatron-LM issue #2976, Architecture
+ * Analysis; Megatron-Bridge API doc "mimo_v2_flash_bridge", module summary):
+ *
+ *   For every packed sequence b (tokens cu_seqlens[b] .. cu_seqlens[b+1]-1),
+ *   local position p and query head h, with KV head g = h / (Hq / Hkv):
+ *     q~ = rope(q[t, h], p), k~_j = rope(k[s_b + j, g], j)   (first rope_dims
+ *          dims, rotate-half pairs (i, i + rope_dims/2), theta_i =
+ *          rope_base^(-2i/rope_dims), positions restart at 0 per sequence)
+ *     keys j with 0 <= j <= p and (global layer, or p - j <= window)
+ *     s_j = q~ . k~_j / sqrt(head_dim_qk)
+ *     lse = ln( sum_j exp(s_j) + exp(sink[h]) )   (sink term only if sink != NULL)
+ *     out[t, h] = sum_j exp(s_j - lse) * v_scale * v[s_b + j, g]
+ *   window = 128 gives the query plus 128 previous keys, 129 in total (miles
+ *   docs section 5.4); window = 127 gives the 128-key HF variant.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are caller-owned CUDA global memory on the current
+ *     device; host pointers are caller-owned host memory.  The library keeps
+ *     no pointer after a call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Kernels run asynchronously on it; only the entry points that
+ *     say so synchronise.
+ *   - Return values are mimo_status codes.  Argument checks happen before any
+ *     CUDA call, so a rejected call has no side effect.
+ *   - All tensors are dense, row-major and contiguous in THD layout
+ *     (tokens, heads, dims).  Every device pointer must be 16-byte aligned.
+ */
+#ifndef MIMO_ATTN_H_
+#define MIMO_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MIMO_API __attribute__((visibility("default")))
+#else
+#define MIMO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MIMO_LAYER_SWA = 0,    /* sliding window (`window` previous keys) with optional sink */
+  MIMO_LAYER_GLOBAL = 1  /* causal over the whole sequence, no sink */
+} mimo_layer_kind;
+
+typedef enum {
+  MIMO_OK = 0,
+  MIMO_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, inconsistent dims */
+  MIMO_ERR_UNSUPPORTED = 2, /* valid for the method but not built: head dims other than 192/128, rope_dims != 64 */
+  MIMO_ERR_CUDA = 3,        /* a CUDA runtime/driver call or kernel launch failed */
+  MIMO_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (reported by mimo_attn_check) */
+  MIMO_ERR_RANGE = 5,       /* a rotated Q/K value exceeded the FP16 range (|x| > 65504) */
+  MIMO_ERR_BAD_SEQLENS = 6  /* the kernel found cu_seqlens inconsistent with dims (reported by mimo_attn_check) */
+} mimo_status;
+
+/* Shapes.  Supported: head_dim_qk = 192, head_dim_v = 128,
+ * num_q_heads % num_kv_heads == 0, num_seqs >= 1, total_tokens >= 0,
+ * max_seqlen >= every sequence length (it sizes the launch grid). */
+typedef struct {
+  int32_t num_seqs;
+  int32_t total_tokens;
+  int32_t max_seqlen;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim_qk;
+  int32_t head_dim_v;
+} mimo_attn_dims;
+
+/*
+ * Attention forward on device buffers.
+ *   q          bf16 [T, Hq, 192]          (device)
+ *   k          bf16 [T, Hkv, 192]         (device)
+ *   v          bf16 [T, Hkv, 128]         (device)
+ *   sink       fp32 [Hq] or NULL          (device) per-query-head sink logit in
+ *              score units (not multiplied by the softmax scale); it joins the
+ *              softmax denominator and carries no value.  SWA only: a non-NULL
+ *              sink with MIMO_LAYER_GLOBAL is MIMO_ERR_INVALID_ARG.
+ *   cu_seqlens int32 [num_seqs + 1]       (device) cu[0] = 0, non-decreasing,
+ *              cu[num_seqs] = T, lengths <= max_seqlen.  The host cannot read it
+ *              without a sync, so a violation is detected by the kernel, which
+ *              skips that sequence and records MIMO_ERR_BAD_SEQLENS for
+ *              mimo_attn_check.  Empty sequences are allowed.
+ *   layer_kind MIMO_LAYER_SWA or MIMO_LAYER_GLOBAL
+ *   window     SWA: keys j with p - window <= j <= p (window >= 0); ignored for GLOBAL
+ *   rope_base  RoPE base (1e4 for SWA, 1e7 for global in MiMo-V2.6), > 0
+ *   rope_dims  must be 64 (the first 64 of the 192 Q/K dims are rotated)
+ *   v_scale    factor applied to V before P.V (0.707 in the model)
+ *   out        bf16 [T, Hq, 128]          (device) every row of every head is written
+ *   lse        fp32 [Hq, T]               (device) natural-log normaliser, including
+ *              the sink term
+ * Rotated Q/K rope dims enter the tensor cores as FP16 (the pass-through dims
+ * stay BF16), so |q|, |k| on the first 64 dims must stay below 2^15; a larger
+ * rotated value is recorded as MIMO_ERR_RANGE for mimo_attn_check.
+ * Allocates nothing.  Does not synchronise.
+ */
+MIMO_API int mimo_attn_fwd(const void* q, const void* k, const void* v, const float* sink,
+                  const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind,
+                  int window, double rope_base, int rope_dims, float v_scale, void* out,
+                  float* lse, void* stream);
+
+/*
+ * Bytes of device workspace mimo_attn_fwd_host needs for these dims
+ * (q, k, v, sink, cu_seqlens, out and lse, each 256-byte aligned).
+ * Returns 0 for invalid dims.
+ */
+MIMO_API size_t mimo_attn_host_workspace_size(const mimo_attn_dims* dims, int has_sink);
+
+/*
+ * End-to-end forward from HOST buffers (same layouts and meaning as
+ * mimo_attn_fwd; q/k/v/out are bf16 bit patterns in host memory, pinned for
+ * asynchronous copies).  The caller passes a device workspace of at least
+ * mimo_attn_host_workspace_size bytes, 256-byte aligned.  The call copies the
+ * inputs host->device on `stream`, runs the forward, copies out and lse
+ * device->host and synchronises the stream before returning, so the host
+ * buffers hold the result on return.  Allocates nothing.
+ */
+MIMO_API int mimo_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                       const float* sink_host, const int32_t* cu_seqlens_host,
+                       const mimo_attn_dims* dims, int layer_kind, int window, double rope_base,
+                       int rope_dims, float v_scale, void* out_host, float* lse_host,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error
+ * word for the current device: MIMO_ERR_TIMEOUT, MIMO_ERR_RANGE or
+ * MIMO_ERR_BAD_SEQLENS if a kernel recorded one since the last check (the
+ * lowest-numbered one is returned), MIMO_ERR_CUDA if the sync failed, else
+ * MIMO_OK.
+ */
+MIMO_API int mimo_attn_check(void* stream);
+
+/*
+ * Failure-detection self test: launches one CTA that waits on a shared-memory
+ * barrier nothing ever arrives on, with a wait limit of `limit_ns`
+ * nanoseconds (1e3 .. 1e10).  The wait gives up, records MIMO_ERR_TIMEOUT
+ * and the kernel returns; this call synchronises `stream` and returns what
+ * mimo_attn_check returns (MIMO_ERR_TIMEOUT when the bounded wait works).
+ */
+MIMO_API int mimo_attn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/* Static description of a status code (never NULL). */
+MIMO_API const char* mimo_attn_status_string(int status);
+
+/* ABI version: (major << 16) | minor. */
+MIMO_API int mimo_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MIMO_ATTN_H_ */

@@ -1,0 +1,111 @@
+"""The C-ABI library: it loads, exports every symbol include/mimo_attn.h
+declares, and rejects bad arguments before touching CUDA (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from global_attention_moe_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def M():
+    build.build()
+    from global_attention_moe_b200 import mimo_attn
+    return mimo_attn
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "mimo_attn.h")).read()
+    return sorted(set(re.findall(r"MIMO_API\s+[\w\s\*]*?\b(mimo_attn_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(M):
+    declared = header_functions()
+    assert declared and sorted(M.SYMBOLS) == declared
+    nm = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (mimo_attn_\w+)", nm))
+    assert set(declared) <= exported
+    for name in declared:
+        assert getattr(M.LIB, name) is not None
+
+
+def test_status_strings_and_version(M):
+    for s in range(7):
+        assert M.status_string(s) and M.status_string(s) != "unknown status"
+    assert M.status_string(99) == "unknown status"
+    assert M.version()[0] == 1
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def call(M, dims, layer=0, window=128, base=1e4, rope_dims=64, sink=None, q=FAKE, out=FAKE, lse=FAKE):
+    return M.fwd_raw(q, FAKE, FAKE, sink, FAKE, dims, layer, window, base, rope_dims, 0.707, out, lse, None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(dims=dict(hq=6, hkv=4)), 1),             # Hq % Hkv != 0
+    (dict(dims=dict(dqk=128)), 2),                  # head dims other than 192/128
+    (dict(dims=dict(dv=192)), 2),
+    (dict(rope_dims=32), 2),                        # only 64 rotary dims are built
+    (dict(rope_dims=63), 1),                        # odd
+    (dict(rope_dims=256), 1),                       # > head dim
+    (dict(window=-1), 1),                           # SWA needs window >= 0
+    (dict(layer=1, sink=FAKE), 1),                  # global layers have no sink
+    (dict(layer=7), 1),                             # unknown layer kind
+    (dict(base=0.0), 1),
+    (dict(base=float("nan")), 1),
+    (dict(q=FAKE + 8), 1),                          # misaligned
+    (dict(out=0), 1),                               # null output
+    (dict(dims=dict(num_seqs=0)), 1),
+    (dict(dims=dict(max_seqlen=10 ** 6)), 1),       # max_seqlen > total tokens
+])
+def test_validation_rejects(M, case, expect):
+    d = dict(num_seqs=1, total_tokens=512, max_seqlen=512, hq=4, hkv=1, dqk=192, dv=128)
+    d.update(case.pop("dims", {}))
+    dims = M.make_dims(d["num_seqs"], d["total_tokens"], d["max_seqlen"], d["hq"], d["hkv"], d["dqk"], d["dv"])
+    assert call(M, dims, **case) == expect
+
+
+def test_null_dims_rejected(M):
+    st = M.LIB.mimo_attn_fwd(FAKE, FAKE, FAKE, None, FAKE, None, 0, 128, 1e4, 64, 0.707, FAKE, FAKE, None)
+    assert st == M.ERR_INVALID_ARG
+
+
+def test_host_entry_checks_cu_seqlens_on_host(M):
+    import torch
+    dims = M.make_dims(2, 300, 200, 4, 1)
+    ws_bytes = M.host_workspace_size(dims, True)
+    assert ws_bytes > 300 * 4 * 192 * 2
+    q = torch.zeros(300, 4, 192, dtype=torch.bfloat16)
+    k = torch.zeros(300, 1, 192, dtype=torch.bfloat16)
+    v = torch.zeros(300, 1, 128, dtype=torch.bfloat16)
+    o = torch.zeros(300, 4, 128, dtype=torch.bfloat16)
+    l = torch.zeros(4, 300)
+    s = torch.zeros(4)
+
+    class FakeWs:  # only size and address are read before the cu_seqlens check fails
+        def data_ptr(self):
+            return 1 << 20
+
+        def numel(self):
+            return ws_bytes
+
+        def element_size(self):
+            return 1
+
+    for bad in ([0, 250, 300], [1, 100, 300], [0, 100, 299], [0, 150, 100]):
+        cu = torch.tensor(bad, dtype=torch.int32)
+        with pytest.raises(M.MimoAttnError) as e:
+            M.LIB.mimo_attn_fwd_host  # noqa: B018
+            st = M.LIB.mimo_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), s.data_ptr(), cu.data_ptr(),
+                                          ctypes.byref(dims), 0, 128, 1e4, 64, 0.707, o.data_ptr(), l.data_ptr(),
+                                          FakeWs().data_ptr(), ws_bytes, None)
+            if st != 0:
+                raise M.MimoAttnError(st, "fwd_host")
+        assert e.value.status == M.ERR_INVALID_ARG

@@ -1,0 +1,160 @@
+"""GPU parity: the CUDA path through the C-ABI against the FP64 oracle on the
+same seeded inputs, at sizes the oracle finishes in seconds (element by
+element) and at the full workload sizes (sampled rows), plus edge cases."""
+import numpy as np
+import pytest
+import torch
+
+from global_attention_moe_b200 import workloads as W
+from gpu_helpers import (assert_within, errors, out_to_f64, run_gpu, run_oracle, sample_rows, to_device)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from global_attention_moe_b200 import mimo_attn
+    assert mimo_attn.check() == mimo_attn.OK
+
+
+def full_parity(w):
+    x = W.make_inputs(w)
+    out, lse = run_gpu(w, x)
+    ref_out, ref_lse = run_oracle(w, x)
+    err = errors(out_to_f64(out), lse.cpu().numpy().astype(np.float64), ref_out, ref_lse)
+    assert_within(err, w.name)
+    return err
+
+
+def test_tiny_swa_sink_full():
+    full_parity(W.tiny_swa())
+
+
+@pytest.mark.parametrize("lengths", [[1], [127], [128], [129], [130], [255], [256], [257],
+                                     [1, 127, 128, 129, 130, 255, 256, 257], [0, 300, 0, 5]])
+def test_ragged_lengths_swa(lengths):
+    full_parity(W.custom("ragged", W.LAYER_SWA, lengths, 4, 1, 128, 1e4, True, seed=1))
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 1), (16, 1), (64, 8)])
+def test_gqa_ratios(hq, hkv):
+    full_parity(W.custom("gqa", W.LAYER_SWA, [200, 333], hq, hkv, 128, 1e4, True, seed=2))
+
+
+@pytest.mark.parametrize("window", [0, 1, 5, 127, 128, 129, 200, 300])
+def test_windows(window):
+    full_parity(W.custom("win", W.LAYER_SWA, [700, 61], 4, 2, window, 1e4, False, seed=3))
+
+
+def test_sink_extremes():
+    w = W.custom("sink", W.LAYER_SWA, [400], 8, 2, 128, 1e4, True, seed=4)
+    x = W.make_inputs(w)
+    x.sink = np.array([8, -8, 8, -8, 0, 3, -3, 20], dtype=np.float32)
+    out, lse = run_gpu(w, x)
+    ro, rl = run_oracle(w, x)
+    assert_within(errors(out_to_f64(out), lse.cpu().numpy().astype(np.float64), ro, rl), "sink extremes")
+
+
+@pytest.mark.parametrize("lengths", [[300], [1, 129, 640], [1024]])
+def test_global_small(lengths):
+    full_parity(W.custom("global", W.LAYER_GLOBAL, lengths, 8, 2, -1, 1e7, False, seed=5))
+
+
+@pytest.mark.parametrize("name", ["swa4096", "swa_varlen", "global", "swa_long"])
+def test_full_size_sampled(name):
+    w = W.WORKLOADS[name]()
+    x = W.make_inputs(w)
+    out, lse = run_gpu(w, x)
+    rows = sample_rows(w)
+    ref_out, ref_lse = run_oracle(w, x, rows=rows)
+    rows_t = torch.from_numpy(rows).to(out.device)
+    g_out = out_to_f64(out.index_select(0, rows_t))
+    g_lse = lse.index_select(1, rows_t).cpu().numpy().astype(np.float64)
+    assert_within(errors(g_out, g_lse, ref_out, ref_lse), name)
+    # properties that hold at any size: finite everywhere, lse >= sink, |out| bounded by v_scale*max|v|
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    if x.sink is not None:
+        assert (lse >= torch.from_numpy(x.sink).to(lse.device)[:, None] - 1e-4).all()
+    vmax = float(np.abs(W.synth.bf16_bits_to_f32(x.v)).max())
+    assert float(out.float().abs().max()) <= w.v_scale * vmax * 1.01
+
+
+def test_packed_equals_separate():
+    w = W.custom("pack", W.LAYER_SWA, [130, 1, 257, 64], 8, 2, 128, 1e4, True, seed=6)
+    x = W.make_inputs(w)
+    out, lse = run_gpu(w, x)
+    for b, L in enumerate(w.lengths):
+        s = int(x.cu_seqlens[b])
+        wb = W.custom("one", W.LAYER_SWA, [L], 8, 2, 128, 1e4, True, seed=6)
+        xb = W.Inputs(x.q[s:s + L], x.k[s:s + L], x.v[s:s + L], x.sink, np.array([0, L], dtype=np.int32))
+        ob, lb = run_gpu(wb, xb)
+        assert torch.equal(ob, out[s:s + L]) and torch.equal(lb, lse[:, s:s + L])
+
+
+def test_every_row_written_and_no_overrun():
+    """Outputs live inside larger buffers pre-filled with NaN: every in-range
+    element must be overwritten and every guard element left untouched."""
+    w = W.custom("guard", W.LAYER_SWA, [1, 200, 129], 4, 1, 128, 1e4, True, seed=7)
+    x = W.make_inputs(w)
+    T, G = w.total_tokens, 4096
+    dev = to_device(x)
+    ob = torch.full((T * 4 * 128 + 2 * G,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lb = torch.full((4 * T + 2 * G,), float("nan"), dtype=torch.float32, device="cuda")
+    out = ob[G:G + T * 4 * 128].view(T, 4, 128)
+    lse = lb[G:G + 4 * T].view(4, T)
+    run_gpu(w, x, dev_inputs=dev, out=out, lse=lse)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    assert torch.isnan(ob[:G].float()).all() and torch.isnan(ob[-G:].float()).all()
+    assert torch.isnan(lb[:G]).all() and torch.isnan(lb[-G:]).all()
+
+
+def test_host_entry_matches_device_entry():
+    from global_attention_moe_b200 import mimo_attn
+    w = W.custom("host", W.LAYER_SWA, [300, 77], 8, 2, 128, 1e4, True, seed=8)
+    x = W.make_inputs(w)
+    out, lse = run_gpu(w, x)
+    dims = mimo_attn.make_dims(w.num_seqs, w.total_tokens, w.max_seqlen, 8, 2)
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    qh, kh, vh = (pin(a.view(np.int16)) for a in (x.q, x.k, x.v))
+    sh, ch = pin(x.sink), pin(x.cu_seqlens)
+    oh = torch.empty(w.total_tokens, 8, 128, dtype=torch.int16).pin_memory()
+    lh = torch.empty(8, w.total_tokens, dtype=torch.float32).pin_memory()
+    ws = torch.empty(mimo_attn.host_workspace_size(dims, True), dtype=torch.uint8, device="cuda")
+    mimo_attn.fwd_host(qh, kh, vh, sh, ch, dims, w.layer_kind, w.window, w.rope_base, 64, w.v_scale, oh, lh, ws)
+    assert torch.equal(oh.view(torch.bfloat16), out.cpu()) and torch.equal(lh, lse.cpu())
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    from global_attention_moe_b200 import mimo_attn
+    assert mimo_attn.selftest_wait_timeout(2_000_000) == mimo_attn.ERR_TIMEOUT
+    assert mimo_attn.check() == mimo_attn.OK
+    test_tiny_swa_sink_full()
+
+
+def test_range_error_recorded():
+    from global_attention_moe_b200 import mimo_attn
+    w = W.custom("range", W.LAYER_SWA, [64], 4, 1, 128, 1e4, False, seed=9)
+    x = W.make_inputs(w)
+    q = x.q.copy()
+    q[5, 0, 3] = W.synth.f32_to_bf16_bits(np.array([60000.0], dtype=np.float32))[0]
+    q[5, 0, 35] = W.synth.f32_to_bf16_bits(np.array([60000.0], dtype=np.float32))[0]
+    x.q = q
+    dq, dk, dv, ds, dcu = to_device(x)
+    mimo_attn.fwd(dq, dk, dv, ds, dcu, 64, 0, 128, 1e4)
+    assert mimo_attn.check() == mimo_attn.ERR_RANGE
+
+
+def test_bad_cu_seqlens_detected_without_overrun():
+    from global_attention_moe_b200 import mimo_attn
+    w = W.custom("badcu", W.LAYER_SWA, [100, 100], 4, 1, 128, 1e4, False, seed=10)
+    x = W.make_inputs(w)
+    dq, dk, dv, ds, _ = to_device(x)
+    cu = torch.tensor([0, 150, 260], dtype=torch.int32, device="cuda")  # ends past T = 200
+    G = 4096
+    ob = torch.full((200 * 4 * 128 + 2 * G,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = ob[G:G + 200 * 4 * 128].view(200, 4, 128)
+    mimo_attn.fwd(dq, dk, dv, ds, cu, 200, 0, 128, 1e4, out=out)
+    assert mimo_attn.check() == mimo_attn.ERR_BAD_SEQLENS
+    assert torch.isnan(ob[:G].float()).all() and torch.isnan(ob[-G:].float()).all()
