@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the MiMo-V2 attention forward on B200.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one attention forward (one layer) over one batch of the workload.
+Default workload: the 4096-token sliding-window layer with sink, 64 query /
+8 KV heads (the single-GPU configuration the metric is quoted on).
+
+Our arm: inputs already resident in HBM, rotated over several buffer sets
+whose total footprint exceeds the 126 MB L2, so consecutive steps never hit
+L2 and one CUDA-event pair brackets all K steps (barrier + synchronize on both
+sides, max over ranks).  Under torchrun every rank runs its own batch of the
+same shape (weak scaling; no data-path collective).  Rank 0 prints one JSON
+line.  The reference arm (--impl reference) times the FP64 CPU oracle on
+bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from global_attention_moe_b200 import workloads as W  # noqa: E402
+
+METRIC = "attn fwd tokens/s and TFLOP/s on 1 B200 (SWA-sink and global); % of roofline"
+L2_BYTES = 126 * 2 ** 20
+FLOPS_PER_PAIR = 2 * 192 + 2 * 128
+KERNEL_SOURCES = ["csrc/sm100.cuh", "csrc/rope_smem.cuh", "csrc/params.cuh", "csrc/attn_fwd_simple.cuh",
+                  "csrc/attn_fwd_pipelined.cuh", "csrc/mimo_attn_api.cu"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="swa4096", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-parity", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--ref-budget-s", type=float, default=90.0, help="reference arm: total CPU seconds to aim for")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ accounting
+def bytes_per_step(w: W.Workload) -> int:
+    """Algorithmic bytes: q, k, v read once, out and lse written once."""
+    T = w.total_tokens
+    return T * (2 * w.num_q_heads * w.head_dim_qk + 2 * w.num_kv_heads * w.head_dim_qk
+                + 2 * w.num_kv_heads * w.head_dim_v + 2 * w.num_q_heads * w.head_dim_v + 4 * w.num_q_heads)
+
+
+def flops_per_step(w: W.Workload) -> int:
+    return FLOPS_PER_PAIR * W.attended_pairs(w.lengths, w.window, w.num_q_heads)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "global_attention_moe_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("sources_sha") != kernel_sources_sha():
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:  # NVML missing: clocks reported as unavailable
+            self._ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_oracle_rate(w: W.Workload, x: W.Inputs, target_s: float, max_rows_per_call: int | None = None):
+    """Time the oracle (as it stands) on samples of the workload's rows.
+    Returns (tokens/s, cores, description)."""
+    import oracle
+    cores = oracle.default_threads()
+    rng = np.random.default_rng(0)
+    order = rng.permutation(w.total_tokens)
+    # calibrate on a small sample
+    n = min(w.total_tokens, 64)
+    t0 = time.perf_counter()
+    oracle.attn_fwd(x.q, x.k, x.v, x.sink, x.cu_seqlens, w.window, w.rope_base, w.rope_dims, w.v_scale,
+                    rows=order[:n], threads=cores)
+    t_small = time.perf_counter() - t0
+    per_row = max(t_small / n, 1e-6)
+    rows = int(min(w.total_tokens, max(1, target_s / per_row)))
+    if max_rows_per_call:
+        rows = min(rows, max_rows_per_call)
+    done, elapsed, calls = 0, 0.0, 0
+    while elapsed < target_s and calls < 1000:
+        start = (calls * rows) % w.total_tokens
+        sel = np.take(order, np.arange(start, start + rows), mode="wrap")
+        t0 = time.perf_counter()
+        oracle.attn_fwd(x.q, x.k, x.v, x.sink, x.cu_seqlens, w.window, w.rope_base, w.rope_dims, w.v_scale,
+                        rows=sel, threads=cores)
+        elapsed += time.perf_counter() - t0
+        done += rows
+        calls += 1
+        if rows == w.total_tokens and elapsed >= 0.5 * target_s:
+            break
+    desc = (f"{calls} oracle call(s) of {rows} seeded-random token rows (all {w.num_q_heads} heads each) of "
+            f"{w.name}; {elapsed:.1f} s of CPU time")
+    return done / elapsed, cores, desc
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    w = W.WORKLOADS[args.workload]()
+    x = W.make_inputs(w)
+    import oracle
+    cores = oracle.default_threads()
+    rng = np.random.default_rng(0)
+    order = rng.permutation(w.total_tokens)
+    n = min(w.total_tokens, 32)
+    t0 = time.perf_counter()
+    oracle.attn_fwd(x.q, x.k, x.v, x.sink, x.cu_seqlens, w.window, w.rope_base, w.rope_dims, w.v_scale,
+                    rows=order[:n], threads=cores)
+    per_call_fixed_and_rows = time.perf_counter() - t0
+    per_row = per_call_fixed_and_rows / n
+    total_steps = max(1, args.steps + args.warmup)
+    rows = int(max(1, min(w.total_tokens, args.ref_budget_s / total_steps / max(per_row, 1e-6))))
+
+    def step(i):
+        start = (i * rows) % w.total_tokens
+        sel = np.take(order, np.arange(start, start + rows), mode="wrap")
+        oracle.attn_fwd(x.q, x.k, x.v, x.sink, x.cu_seqlens, w.window, w.rope_base, w.rope_dims, w.v_scale,
+                        rows=sel, threads=cores)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    el = time.perf_counter() - t0
+    value = args.steps * rows / el
+    sample = (f"each step: {rows} seeded-random token rows (all {w.num_q_heads} heads) of {w.name}, "
+              f"FP64 C oracle on {cores} host threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**w.describe(), "rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from global_attention_moe_b200 import mimo_attn
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and rank == 0:
+        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    w = W.WORKLOADS[args.workload](seed=0)
+    w.seed = rank  # weak scaling: every rank draws its own batch of the same shape
+    x = W.make_inputs(w)
+    T = w.total_tokens
+    stream = torch.cuda.current_stream()
+    sh = ctypes.c_void_p(stream.cuda_stream)
+
+    def dev_set():
+        q = torch.from_numpy(x.q.view(np.int16)).to(dev).view(torch.bfloat16)
+        k = torch.from_numpy(x.k.view(np.int16)).to(dev).view(torch.bfloat16)
+        v = torch.from_numpy(x.v.view(np.int16)).to(dev).view(torch.bfloat16)
+        s = None if x.sink is None else torch.from_numpy(x.sink).to(dev)
+        cu = torch.from_numpy(x.cu_seqlens).to(dev)
+        out = torch.empty(T, w.num_q_heads, w.head_dim_v, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(w.num_q_heads, T, dtype=torch.float32, device=dev)
+        return q, k, v, s, cu, out, lse
+
+    set_bytes = bytes_per_step(w)
+    n_sets = max(2, -(-3 * L2_BYTES // set_bytes))
+    sets = [dev_set() for _ in range(n_sets)]
+    dims = mimo_attn.make_dims(w.num_seqs, T, w.max_seqlen, w.num_q_heads, w.num_kv_heads)
+    calls = [(q.data_ptr(), k.data_ptr(), v.data_ptr(), s.data_ptr() if s is not None else None, cu.data_ptr(),
+              out.data_ptr(), lse.data_ptr()) for (q, k, v, s, cu, out, lse) in sets]
+    fn = mimo_attn.LIB.mimo_attn_fwd
+    dref = ctypes.byref(dims)
+    lk, win, base, rd, vs = w.layer_kind, w.window, w.rope_base, w.rope_dims, w.v_scale
+
+    def step(i):
+        a = calls[i % n_sets]
+        st = fn(a[0], a[1], a[2], a[3], a[4], dref, lk, win, base, rd, vs, a[5], a[6], sh)
+        if st != 0:
+            raise mimo_attn.MimoAttnError(st, "mimo_attn_fwd")
+
+    for i in range(max(args.warmup, 0)):
+        step(i)
+    st = mimo_attn.check()
+    if st != mimo_attn.OK:
+        raise mimo_attn.MimoAttnError(st, "warm-up")
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    st = mimo_attn.check()
+    if st != mimo_attn.OK:
+        raise mimo_attn.MimoAttnError(st, "timed region")
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / max(args.steps, 1)
+    value = world * T * args.steps / (ms / 1e3)
+
+    # --- end to end through the host-buffer C-ABI entry (pinned host memory, copies inside the region)
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(a).pin_memory()
+        qh, kh, vh = (pin(a.view(np.int16)) for a in (x.q, x.k, x.v))
+        shh = pin(x.sink) if x.sink is not None else None
+        ch = pin(x.cu_seqlens)
+        oh = torch.empty(T, w.num_q_heads, w.head_dim_v, dtype=torch.int16).pin_memory()
+        lh = torch.empty(w.num_q_heads, T, dtype=torch.float32).pin_memory()
+        ws = torch.empty(mimo_attn.host_workspace_size(dims, x.sink is not None), dtype=torch.uint8, device=dev)
+        h2d = sum(a.numel() * a.element_size() for a in (qh, kh, vh, ch) + ((shh,) if shh is not None else ()))
+        d2h = oh.numel() * 2 + lh.numel() * 4
+        for _ in range(2):
+            mimo_attn.fwd_host(qh, kh, vh, shh, ch, dims, lk, win, base, rd, vs, oh, lh, ws)
+        ne = max(1, min(args.e2e_steps, args.steps))
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(ne):
+            mimo_attn.fwd_host(qh, kh, vh, shh, ch, dims, lk, win, base, rd, vs, oh, lh, ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * T * ne / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": ne}
+
+    # --- parity spot check of this run's output against the oracle (rank 0)
+    parity = None
+    if rank == 0 and not args.no_parity:
+        import oracle
+        q, k, v, s, cu, out, lse = sets[(args.steps - 1) % n_sets]
+        rng = np.random.default_rng(1)
+        rows = np.unique(np.concatenate([[0, T - 1, min(T - 1, 128)], rng.integers(0, T, 24)])).astype(np.int64)
+        ro, rl = oracle.attn_fwd(x.q, x.k, x.v, x.sink, x.cu_seqlens, w.window, w.rope_base, w.rope_dims, w.v_scale,
+                                 rows=rows)
+        idx = torch.from_numpy(rows).to(dev)
+        go = out.index_select(0, idx).float().cpu().numpy().astype(np.float64)
+        gl = lse.index_select(1, idx).cpu().numpy().astype(np.float64)
+        d = go - ro
+        parity = {"rows": int(len(rows)), "max_abs": float(np.abs(d).max()),
+                  "rel_l2": float(np.linalg.norm(d) / np.linalg.norm(ro)), "lse_max_abs": float(np.abs(gl - rl).max())}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, desc = cpu_oracle_rate(w, x, target_s=12.0)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    flops = flops_per_step(w)
+    nbytes = bytes_per_step(w)
+    t_s = ms_per_step / 1e3
+    tflops = flops / t_s / 1e12
+    gbs = nbytes / t_s / 1e9
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    long_region = ms > 1000.0
+    tc_peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
+    t_tc = flops / (tc_peak * 1e12)
+    kernel = "attn_fwd_pipelined_kernel" if (w.num_q_heads // w.num_kv_heads) % 2 == 0 else "attn_fwd_simple_kernel"
+    traffic = recorded_traffic(kernel, w.name)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": tflops, "peak": tc_peak, "unit": "TFLOP/s", "frac": tflops / tc_peak}
+    roof.update({"traffic": traffic, "peak_source": f"{peak_src} ({'sustained' if long_region and roof['bound'] == 'tensor' else 'burst'})",
+                 "kernel": kernel, "algorithmic_bytes": nbytes, "algorithmic_flops": flops})
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**w.describe(), "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"inputs rotated over {n_sets} device buffer sets ({n_sets * set_bytes / 2**20:.0f} MiB > 126 MiB L2), no flush"},
+        "tflops": tflops, "gbs": gbs, "roofline_time_us": max(t_hbm, t_tc) * 1e6,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "parity": parity,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -5,12 +5,15 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/mimo_attn.h"
+#include "attn_fwd_pipelined.cuh"
 #include "attn_fwd_simple.cuh"
 #include "params.cuh"
 
@@ -33,13 +36,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensormap_encoder() {
   return fn;
 }
 
-// 2-D bf16 view [rows, inner] (row-major) with a {64, 128} box and 128-byte swizzle.
-bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+// 2-D bf16 view [rows, inner] (row-major) with a {64, box_rows} box and 128-byte swizzle.
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows = 128) {
   auto enc = tensormap_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -97,24 +100,55 @@ void fill_params(FwdParams& P, const float* sink, const int32_t* cu, const mimo_
   for (int i = 0; i < kRopeDims / 2; ++i) P.theta[i] = std::pow(rope_base, -2.0 * i / kRopeDims);
 }
 
-int launch_simple(const void* q, const void* k, const void* v, const FwdParams& P, cudaStream_t stream) {
+std::atomic<int> g_kernel_choice{MIMO_KERNEL_AUTO};
+
+struct DeviceInfo {
+  int sms = 0;
+  bool simple_ready = false;
+  bool pipelined_ready = false;
+};
+
+DeviceInfo* device_info(int dev) {
+  static DeviceInfo infos[64];
+  static std::mutex mu;
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceInfo& d = infos[dev];
+  if (d.sms == 0) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+    d.simple_ready = cudaFuncSetAttribute(attn_fwd_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          simple::kSmemBytes) == cudaSuccess;
+    d.pipelined_ready = cudaFuncSetAttribute(attn_fwd_pipelined_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             pipe::kSmemBytes) == cudaSuccess;
+  }
+  return &d;
+}
+
+int launch(const void* q, const void* k, const void* v, const FwdParams& P, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
+  DeviceInfo* info = device_info(dev);
+  if (!info) return MIMO_ERR_CUDA;
+  if (P.max_seqlen == 0) return MIMO_OK;
+  const int choice = g_kernel_choice.load();
+  const bool pipelined = (choice == MIMO_KERNEL_PIPELINED) || (choice == MIMO_KERNEL_AUTO && P.group % 2 == 0);
+  if (pipelined && P.group % 2 != 0) return MIMO_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv;
   if (!encode_2d(&tq, q, (uint64_t)P.hq * kHeadDimQK, P.total_tokens) ||
       !encode_2d(&tk, k, (uint64_t)P.hkv * kHeadDimQK, P.total_tokens) ||
-      !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, P.total_tokens))
+      !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, P.total_tokens, pipelined ? 64 : 128))
     return MIMO_ERR_CUDA;
-  static thread_local int configured_device = -1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
-  if (configured_device != dev) {
-    if (cudaFuncSetAttribute(attn_fwd_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             simple::kSmemBytes) != cudaSuccess)
-      return MIMO_ERR_CUDA;
-    configured_device = dev;
+  if (pipelined) {
+    if (!info->pipelined_ready) return MIMO_ERR_CUDA;
+    const long long units = (long long)(P.hq / 2) * ((P.total_tokens + kBlockM - 1) / kBlockM + P.num_seqs);
+    const int grid = (int)std::min<long long>(units, info->sms);
+    attn_fwd_pipelined_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tk, tv, P);
+  } else {
+    if (!info->simple_ready) return MIMO_ERR_CUDA;
+    dim3 grid((P.max_seqlen + kBlockM - 1) / kBlockM, P.num_seqs, P.hq);
+    attn_fwd_simple_kernel<<<grid, simple::kThreads, simple::kSmemBytes, stream>>>(tq, tk, tv, P);
   }
-  if (P.max_seqlen == 0) return MIMO_OK;
-  dim3 grid((P.max_seqlen + kBlockM - 1) / kBlockM, P.num_seqs, P.hq);
-  attn_fwd_simple_kernel<<<grid, simple::kThreads, simple::kSmemBytes, stream>>>(tq, tk, tv, P);
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 
@@ -144,7 +178,7 @@ int mimo_attn_fwd(const void* q, const void* k, const void* v, const float* sink
   if (dims->total_tokens == 0) return MIMO_OK;
   FwdParams P;
   fill_params(P, sink, cu_seqlens, dims, layer_kind, window, rope_base, v_scale, out, lse);
-  return launch_simple(q, k, v, P, static_cast<cudaStream_t>(stream));
+  return launch(q, k, v, P, static_cast<cudaStream_t>(stream));
 }
 
 size_t mimo_attn_host_workspace_size(const mimo_attn_dims* d, int has_sink) {
@@ -250,6 +284,13 @@ const char* mimo_attn_status_string(int status) {
   }
 }
 
-int mimo_attn_version(void) { return (1 << 16) | 0; }
+int mimo_attn_version(void) { return (1 << 16) | 1; }
+
+int mimo_attn_set_kernel(int choice) {
+  if (choice != MIMO_KERNEL_AUTO && choice != MIMO_KERNEL_SIMPLE && choice != MIMO_KERNEL_PIPELINED)
+    return MIMO_ERR_INVALID_ARG;
+  g_kernel_choice.store(choice);
+  return MIMO_OK;
+}
 
 }  // extern "C"

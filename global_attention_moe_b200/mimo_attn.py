@@ -19,7 +19,9 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BAD_
 
 # Every symbol include/mimo_attn.h declares.
 SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host", "mimo_attn_check",
-           "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_version")
+           "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_set_kernel",
+           "mimo_attn_version")
+KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED = 0, 1, 2
 
 
 class Dims(ctypes.Structure):
@@ -52,6 +54,8 @@ def _load():
     lib.mimo_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
     lib.mimo_attn_status_string.restype = ctypes.c_char_p
     lib.mimo_attn_status_string.argtypes = [I]
+    lib.mimo_attn_set_kernel.restype = I
+    lib.mimo_attn_set_kernel.argtypes = [I]
     lib.mimo_attn_version.restype = I
     lib.mimo_attn_version.argtypes = []
     return lib
@@ -67,6 +71,13 @@ def status_string(status: int) -> str:
 def version() -> tuple[int, int]:
     v = LIB.mimo_attn_version()
     return v >> 16, v & 0xFFFF
+
+
+def set_kernel(choice: int) -> None:
+    """Select the kernel mimo_attn_fwd launches (KERNEL_AUTO / KERNEL_SIMPLE / KERNEL_PIPELINED)."""
+    st = LIB.mimo_attn_set_kernel(int(choice))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_attn_set_kernel")
 
 
 def make_dims(num_seqs, total_tokens, max_seqlen, hq, hkv, dqk=192, dv=128) -> Dims:

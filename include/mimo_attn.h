@@ -151,6 +151,18 @@ MIMO_API int mimo_attn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 /* Static description of a status code (never NULL). */
 MIMO_API const char* mimo_attn_status_string(int status);
 
+/* Kernel selection for mimo_attn_fwd (process-wide; default AUTO).
+ *   MIMO_KERNEL_AUTO       pipelined kernel when Hq/Hkv is even, else the simple one
+ *   MIMO_KERNEL_SIMPLE     one CTA per (128-query tile, head), every step serialised;
+ *                          any Hq/Hkv ratio (the cross-check path)
+ *   MIMO_KERNEL_PIPELINED  warp-specialised persistent kernel, two heads per CTA;
+ *                          Hq/Hkv must be even (else mimo_attn_fwd returns
+ *                          MIMO_ERR_UNSUPPORTED)
+ * Returns MIMO_ERR_INVALID_ARG for any other value.  Both kernels compute the
+ * same operation with the same rounding steps. */
+typedef enum { MIMO_KERNEL_AUTO = 0, MIMO_KERNEL_SIMPLE = 1, MIMO_KERNEL_PIPELINED = 2 } mimo_kernel_choice;
+MIMO_API int mimo_attn_set_kernel(int choice);
+
 /* ABI version: (major << 16) | minor. */
 MIMO_API int mimo_attn_version(void);
 

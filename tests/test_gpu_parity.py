@@ -19,6 +19,15 @@ def _cuda():
     assert mimo_attn.check() == mimo_attn.OK
 
 
+@pytest.fixture(params=["auto", "simple"])
+def kernel(request):
+    """Run a test with the default kernel choice and again with the serialised cross-check kernel."""
+    from global_attention_moe_b200 import mimo_attn
+    mimo_attn.set_kernel(mimo_attn.KERNEL_SIMPLE if request.param == "simple" else mimo_attn.KERNEL_AUTO)
+    yield request.param
+    mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
+
+
 def full_parity(w):
     x = W.make_inputs(w)
     out, lse = run_gpu(w, x)
@@ -28,27 +37,27 @@ def full_parity(w):
     return err
 
 
-def test_tiny_swa_sink_full():
+def test_tiny_swa_sink_full(kernel):
     full_parity(W.tiny_swa())
 
 
 @pytest.mark.parametrize("lengths", [[1], [127], [128], [129], [130], [255], [256], [257],
                                      [1, 127, 128, 129, 130, 255, 256, 257], [0, 300, 0, 5]])
-def test_ragged_lengths_swa(lengths):
+def test_ragged_lengths_swa(lengths, kernel):
     full_parity(W.custom("ragged", W.LAYER_SWA, lengths, 4, 1, 128, 1e4, True, seed=1))
 
 
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 1), (16, 1), (64, 8)])
-def test_gqa_ratios(hq, hkv):
+def test_gqa_ratios(hq, hkv, kernel):
     full_parity(W.custom("gqa", W.LAYER_SWA, [200, 333], hq, hkv, 128, 1e4, True, seed=2))
 
 
 @pytest.mark.parametrize("window", [0, 1, 5, 127, 128, 129, 200, 300])
-def test_windows(window):
+def test_windows(window, kernel):
     full_parity(W.custom("win", W.LAYER_SWA, [700, 61], 4, 2, window, 1e4, False, seed=3))
 
 
-def test_sink_extremes():
+def test_sink_extremes(kernel):
     w = W.custom("sink", W.LAYER_SWA, [400], 8, 2, 128, 1e4, True, seed=4)
     x = W.make_inputs(w)
     x.sink = np.array([8, -8, 8, -8, 0, 3, -3, 20], dtype=np.float32)
@@ -58,7 +67,7 @@ def test_sink_extremes():
 
 
 @pytest.mark.parametrize("lengths", [[300], [1, 129, 640], [1024]])
-def test_global_small(lengths):
+def test_global_small(lengths, kernel):
     full_parity(W.custom("global", W.LAYER_GLOBAL, lengths, 8, 2, -1, 1e7, False, seed=5))
 
 
@@ -81,7 +90,7 @@ def test_full_size_sampled(name):
     assert float(out.float().abs().max()) <= w.v_scale * vmax * 1.01
 
 
-def test_packed_equals_separate():
+def test_packed_equals_separate(kernel):
     w = W.custom("pack", W.LAYER_SWA, [130, 1, 257, 64], 8, 2, 128, 1e4, True, seed=6)
     x = W.make_inputs(w)
     out, lse = run_gpu(w, x)
@@ -93,7 +102,7 @@ def test_packed_equals_separate():
         assert torch.equal(ob, out[s:s + L]) and torch.equal(lb, lse[:, s:s + L])
 
 
-def test_every_row_written_and_no_overrun():
+def test_every_row_written_and_no_overrun(kernel):
     """Outputs live inside larger buffers pre-filled with NaN: every in-range
     element must be overwritten and every guard element left untouched."""
     w = W.custom("guard", W.LAYER_SWA, [1, 200, 129], 4, 1, 128, 1e4, True, seed=7)
@@ -130,7 +139,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     from global_attention_moe_b200 import mimo_attn
     assert mimo_attn.selftest_wait_timeout(2_000_000) == mimo_attn.ERR_TIMEOUT
     assert mimo_attn.check() == mimo_attn.OK
-    test_tiny_swa_sink_full()
+    full_parity(W.tiny_swa())
 
 
 def test_range_error_recorded():
@@ -158,3 +167,20 @@ def test_bad_cu_seqlens_detected_without_overrun():
     mimo_attn.fwd(dq, dk, dv, ds, cu, 200, 0, 128, 1e4, out=out)
     assert mimo_attn.check() == mimo_attn.ERR_BAD_SEQLENS
     assert torch.isnan(ob[:G].float()).all() and torch.isnan(ob[-G:].float()).all()
+
+
+def test_kernels_agree_closely():
+    """The pipelined and the serialised kernel take the same rounding steps; on the
+    same inputs their outputs agree to a few BF16 ulps (summation order differs)."""
+    from global_attention_moe_b200 import mimo_attn
+    w = W.custom("agree", W.LAYER_GLOBAL, [700, 129], 8, 2, -1, 1e7, False, seed=11)
+    x = W.make_inputs(w)
+    dev = to_device(x)
+    mimo_attn.set_kernel(mimo_attn.KERNEL_SIMPLE)
+    try:
+        o1, l1 = run_gpu(w, x, dev_inputs=dev)
+    finally:
+        mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
+    o2, l2 = run_gpu(w, x, dev_inputs=dev)
+    assert float((o1.float() - o2.float()).abs().max()) < 1e-2
+    assert float((l1 - l2).abs().max()) < 2e-4
