@@ -12,8 +12,8 @@
 //   Q region : 6 units = 2 heads x {dims 0..63 (rotated, FP16), 64..127, 128..191}
 //              each unit = 128 query rows x 64 dims
 //   K/V ring : 8 unit slots; every KV tile is 5 units, in this order:
-//              K dims 0..63 (rotated in place to FP16), K dims 64..127,
-//              K dims 128..191 (128 keys x 64 dims each), then
+//              K dims 0..63 (already rotated, FP16, from the RoPE pre-pass),
+//              K dims 64..127, K dims 128..191 (128 keys x 64 dims each), then
 //              V keys 0..63 and V keys 64..127 (64 keys x 128 dims each, stored
 //              as two 8 KB halves: dims 0..63 then 64..127).
 //   The ring is consumed and released in load order, so with 8 slots every
@@ -22,19 +22,22 @@
 // overwrites the first 64 columns of S_h and is the A operand of PV.
 //
 // Warp roles (16 warps, 512 threads):
-//   warp 0      Q loader (TMA)
+//   warp 0      Q loader (TMA), per head as soon as that head's Q region frees
 //   warp 1      MMA issuer (one thread) and TMEM owner
 //   warp 2      K/V loader (TMA); runs ahead across units, bounded by the ring
 //   warp 3      idle
 //   warps 4-7   softmax + epilogue for the unit's first head (thread = query row = TMEM lane)
 //   warps 8-11  softmax + epilogue for the second head
-//   warps 12-15 RoPE: rotates the rope unit of Q (per unit) and of every K tile
-//               in place, BF16 in, FP16 out.  Each thread owns one row; its
-//               per-row angle offsets r*theta_i live in registers, the tile-start
-//               angle is evaluated once per frequency per tile.
+//   warps 12-15 RoPE for Q: rotates each head's rope unit in place, BF16 in,
+//               FP16 out.  Each thread owns one row; its per-row angle offsets
+//               r*theta_i live in registers, the tile-start angle is evaluated
+//               once per frequency per unit.
 //
-// MMA issue order per unit:
-//   S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ... | PV0(last) PV1(last)
+// MMA issue order: one stream over all tiles of all units of the CTA,
+//   S0(0) S1(0) | PV0(t) S0(t+1) PV1(t) S1(t+1) | ...
+// where tile t+1 may be the first tile of the next unit; a head's Q region is
+// released after its last S of a unit, so the next unit's Q loads and rotates
+// while the current unit's softmax and PV finish.
 #pragma once
 
 #include "params.cuh"
@@ -51,8 +54,8 @@ constexpr int kUnitsPerTile = 5;
 constexpr uint32_t kQOff = 0;
 constexpr uint32_t kRingOff = 6 * kUnit;
 constexpr uint32_t kCtrlOff = kRingOff + kSlots * kUnit;  // 229376
-constexpr uint32_t kCtrlBytes = 1024;
-constexpr uint32_t kSmemBytes = kCtrlOff + kCtrlBytes;  // 230400 <= 232448
+constexpr uint32_t kCtrlBytes = 2048;
+constexpr uint32_t kSmemBytes = kCtrlOff + kCtrlBytes;  // 231424 <= 232448
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int h) { return 128u * h; }        // S_h: columns [128h, 128h+128)
 __host__ __device__ constexpr uint32_t col_o(int h) { return 256u + 128u * h; }  // O_h: columns [256+128h, ...)
@@ -76,14 +79,16 @@ constexpr uint32_t kRopeBarId = 1;
 constexpr uint32_t kRegsCtl = MIMO_REGS_CTL, kRegsSoftmax = MIMO_REGS_SOFTMAX, kRegsRope = MIMO_REGS_ROPE;
 static_assert(128 * kRegsCtl + 256 * kRegsSoftmax + 128 * kRegsRope <= 65536, "register split exceeds the launch");
 
+constexpr int kMaxStagedSinks = 256;
 struct Ctrl {
-  uint64_t q_full, q_roped, q_empty;
-  uint64_t slot_full[kSlots], slot_empty[kSlots], slot_ready[kSlots];
+  uint64_t q_full[2], q_roped[2], q_empty[2];
+  uint64_t slot_full[kSlots], slot_empty[kSlots];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint32_t tmem_base;
   int abort;
+  double theta[kRopeDims / 2];
   float2 base_q[kRopeDims / 2];
-  float2 base_k[kRopeDims / 2];
+  float sink[kMaxStagedSinks];  // sink logits staged once per CTA (when hq <= kMaxStagedSinks)
 };
 static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
 }  // namespace pipe
@@ -153,9 +158,7 @@ __device__ __forceinline__ void kv_range(const FwdParams& P, int q0, int& kt_lo,
 __device__ __forceinline__ bool pwait_slow(pipe::Ctrl* C, uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kWaitSliceNs)) return true;
     if (*reinterpret_cast<volatile int*>(&C->abort)) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *reinterpret_cast<volatile int*>(&C->abort) = 1;
@@ -240,12 +243,11 @@ namespace pipe {
 __device__ __forceinline__ uint32_t kslot(uint32_t t, int i) { return (t * kUnitsPerTile + i) % kSlots; }
 __device__ __forceinline__ uint32_t kphase(uint32_t t, int i) { return ((t * kUnitsPerTile + i) / kSlots) & 1; }
 
-// Waits until tile t's three K units are usable (rope unit rotated, pass units landed).
+// Waits until tile t's three K units have landed.
 __device__ __forceinline__ bool wait_k(Ctrl* C, uint32_t t, uint64_t lim) {
-  // the rope unit of tile t sits in slot 5t mod 8, which every slot takes once per 8 tiles
-  if (!pwait(C, &C->slot_ready[kslot(t, 0)], (t / kSlots) & 1, lim)) return false;
-  if (!pwait(C, &C->slot_full[kslot(t, 1)], kphase(t, 1), lim)) return false;
-  if (!pwait(C, &C->slot_full[kslot(t, 2)], kphase(t, 2), lim)) return false;
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+    if (!pwait(C, &C->slot_full[kslot(t, i)], kphase(t, i), lim)) return false;
   tc_fence_after_sync();
   return true;
 }
@@ -263,24 +265,32 @@ __device__ __forceinline__ void mma_pv(uint32_t tmem, uint32_t rdesc_v, uint32_t
   issue_pv_half(tmem + col_o(h), tmem + col_s(h) + 32, rdesc_v + kslot(t, 4) * kStep, false);
 }
 
+__device__ __forceinline__ int unit_tiles(const FwdParams& P, int q0) {
+  int kt_lo, kt_hi;
+  kv_range(P, q0, kt_lo, kt_hi);
+  return kt_hi - kt_lo + 1;
+}
+
 __device__ void role_q_loader(uint8_t* smem, Ctrl* C, const CUtensorMap* tm_q, const FwdParams& P) {
   UnitWalker W(P);
   int q0, h0;
   uint32_t n_u = 0;
   for (long long u = blockIdx.x; W.unit(u, q0, h0); u += gridDim.x, ++n_u) {
-    if (n_u > 0 && !pwait(C, &C->q_empty, (n_u - 1) & 1, P.wait_limit_ns)) return;
-    mbar_arrive_expect_tx(&C->q_full, 6 * kUnit);
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      if (n_u > 0 && !pwait(C, &C->q_empty[h], (n_u - 1) & 1, P.wait_limit_ns)) return;
+      mbar_arrive_expect_tx(&C->q_full[h], 3 * kUnit);
 #pragma unroll
       for (int c = 0; c < 3; ++c)
-        tma_load_2d(smem + kQOff + (3 * h + c) * kUnit, tm_q, &C->q_full, (h0 + h) * kHeadDimQK + 64 * c, W.s_b + q0);
+        tma_load_2d(smem + kQOff + (3 * h + c) * kUnit, tm_q, &C->q_full[h], (h0 + h) * kHeadDimQK + 64 * c,
+                    W.s_b + q0);
+    }
   }
   if (W.bad) atomicOr(&g_mimo_error, kErrSeqlens);
 }
 
-__device__ void role_kv_loader(uint8_t* smem, Ctrl* C, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                               const FwdParams& P) {
+__device__ void role_kv_loader(uint8_t* smem, Ctrl* C, const CUtensorMap* tm_kr, const CUtensorMap* tm_k,
+                               const CUtensorMap* tm_v, const FwdParams& P) {
   UnitWalker W(P);
   int q0, h0;
   uint32_t n = 0;
@@ -296,7 +306,9 @@ __device__ void role_kv_loader(uint8_t* smem, Ctrl* C, const CUtensorMap* tm_k, 
         if (n >= kSlots && !pwait(C, &C->slot_empty[slot], ((n / kSlots) - 1) & 1, P.wait_limit_ns)) return;
         uint8_t* dst = smem + kRingOff + slot * kUnit;
         mbar_arrive_expect_tx(&C->slot_full[slot], kUnit);
-        if (i < 3) {
+        if (i == 0) {
+          tma_load_2d(dst, tm_kr, &C->slot_full[slot], g * kRopeDims, row);  // rotated FP16 rope dims
+        } else if (i < 3) {
           tma_load_2d(dst, tm_k, &C->slot_full[slot], g * kHeadDimQK + 64 * i, row);
         } else {
           const int r0 = row + 64 * (i - 3);
@@ -315,55 +327,81 @@ __device__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, const FwdParams&
   const uint32_t rdesc_v = sdesc_lo(smem_u32(smem + kRingOff), kUnit / 2);
   UnitWalker W(P);
   int q0, h0;
-  uint32_t n_u = 0, n_t = 0;
-  for (long long u = blockIdx.x; W.unit(u, q0, h0); u += gridDim.x, ++n_u) {
-    int kt_lo, kt_hi;
-    kv_range(P, q0, kt_lo, kt_hi);
-    const int ntile = kt_hi - kt_lo + 1;
-    if (!pwait(C, &C->q_roped, n_u & 1, lim)) return;
-    if (!wait_k(C, n_t, lim)) return;
-    mma_s(tmem, qdesc, rdesc_k, n_t, 0);
-    tc_commit(&C->s_full[0]);
-    mma_s(tmem, qdesc, rdesc_k, n_t, 1);
-    tc_commit(&C->s_full[1]);
-    tc_commit(&C->slot_empty[kslot(n_t, 0)]);
-    tc_commit(&C->slot_empty[kslot(n_t, 1)]);
-    tc_commit(&C->slot_empty[kslot(n_t, 2)]);
-    if (ntile == 1) tc_commit(&C->q_empty);
-    for (int j = 0; j < ntile; ++j) {
-      const uint32_t t = n_t + j;
-      const bool last = (j == ntile - 1);
-      if (!pwait(C, &C->slot_full[kslot(t, 3)], kphase(t, 3), lim)) return;
-      if (!pwait(C, &C->slot_full[kslot(t, 4)], kphase(t, 4), lim)) return;
-      // head 0: PV(t), then S(t+1)
-      if (!pwait(C, &C->p_full[0], t & 1, lim)) return;
-      if (j == 0 && n_u > 0 && !pwait(C, &C->o_empty[0], (n_u - 1) & 1, lim)) return;
-      tc_fence_after_sync();
-      mma_pv(tmem, rdesc_v, t, 0, j == 0);
-      if (last) tc_commit(&C->o_full[0]);
-      if (!last) {
-        if (!wait_k(C, t + 1, lim)) return;
-        mma_s(tmem, qdesc, rdesc_k, t + 1, 0);
-        tc_commit(&C->s_full[0]);
-      }
-      // head 1: PV(t), then S(t+1)
-      if (!pwait(C, &C->p_full[1], t & 1, lim)) return;
-      if (j == 0 && n_u > 0 && !pwait(C, &C->o_empty[1], (n_u - 1) & 1, lim)) return;
-      tc_fence_after_sync();
-      mma_pv(tmem, rdesc_v, t, 1, j == 0);
-      tc_commit(&C->slot_empty[kslot(t, 3)]);
-      tc_commit(&C->slot_empty[kslot(t, 4)]);
-      if (last) tc_commit(&C->o_full[1]);
-      if (!last) {
-        mma_s(tmem, qdesc, rdesc_k, t + 1, 1);
-        tc_commit(&C->s_full[1]);
-        tc_commit(&C->slot_empty[kslot(t + 1, 0)]);
-        tc_commit(&C->slot_empty[kslot(t + 1, 1)]);
-        tc_commit(&C->slot_empty[kslot(t + 1, 2)]);
-        if (j + 1 == ntile - 1) tc_commit(&C->q_empty);
+  long long u = blockIdx.x;
+  if (!W.unit(u, q0, h0)) return;
+  int ntile = unit_tiles(P, q0);
+  uint32_t n_u = 0, t = 0;
+  int j = 0;
+  // S of the very first tile
+  if (!pwait(C, &C->q_roped[0], 0, lim) || !wait_k(C, 0, lim)) return;
+  mma_s(tmem, qdesc, rdesc_k, 0, 0);
+  tc_commit(&C->s_full[0]);
+  if (ntile == 1) tc_commit(&C->q_empty[0]);
+  if (!pwait(C, &C->q_roped[1], 0, lim)) return;
+  tc_fence_after_sync();
+  mma_s(tmem, qdesc, rdesc_k, 0, 1);
+  tc_commit(&C->s_full[1]);
+#pragma unroll
+  for (int i = 0; i < 3; ++i) tc_commit(&C->slot_empty[kslot(0, i)]);
+  if (ntile == 1) tc_commit(&C->q_empty[1]);
+  while (true) {
+    // the tile after t: the next one of this unit, or the first one of the next unit
+    bool has_next, next_first = false, next_last = false;
+    int next_ntile = ntile;
+    if (j + 1 < ntile) {
+      has_next = true;
+      next_last = (j + 1 == ntile - 1);
+    } else {
+      int nq0, nh0;
+      has_next = W.unit(u + gridDim.x, nq0, nh0);
+      if (has_next) {
+        next_ntile = unit_tiles(P, nq0);
+        next_first = true;
+        next_last = (next_ntile == 1);
       }
     }
-    n_t += ntile;
+    const uint32_t next_nu = next_first ? n_u + 1 : n_u;
+    const bool first = (j == 0), last = (j == ntile - 1);
+    if (!pwait(C, &C->slot_full[kslot(t, 3)], kphase(t, 3), lim)) return;
+    if (!pwait(C, &C->slot_full[kslot(t, 4)], kphase(t, 4), lim)) return;
+    // head 0: PV(t), then S(t+1)
+    if (!pwait(C, &C->p_full[0], t & 1, lim)) return;
+    if (first && n_u > 0 && !pwait(C, &C->o_empty[0], (n_u - 1) & 1, lim)) return;
+    tc_fence_after_sync();
+    mma_pv(tmem, rdesc_v, t, 0, first);
+    if (last) tc_commit(&C->o_full[0]);
+    if (has_next) {
+      if (next_first && !pwait(C, &C->q_roped[0], next_nu & 1, lim)) return;
+      if (!wait_k(C, t + 1, lim)) return;
+      mma_s(tmem, qdesc, rdesc_k, t + 1, 0);
+      tc_commit(&C->s_full[0]);
+      if (next_last) tc_commit(&C->q_empty[0]);
+    }
+    // head 1: PV(t), then S(t+1)
+    if (!pwait(C, &C->p_full[1], t & 1, lim)) return;
+    if (first && n_u > 0 && !pwait(C, &C->o_empty[1], (n_u - 1) & 1, lim)) return;
+    tc_fence_after_sync();
+    mma_pv(tmem, rdesc_v, t, 1, first);
+    tc_commit(&C->slot_empty[kslot(t, 3)]);
+    tc_commit(&C->slot_empty[kslot(t, 4)]);
+    if (last) tc_commit(&C->o_full[1]);
+    if (!has_next) break;
+    if (next_first && !pwait(C, &C->q_roped[1], next_nu & 1, lim)) return;
+    tc_fence_after_sync();
+    mma_s(tmem, qdesc, rdesc_k, t + 1, 1);
+    tc_commit(&C->s_full[1]);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) tc_commit(&C->slot_empty[kslot(t + 1, i)]);
+    if (next_last) tc_commit(&C->q_empty[1]);
+    ++t;
+    if (next_first) {
+      u += gridDim.x;
+      ++n_u;
+      ntile = next_ntile;
+      j = 0;
+    } else {
+      ++j;
+    }
   }
 }
 
@@ -383,7 +421,7 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
     kv_range(P, q0, kt_lo, kt_hi);
     float m = -INFINITY, l = 0.f;  // m in log2 units (scores x log2(e)/sqrt(d))
     if (P.sink != nullptr) {
-      m = __ldg(P.sink + head) * kLog2e;
+      m = (P.hq <= kMaxStagedSinks ? C->sink[head] : __ldg(P.sink + head)) * kLog2e;
       l = 1.f;
     }
     for (int kt = kt_lo; kt <= kt_hi; ++kt, ++n_t) {
@@ -396,27 +434,39 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
       reg_fence(s[1]);
       reg_fence(s[2]);
       reg_fence(s[3]);
-      // key column c is allowed iff d - window <= c <= d (d = query pos - tile's first key pos)
+      // key column c is allowed iff d - window <= c <= d (d = query pos - tile's first key pos).
+      // The allowed columns form one contiguous run [c_lo, c_hi]; masking uses a 32-bit run mask
+      // per chunk, and the row max uses 8 independent accumulators (short dependency chains).
       const int d = q0 - kt * kBlockN + r;
-      const bool full_tile = (d >= kBlockN - 1) && (P.window < 0 || d - P.window <= 0);
-      float mt = -INFINITY;
-      if (full_tile) {
+      const int c_hi = min(d, kBlockN - 1);
+      const int c_lo = (P.window >= 0) ? max(d - P.window, 0) : 0;
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+      if (c_lo == 0 && c_hi == kBlockN - 1) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mt = fmaxf(mt, __uint_as_float(s[q][i]));
+          for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(s[q][i]));
       } else {
-        const int cmin = (P.window >= 0) ? d - P.window : -1;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 4; ++q) {
+          const int lo = c_lo - 32 * q, hi = c_hi - 32 * q;  // run relative to this chunk
+          uint32_t run = 0u;
+          if (hi >= 0 && lo <= 31 && lo <= hi) {
+            const uint32_t upto = (hi >= 31) ? 0xffffffffu : ((2u << hi) - 1u);
+            const uint32_t below = (lo <= 0) ? 0u : ((1u << lo) - 1u);
+            run = upto & ~below;
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int c = 32 * q + i;
-            const float x = (c <= d && c >= cmin) ? __uint_as_float(s[q][i]) : -INFINITY;
+            const float x = ((run >> i) & 1u) ? __uint_as_float(s[q][i]) : -INFINITY;
             s[q][i] = __float_as_uint(x);
-            mt = fmaxf(mt, x);
+            mx[i & 7] = fmaxf(mx[i & 7], x);
           }
+        }
       }
+      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       mt *= sl2;
       // lazy rescale: keep the running max unless it grows by more than the threshold
       const bool grow = mt > m + kRescaleThreshold;
@@ -424,7 +474,9 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
       const float corr = grow ? ex2_approx(m - m_new) : 1.f;  // m = -inf -> 0
       const float base = (m_new == -INFINITY) ? 0.f : m_new;
       // P = exp2(s * scale - m) as bf16 pairs, stored 32 keys (16 columns) at a time as S registers retire
-      float sum0 = 0.f, sum1 = 0.f;
+      float sm[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sm[k] = 0.f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
@@ -432,13 +484,13 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
         for (int i = 0; i < 32; i += 2) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(s[q][i]), sl2, -base));
           const float p1 = ex2_approx(fmaf(__uint_as_float(s[q][i + 1]), sl2, -base));
-          sum0 += p0;
-          sum1 += p1;
+          sm[i & 7] += p0;
+          sm[(i + 1) & 7] += p1;
           pk[i >> 1] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + 16 * q, pk);
       }
-      l = l * corr + (sum0 + sum1);
+      l = l * corr + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
       m = m_new;
       if (kt != kt_lo && __any_sync(0xffffffffu, grow)) {
         // rescale O; the previous PV has completed (it was issued before this tile's S)
@@ -471,67 +523,49 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
     const int p = q0 + r;
     if (p < W.L) {
       const float inv = P.v_scale / l;
-      uint4* dst = reinterpret_cast<uint4*>(P.out + (static_cast<size_t>(W.s_b + p) * P.hq + head) * kHeadDimV);
+      uint16_t* dst = P.out + (static_cast<size_t>(W.s_b + p) * P.hq + head) * kHeadDimV;
 #pragma unroll
-      for (int qd = 0; qd < 16; ++qd) {
-        const int q = qd >> 2, i = (qd & 3) * 8;
-        uint4 val;
-        val.x = pack_bf16x2(__uint_as_float(o[q][i + 0]) * inv, __uint_as_float(o[q][i + 1]) * inv);
-        val.y = pack_bf16x2(__uint_as_float(o[q][i + 2]) * inv, __uint_as_float(o[q][i + 3]) * inv);
-        val.z = pack_bf16x2(__uint_as_float(o[q][i + 4]) * inv, __uint_as_float(o[q][i + 5]) * inv);
-        val.w = pack_bf16x2(__uint_as_float(o[q][i + 6]) * inv, __uint_as_float(o[q][i + 7]) * inv);
-        dst[qd] = val;
+      for (int qd = 0; qd < 8; ++qd) {  // 16 dims (32 bytes) per store
+        const int q = qd >> 1, i = (qd & 1) * 16;
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(o[q][i + 2 * e]) * inv, __uint_as_float(o[q][i + 2 * e + 1]) * inv);
+        st_global_v8(dst + 16 * qd, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
       }
       P.lse[static_cast<size_t>(head) * P.total_tokens + W.s_b + p] = (m + log2f(l)) * kLn2;
     }
   }
 }
 
-// RoPE warpgroup: thread r owns row r of every rope unit it rotates.
+// RoPE warpgroup: thread r owns row r of each head's Q rope unit.
 __device__ void role_rope(uint8_t* smem, Ctrl* C, const FwdParams& P, int r) {
   const uint64_t lim = P.wait_limit_ns;
   float oc[32], os[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) rope_sincos(r, P.theta[i], os[i], oc[i]);
+  for (int i = 0; i < 32; ++i) rope_sincos(r, C->theta[i], os[i], oc[i]);
   float amax = 0.f;
   UnitWalker W(P);
   int q0, h0;
-  uint32_t n_u = 0, n_t = 0;
+  uint32_t n_u = 0;
   bool ok = true;
   for (long long u = blockIdx.x; ok && W.unit(u, q0, h0); u += gridDim.x, ++n_u) {
     if (r < 32) {
       float sn, cs;
-      rope_sincos(q0, P.theta[r], sn, cs);
+      rope_sincos(q0, C->theta[r], sn, cs);
       C->base_q[r] = make_float2(cs, sn);
     }
     named_bar_sync(kRopeBarId, 128);
-    if (!pwait(C, &C->q_full, n_u & 1, lim)) { ok = false; }
-    if (ok) {
-      amax = fmaxf(amax, rope_row_rotate(smem + kQOff, r, C->base_q, oc, os));
-      amax = fmaxf(amax, rope_row_rotate(smem + kQOff + 3 * kUnit, r, C->base_q, oc, os));
-      fence_proxy_async_smem();
-    }
-    named_bar_sync(kRopeBarId, 128);
-    if (!ok) break;
-    if (r == 0) mbar_arrive(&C->q_roped);
-    int kt_lo, kt_hi;
-    kv_range(P, q0, kt_lo, kt_hi);
-    for (int kt = kt_lo; kt <= kt_hi; ++kt, ++n_t) {
-      if (r < 32) {
-        float sn, cs;
-        rope_sincos(kt * kBlockN, P.theta[r], sn, cs);
-        C->base_k[r] = make_float2(cs, sn);
-      }
-      named_bar_sync(kRopeBarId, 128);
-      const uint32_t slot = kslot(n_t, 0);
-      if (!pwait(C, &C->slot_full[slot], kphase(n_t, 0), lim)) { ok = false; }
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      if (!pwait(C, &C->q_full[h], n_u & 1, lim)) ok = false;
       if (ok) {
-        amax = fmaxf(amax, rope_row_rotate(smem + kRingOff + slot * kUnit, r, C->base_k, oc, os));
+        amax = fmaxf(amax, rope_row_rotate(smem + kQOff + 3 * h * kUnit, r, C->base_q, oc, os));
         fence_proxy_async_smem();
       }
       named_bar_sync(kRopeBarId, 128);
       if (!ok) break;
-      if (r == 0) mbar_arrive(&C->slot_ready[slot]);
+      if (r == 0) mbar_arrive(&C->q_roped[h]);
     }
   }
   if (amax > 65504.f) atomicOr(&g_mimo_error, kErrRange);
@@ -541,8 +575,9 @@ __device__ void role_rope(uint8_t* smem, Ctrl* C, const FwdParams& P, int r) {
 
 // ---------------------------------------------------------------- kernel
 __global__ void __launch_bounds__(pipe::kThreads, 1)
-    attn_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ FwdParams P) {
+    attn_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kr,
+                              const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                              const __grid_constant__ FwdParams P) {
   using namespace pipe;
   extern __shared__ __align__(1024) uint8_t smem[];
   Ctrl* C = reinterpret_cast<Ctrl*>(smem + kCtrlOff);
@@ -560,25 +595,29 @@ __global__ void __launch_bounds__(pipe::kThreads, 1)
 
   if (tid == 0) {
     prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_kr);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
-    mbar_init(&C->q_full, 1);
-    mbar_init(&C->q_roped, 1);
-    mbar_init(&C->q_empty, 1);
-    for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&C->slot_full[s], 1);
-      mbar_init(&C->slot_empty[s], 1);
-      mbar_init(&C->slot_ready[s], 1);
-    }
     for (int h = 0; h < 2; ++h) {
+      mbar_init(&C->q_full[h], 1);
+      mbar_init(&C->q_roped[h], 1);
+      mbar_init(&C->q_empty[h], 1);
       mbar_init(&C->s_full[h], 1);
       mbar_init(&C->p_full[h], 128);
       mbar_init(&C->o_full[h], 1);
       mbar_init(&C->o_empty[h], 128);
     }
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&C->slot_full[s], 1);
+      mbar_init(&C->slot_empty[s], 1);
+    }
     C->abort = 0;
+#pragma unroll
+    for (int i = 0; i < kRopeDims / 2; ++i) C->theta[i] = P.theta[i];
     fence_barrier_init();
   }
+  if (P.sink != nullptr && P.hq <= kMaxStagedSinks)
+    for (int h = tid; h < P.hq; h += kThreads) C->sink[h] = __ldg(P.sink + h);
   if (warp == 1) {
     tmem_alloc(&C->tmem_base, kTmemCols);
     tmem_relinquish();
@@ -593,7 +632,7 @@ __global__ void __launch_bounds__(pipe::kThreads, 1)
     if (lane == 0) {
       if (warp == 0) role_q_loader(smem, C, &tm_q, P);
       else if (warp == 1) role_mma(smem, C, tmem, P);
-      else if (warp == 2) role_kv_loader(smem, C, &tm_k, &tm_v, P);
+      else if (warp == 2) role_kv_loader(smem, C, &tm_kr, &tm_k, &tm_v, P);
     }
   } else if (warp < 12) {
     setmaxnreg_inc<kRegsSoftmax>();

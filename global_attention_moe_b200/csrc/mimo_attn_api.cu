@@ -15,6 +15,7 @@
 #include "../../include/mimo_attn.h"
 #include "attn_fwd_pipelined.cuh"
 #include "attn_fwd_simple.cuh"
+#include "rope_k_prepass.cuh"
 #include "params.cuh"
 
 using namespace mimo;
@@ -36,15 +37,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensormap_encoder() {
   return fn;
 }
 
-// 2-D bf16 view [rows, inner] (row-major) with a {64, box_rows} box and 128-byte swizzle.
-bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows = 128) {
+// 2-D 16-bit view [rows, inner] (row-major) with a {64, box_rows} box and 128-byte swizzle.
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows = 128,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = tensormap_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -106,6 +108,7 @@ struct DeviceInfo {
   int sms = 0;
   bool simple_ready = false;
   bool pipelined_ready = false;
+  cudaMemPool_t pool = nullptr;  // stream-ordered scratch, kept by the library (never released to the OS)
 };
 
 DeviceInfo* device_info(int dev) {
@@ -121,6 +124,17 @@ DeviceInfo* device_info(int dev) {
     d.pipelined_ready = cudaFuncSetAttribute(attn_fwd_pipelined_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              pipe::kSmemBytes) == cudaSuccess;
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof props);
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    if (cudaMemPoolCreate(&d.pool, &props) == cudaSuccess) {
+      uint64_t keep = UINT64_MAX;
+      cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    } else {
+      d.pool = nullptr;
+    }
   }
   return &d;
 }
@@ -139,17 +153,42 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& P, cuda
       !encode_2d(&tk, k, (uint64_t)P.hkv * kHeadDimQK, P.total_tokens) ||
       !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, P.total_tokens, pipelined ? 64 : 128))
     return MIMO_ERR_CUDA;
-  if (pipelined) {
-    if (!info->pipelined_ready) return MIMO_ERR_CUDA;
-    const long long units = (long long)(P.hq / 2) * ((P.total_tokens + kBlockM - 1) / kBlockM + P.num_seqs);
-    const int grid = (int)std::min<long long>(units, info->sms);
-    attn_fwd_pipelined_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tk, tv, P);
-  } else {
+  if (!pipelined) {
     if (!info->simple_ready) return MIMO_ERR_CUDA;
     dim3 grid((P.max_seqlen + kBlockM - 1) / kBlockM, P.num_seqs, P.hq);
     attn_fwd_simple_kernel<<<grid, simple::kThreads, simple::kSmemBytes, stream>>>(tq, tk, tv, P);
+    return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+  if (!info->pipelined_ready || !info->pool) return MIMO_ERR_CUDA;
+  // K's rope dims, rotated once: transient scratch from the library's stream-ordered pool
+  const size_t kr_rows = (size_t)P.total_tokens * P.hkv;
+  void* k_rope = nullptr;
+  if (cudaMallocFromPoolAsync(&k_rope, kr_rows * kRopeDims * 2, info->pool, stream) != cudaSuccess)
+    return MIMO_ERR_CUDA;
+  RopeKParams R;
+  std::memset(&R, 0, sizeof R);
+  R.k = static_cast<const uint16_t*>(k);
+  R.k_rope = static_cast<uint16_t*>(k_rope);
+  R.cu_seqlens = P.cu_seqlens;
+  R.num_seqs = P.num_seqs;
+  R.total_tokens = P.total_tokens;
+  R.hkv = P.hkv;
+  for (int i = 0; i < kRopeDims / 2; ++i) R.theta[i] = P.theta[i];
+  const long long threads = (long long)kr_rows * 4;
+  rope_k_prepass_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(R);
+  int st = cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+  CUtensorMap tkr;
+  if (st == MIMO_OK && !encode_2d(&tkr, k_rope, (uint64_t)P.hkv * kRopeDims, P.total_tokens, 128,
+                                  CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    st = MIMO_ERR_CUDA;
+  if (st == MIMO_OK) {
+    const long long units = (long long)(P.hq / 2) * ((P.total_tokens + kBlockM - 1) / kBlockM + P.num_seqs);
+    const int grid = (int)std::min<long long>(units, info->sms);
+    attn_fwd_pipelined_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tkr, tk, tv, P);
+    if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+  }
+  if (cudaFreeAsync(k_rope, stream) != cudaSuccess) st = MIMO_ERR_CUDA;
+  return st;
 }
 
 __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {

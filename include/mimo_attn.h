@@ -23,7 +23,7 @@
  * Conventions for every entry point:
  *   - Device pointers are caller-owned CUDA global memory on the current
  *     device; host pointers are caller-owned host memory.  The library keeps
- *     no pointer after a call returns.
+ *     no caller pointer after a call returns.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Kernels run asynchronously on it; only the entry points that
  *     say so synchronise.
@@ -101,7 +101,11 @@ typedef struct {
  * Rotated Q/K rope dims enter the tensor cores as FP16 (the pass-through dims
  * stay BF16), so |q|, |k| on the first 64 dims must stay below 2^15; a larger
  * rotated value is recorded as MIMO_ERR_RANGE for mimo_attn_check.
- * Allocates nothing.  Does not synchronise.
+ * Scratch: when Hq/Hkv is even (the pipelined kernel), the call rotates K's
+ * rope dims once into T * Hkv * 128 bytes of transient device scratch taken
+ * from a library-owned stream-ordered memory pool (cudaMallocFromPoolAsync on
+ * `stream`, returned with cudaFreeAsync on the same stream; the pool keeps
+ * its memory for reuse until the process exits).  Does not synchronise.
  */
 MIMO_API int mimo_attn_fwd(const void* q, const void* k, const void* v, const float* sink,
                   const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind,
@@ -122,7 +126,8 @@ MIMO_API size_t mimo_attn_host_workspace_size(const mimo_attn_dims* dims, int ha
  * mimo_attn_host_workspace_size bytes, 256-byte aligned.  The call copies the
  * inputs host->device on `stream`, runs the forward, copies out and lse
  * device->host and synchronises the stream before returning, so the host
- * buffers hold the result on return.  Allocates nothing.
+ * buffers hold the result on return.  Takes the same transient scratch as
+ * mimo_attn_fwd.
  */
 MIMO_API int mimo_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                        const float* sink_host, const int32_t* cu_seqlens_host,
