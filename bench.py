@@ -102,6 +102,31 @@ def recorded_traffic(kernel: str, workload: str):
     return float(e["dram_bytes_per_launch"])
 
 
+# ------------------------------------------------------------------ multi-rank plumbing
+def rank_workload(name: str, rank: int) -> W.Workload:
+    """Weak scaling: every rank draws its own batch of the workload's shape (seed = rank)."""
+    w = W.WORKLOADS[name](seed=0)
+    if rank:
+        w.seed = rank
+    return w
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Largest value over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(world: int, units_per_rank_step: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed / the slowest rank's time."""
+    return world * units_per_rank_step * steps / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while running."""
@@ -257,8 +282,7 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    w = W.WORKLOADS[args.workload](seed=0)
-    w.seed = rank  # weak scaling: every rank draws its own batch of the same shape
+    w = rank_workload(args.workload, rank)
     x = W.make_inputs(w)
     T = w.total_tokens
     stream = torch.cuda.current_stream()
@@ -313,12 +337,9 @@ def run_ours(args):
     st = mimo_attn.check()
     if st != mimo_attn.OK:
         raise mimo_attn.MimoAttnError(st, "timed region")
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     ms_per_step = ms / max(args.steps, 1)
-    value = world * T * args.steps / (ms / 1e3)
+    value = aggregate_rate(world, T, args.steps, ms)
 
     # --- end to end through the host-buffer C-ABI entry (pinned host memory, copies inside the region)
     e2e = None
@@ -345,12 +366,8 @@ def run_ours(args):
             mimo_attn.fwd_host(qh, kh, vh, shh, ch, dims, lk, win, base, rd, vs, oh, lh, ws)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * T * ne / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": aggregate_rate(world, T, ne, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": ne}
 
     # --- parity spot check of this run's output against the oracle (rank 0)
