@@ -205,6 +205,92 @@ __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// ---------------------------------------------------------------------------
+// Scratch for mimo_attn_fwd_noalloc.  Some callers cannot allocate device
+// memory while they run: a framework that has already reserved the device
+// for its own caching allocator, or a serving loop that forbids allocation on
+// its hot path.  For them the rotated-K scratch lives in this file-scope
+// array instead of the stream-ordered pool.  Every GPU that loads the library
+// holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB: T * Hkv <= 262144 rows of 64 FP16 dims
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocInfo {
+  int sms = 0;
+  bool ready = false;
+  void* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+};
+
+// Per-device set-up, done by the first no-alloc call on that device with the
+// device current: kernel attributes, SM count and the scratch array's device
+// address (in host code the array's name is only a host-side stand-in).
+NoAllocInfo* noalloc_info(int dev) {
+  static NoAllocInfo infos[64];
+  static std::mutex mu;
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  NoAllocInfo& d = infos[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+    if (cudaFuncSetAttribute(attn_fwd_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             simple::kSmemBytes) != cudaSuccess)
+      return nullptr;
+    if (cudaFuncSetAttribute(attn_fwd_pipelined_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pipe::kSmemBytes) != cudaSuccess)
+      return nullptr;
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return nullptr;
+    d.scratch = ptr;
+    d.ready = true;
+  }
+  return &d;
+}
+
+int launch_noalloc(const void* q, const void* k, const void* v, const FwdParams& P, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
+  const int choice = g_kernel_choice.load();
+  const bool pipelined = (choice == MIMO_KERNEL_PIPELINED) || (choice == MIMO_KERNEL_AUTO && P.group % 2 == 0);
+  if (pipelined && P.group % 2 != 0) return MIMO_ERR_UNSUPPORTED;
+  const size_t kr_rows = (size_t)P.total_tokens * P.hkv;
+  if (pipelined && kr_rows * kRopeDims * 2 > kNoAllocScratchBytes) return MIMO_ERR_SCRATCH_LIMIT;
+  NoAllocInfo* info = noalloc_info(dev);
+  if (!info) return MIMO_ERR_CUDA;
+  if (P.max_seqlen == 0) return MIMO_OK;
+  CUtensorMap tq, tk, tv;
+  if (!encode_2d(&tq, q, (uint64_t)P.hq * kHeadDimQK, P.total_tokens) ||
+      !encode_2d(&tk, k, (uint64_t)P.hkv * kHeadDimQK, P.total_tokens) ||
+      !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, P.total_tokens, pipelined ? 64 : 128))
+    return MIMO_ERR_CUDA;
+  if (!pipelined) {
+    dim3 grid((P.max_seqlen + kBlockM - 1) / kBlockM, P.num_seqs, P.hq);
+    attn_fwd_simple_kernel<<<grid, simple::kThreads, simple::kSmemBytes, stream>>>(tq, tk, tv, P);
+    return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+  }
+  // The pre-pass overwrites every scratch row the attention kernel reads, so
+  // nothing needs clearing between calls.
+  RopeKParams R;
+  std::memset(&R, 0, sizeof R);
+  R.k = static_cast<const uint16_t*>(k);
+  R.k_rope = static_cast<uint16_t*>(info->scratch);
+  R.cu_seqlens = P.cu_seqlens;
+  R.num_seqs = P.num_seqs;
+  R.total_tokens = P.total_tokens;
+  R.hkv = P.hkv;
+  for (int i = 0; i < kRopeDims / 2; ++i) R.theta[i] = P.theta[i];
+  const long long threads = (long long)kr_rows * 4;
+  rope_k_prepass_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(R);
+  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  CUtensorMap tkr;
+  if (!encode_2d(&tkr, info->scratch, (uint64_t)P.hkv * kRopeDims, P.total_tokens, 128,
+                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return MIMO_ERR_CUDA;
+  const long long units = (long long)(P.hq / 2) * ((P.total_tokens + kBlockM - 1) / kBlockM + P.num_seqs);
+  const int grid = (int)std::min<long long>(units, info->sms);
+  attn_fwd_pipelined_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tkr, tk, tv, P);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -319,11 +405,25 @@ const char* mimo_attn_status_string(int status) {
     case MIMO_ERR_TIMEOUT: return "bounded wait timed out in a kernel";
     case MIMO_ERR_RANGE: return "rotated Q/K value outside the FP16 range";
     case MIMO_ERR_BAD_SEQLENS: return "cu_seqlens inconsistent with dims";
+    case MIMO_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the no-alloc entry point holds";
     default: return "unknown status";
   }
 }
 
 int mimo_attn_version(void) { return (1 << 16) | 1; }
+
+int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* sink,
+                          const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind, int window,
+                          double rope_base, int rope_dims, float v_scale, void* out, float* lse, void* stream) {
+  int st = validate(q, k, v, sink, cu_seqlens, dims, layer_kind, window, rope_base, rope_dims, v_scale, out, lse);
+  if (st != MIMO_OK) return st;
+  if (dims->total_tokens == 0) return MIMO_OK;
+  FwdParams P;
+  fill_params(P, sink, cu_seqlens, dims, layer_kind, window, rope_base, v_scale, out, lse);
+  return launch_noalloc(q, k, v, P, static_cast<cudaStream_t>(stream));
+}
+
+size_t mimo_attn_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 int mimo_attn_set_kernel(int choice) {
   if (choice != MIMO_KERNEL_AUTO && choice != MIMO_KERNEL_SIMPLE && choice != MIMO_KERNEL_PIPELINED)

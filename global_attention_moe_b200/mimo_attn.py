@@ -15,12 +15,12 @@ LIB_PATH = os.path.join(HERE, "_build", "libmimo_attn.so")
 
 LAYER_SWA = 0
 LAYER_GLOBAL = 1
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BAD_SEQLENS = range(7)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BAD_SEQLENS, ERR_SCRATCH_LIMIT = range(8)
 
 # Every symbol include/mimo_attn.h declares.
 SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host", "mimo_attn_check",
-           "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_set_kernel",
-           "mimo_attn_version")
+           "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_fwd_noalloc",
+           "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_version")
 KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED = 0, 1, 2
 
 
@@ -54,6 +54,10 @@ def _load():
     lib.mimo_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
     lib.mimo_attn_status_string.restype = ctypes.c_char_p
     lib.mimo_attn_status_string.argtypes = [I]
+    lib.mimo_attn_fwd_noalloc.restype = I
+    lib.mimo_attn_fwd_noalloc.argtypes = [P, P, P, P, P, ctypes.POINTER(Dims), I, I, D, I, F, P, P, P]
+    lib.mimo_attn_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.mimo_attn_noalloc_scratch_bytes.argtypes = []
     lib.mimo_attn_set_kernel.restype = I
     lib.mimo_attn_set_kernel.argtypes = [I]
     lib.mimo_attn_version.restype = I
@@ -119,6 +123,26 @@ def fwd(q, k, v, sink, cu_seqlens, max_seqlen, layer_kind, window, rope_base, ro
     if st != OK:
         raise MimoAttnError(st, "mimo_attn_fwd")
     return out, lse
+
+
+def fwd_noalloc(q, k, v, sink, cu_seqlens, max_seqlen, layer_kind, window, rope_base, out, lse, rope_dims=64,
+                v_scale=0.707, stream=None):
+    """Same as fwd() through mimo_attn_fwd_noalloc: for callers that cannot allocate
+    device memory during the call (the caller passes out and lse; the library's
+    scratch is a fixed array of noalloc_scratch_bytes())."""
+    dims = make_dims(cu_seqlens.numel() - 1, q.shape[0], max_seqlen, q.shape[1], k.shape[1], q.shape[2], v.shape[2])
+    st = LIB.mimo_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                   sink.data_ptr() if sink is not None else None, cu_seqlens.data_ptr(),
+                                   ctypes.byref(dims), int(layer_kind), int(window), float(rope_base),
+                                   int(rope_dims), float(v_scale), out.data_ptr(), lse.data_ptr(),
+                                   _stream_handle(stream))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_attn_fwd_noalloc")
+    return out, lse
+
+
+def noalloc_scratch_bytes() -> int:
+    return LIB.mimo_attn_noalloc_scratch_bytes()
 
 
 def host_workspace_size(dims: Dims, has_sink: bool) -> int:

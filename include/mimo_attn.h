@@ -60,7 +60,8 @@ typedef enum {
   MIMO_ERR_CUDA = 3,        /* a CUDA runtime/driver call or kernel launch failed */
   MIMO_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (reported by mimo_attn_check) */
   MIMO_ERR_RANGE = 5,       /* a rotated Q/K value exceeded the FP16 range (|x| > 65504) */
-  MIMO_ERR_BAD_SEQLENS = 6  /* the kernel found cu_seqlens inconsistent with dims (reported by mimo_attn_check) */
+  MIMO_ERR_BAD_SEQLENS = 6, /* the kernel found cu_seqlens inconsistent with dims (reported by mimo_attn_check) */
+  MIMO_ERR_SCRATCH_LIMIT = 7 /* mimo_attn_fwd_noalloc: T * Hkv * 128 bytes exceed its fixed scratch */
 } mimo_status;
 
 /* Shapes.  Supported: head_dim_qk = 192, head_dim_v = 128,
@@ -155,6 +156,35 @@ MIMO_API int mimo_attn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 /* Static description of a status code (never NULL). */
 MIMO_API const char* mimo_attn_status_string(int status);
+
+/*
+ * Same operation, arguments and results as mimo_attn_fwd, for callers that
+ * cannot allocate device memory during the call -- for example a framework
+ * that has already reserved the device for its own caching allocator, or a
+ * serving loop that forbids allocation on its hot path.  (This entry point
+ * has no counterpart in the pages that describe the layer; it only changes
+ * where the scratch lives.)
+ *   - The rotated-K scratch (T * Hkv * 128 bytes) lives in a fixed device
+ *     array inside the library, mimo_attn_noalloc_scratch_bytes() bytes
+ *     (32 MiB), that every GPU which loads the library holds until the
+ *     process exits.  Larger problems are rejected with
+ *     MIMO_ERR_SCRATCH_LIMIT before anything is launched.
+ *   - The call makes no cudaMalloc/cudaFree or pool allocation.
+ *   - The first call on a device, with that device current, looks up the
+ *     array's device address and sets kernel attributes; make that first
+ *     call before any stream capture.
+ *   - Every call uses the same array, so calls that overlap on the GPU (on
+ *     different streams, or on one stream without ordering) race; calls on
+ *     one stream are ordered and safe.  Each call rewrites every scratch row
+ *     it reads, so nothing needs clearing between calls.
+ */
+MIMO_API int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* sink,
+                                   const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind,
+                                   int window, double rope_base, int rope_dims, float v_scale, void* out,
+                                   float* lse, void* stream);
+
+/* Size in bytes of the fixed scratch array mimo_attn_fwd_noalloc uses. */
+MIMO_API size_t mimo_attn_noalloc_scratch_bytes(void);
 
 /* Kernel selection for mimo_attn_fwd (process-wide; default AUTO).
  *   MIMO_KERNEL_AUTO       pipelined kernel when Hq/Hkv is even, else the simple one
