@@ -11,6 +11,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "../../include/mimo_attn.h"
 #include "attn_fwd_pipelined.cuh"
@@ -104,6 +106,37 @@ void fill_params(FwdParams& P, const float* sink, const int32_t* cu, const mimo_
 
 std::atomic<int> g_kernel_choice{MIMO_KERNEL_AUTO};
 
+// Kernel timing: while enabled, each forward records an event pair around its
+// attention kernel (library-owned events, per device, reused across sessions).
+struct ProfileState {
+  std::mutex mu;
+  bool enabled = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pairs[64];
+  size_t used[64] = {};
+};
+ProfileState& profile_state() {
+  static ProfileState st;
+  return st;
+}
+
+// Returns the event pair to record around the next attention kernel, or null when not profiling.
+std::pair<cudaEvent_t, cudaEvent_t>* profile_slot(int dev) {
+  ProfileState& st = profile_state();
+  std::lock_guard<std::mutex> lock(st.mu);
+  if (!st.enabled || dev < 0 || dev >= 64) return nullptr;
+  auto& v = st.pairs[dev];
+  if (st.used[dev] == v.size()) {
+    cudaEvent_t a, b;
+    if (cudaEventCreate(&a) != cudaSuccess) return nullptr;
+    if (cudaEventCreate(&b) != cudaSuccess) {
+      cudaEventDestroy(a);
+      return nullptr;
+    }
+    v.emplace_back(a, b);
+  }
+  return &v[st.used[dev]++];
+}
+
 struct DeviceInfo {
   int sms = 0;
   bool simple_ready = false;
@@ -184,8 +217,11 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& P, cuda
   if (st == MIMO_OK) {
     const long long units = (long long)(P.hq / 2) * ((P.total_tokens + kBlockM - 1) / kBlockM + P.num_seqs);
     const int grid = (int)std::min<long long>(units, info->sms);
+    auto* ev = profile_slot(dev);
+    if (ev) cudaEventRecord(ev->first, stream);
     attn_fwd_pipelined_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tkr, tk, tv, P);
     if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+    if (ev) cudaEventRecord(ev->second, stream);
   }
   if (cudaFreeAsync(k_rope, stream) != cudaSuccess) st = MIMO_ERR_CUDA;
   return st;
@@ -408,6 +444,37 @@ const char* mimo_attn_status_string(int status) {
     case MIMO_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the no-alloc entry point holds";
     default: return "unknown status";
   }
+}
+
+int mimo_attn_profile_start(void) {
+  ProfileState& st = profile_state();
+  std::lock_guard<std::mutex> lock(st.mu);
+  st.enabled = true;
+  for (auto& u : st.used) u = 0;
+  return MIMO_OK;
+}
+
+int mimo_attn_profile_stop(int* launches, double* total_ms) {
+  if (!launches || !total_ms) return MIMO_ERR_INVALID_ARG;
+  ProfileState& st = profile_state();
+  std::lock_guard<std::mutex> lock(st.mu);
+  st.enabled = false;
+  int n = 0;
+  double ms = 0.0;
+  for (int dev = 0; dev < 64; ++dev) {
+    for (size_t i = 0; i < st.used[dev]; ++i) {
+      auto& pr = st.pairs[dev][i];
+      if (cudaEventSynchronize(pr.second) != cudaSuccess) return MIMO_ERR_CUDA;
+      float e = 0.f;
+      if (cudaEventElapsedTime(&e, pr.first, pr.second) != cudaSuccess) return MIMO_ERR_CUDA;
+      ms += e;
+      ++n;
+    }
+    st.used[dev] = 0;
+  }
+  *launches = n;
+  *total_ms = ms;
+  return MIMO_OK;
 }
 
 int mimo_attn_version(void) { return (1 << 16) | 1; }

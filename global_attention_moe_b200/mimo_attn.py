@@ -20,7 +20,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BAD_
 # Every symbol include/mimo_attn.h declares.
 SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host", "mimo_attn_check",
            "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_fwd_noalloc",
-           "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_version")
+           "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_profile_start",
+           "mimo_attn_profile_stop", "mimo_attn_version")
 KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED = 0, 1, 2
 
 
@@ -58,6 +59,10 @@ def _load():
     lib.mimo_attn_fwd_noalloc.argtypes = [P, P, P, P, P, ctypes.POINTER(Dims), I, I, D, I, F, P, P, P]
     lib.mimo_attn_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.mimo_attn_noalloc_scratch_bytes.argtypes = []
+    lib.mimo_attn_profile_start.restype = I
+    lib.mimo_attn_profile_start.argtypes = []
+    lib.mimo_attn_profile_stop.restype = I
+    lib.mimo_attn_profile_stop.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
     lib.mimo_attn_set_kernel.restype = I
     lib.mimo_attn_set_kernel.argtypes = [I]
     lib.mimo_attn_version.restype = I
@@ -82,6 +87,20 @@ def set_kernel(choice: int) -> None:
     st = LIB.mimo_attn_set_kernel(int(choice))
     if st != OK:
         raise MimoAttnError(st, "mimo_attn_set_kernel")
+
+
+def profile_start() -> None:
+    """Record the attention kernel's duration on every following forward (see profile_stop)."""
+    LIB.mimo_attn_profile_start()
+
+
+def profile_stop() -> tuple[int, float]:
+    """Stop recording; returns (attention-kernel launches, their summed milliseconds)."""
+    n, ms = ctypes.c_int(0), ctypes.c_double(0.0)
+    st = LIB.mimo_attn_profile_stop(ctypes.byref(n), ctypes.byref(ms))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_attn_profile_stop")
+    return n.value, ms.value
 
 
 def make_dims(num_seqs, total_tokens, max_seqlen, hq, hkv, dqk=192, dv=128) -> Dims:

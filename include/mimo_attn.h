@@ -198,6 +198,17 @@ MIMO_API size_t mimo_attn_noalloc_scratch_bytes(void);
 typedef enum { MIMO_KERNEL_AUTO = 0, MIMO_KERNEL_SIMPLE = 1, MIMO_KERNEL_PIPELINED = 2 } mimo_kernel_choice;
 MIMO_API int mimo_attn_set_kernel(int choice);
 
+/*
+ * Kernel timing for measurement tools.  After mimo_attn_profile_start, every
+ * forward that runs the pipelined kernel records a CUDA event pair (events
+ * owned by the library) around that kernel on the call's stream.
+ * mimo_attn_profile_stop ends recording, waits for the recorded events, and
+ * returns how many attention-kernel launches were recorded and their summed
+ * duration in milliseconds (the K RoPE pre-pass is excluded).  Process-wide.
+ */
+MIMO_API int mimo_attn_profile_start(void);
+MIMO_API int mimo_attn_profile_stop(int* launches, double* total_ms);
+
 /* ABI version: (major << 16) | minor. */
 MIMO_API int mimo_attn_version(void);
 
