@@ -39,10 +39,10 @@ from global_attention_moe_b200 import workloads as W  # noqa: E402
 METRIC = "attn fwd tokens/s and TFLOP/s on 1 B200 (SWA-sink and global); % of roofline"
 L2_BYTES = 126 * 2 ** 20
 FLOPS_PER_PAIR = 2 * 192 + 2 * 128
-# Device code of the pipelined path: the traffic recorded in profiles/traffic.json is valid
+# Device code of the two-head kernels: the traffic recorded in profiles/traffic.json is valid
 # only while these files are unchanged.
 KERNEL_SOURCES = ["csrc/sm100.cuh", "csrc/rope_smem.cuh", "csrc/params.cuh", "csrc/rope_k_prepass.cuh",
-                  "csrc/attn_fwd_pipelined.cuh"]
+                  "csrc/attn_fwd_pipelined.cuh", "csrc/attn_fwd_swa.cuh"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -80,6 +80,15 @@ def load_peaks():
             d = json.load(f)
         return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dominant_kernel(w) -> str:
+    """The attention kernel the library's default choice launches for this shape."""
+    if (w.num_q_heads // w.num_kv_heads) % 2 != 0:
+        return "attn_fwd_simple_kernel"
+    if w.layer_kind == W.LAYER_SWA and 0 <= w.window <= 128:
+        return "attn_fwd_swa_kernel"
+    return "attn_fwd_pipelined_kernel"
 
 
 def kernel_sources_sha() -> str:
@@ -423,7 +432,7 @@ def run_ours(args):
     long_region = ms > 1000.0
     tc_peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
     t_tc = flops / (tc_peak * 1e12)
-    kernel = "attn_fwd_pipelined_kernel" if (w.num_q_heads // w.num_kv_heads) % 2 == 0 else "attn_fwd_simple_kernel"
+    kernel = dominant_kernel(w)
     traffic = recorded_traffic(kernel, w.name)
     if t_hbm >= t_tc:
         ach = nbytes / tk_s / 1e9

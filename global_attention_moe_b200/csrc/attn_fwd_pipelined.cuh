@@ -86,6 +86,7 @@ struct Ctrl {
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint32_t tmem_base;
   int abort;
+  long long total_tiles;  // query tiles over all sequences (filled by kernels that schedule by tile)
   double theta[kRopeDims / 2];
   float2 base_q[kRopeDims / 2];
   float sink[kMaxStagedSinks];  // sink logits staged once per CTA (when hq <= kMaxStagedSinks)
@@ -110,6 +111,12 @@ struct UnitWalker {
   __device__ __forceinline__ explicit UnitWalker(const FwdParams& P)
       : cu(P.cu_seqlens), num_seqs(P.num_seqs), total_tokens(P.total_tokens), pairs(P.hq / 2), causal(P.window < 0) {}
 
+  __device__ __forceinline__ void reset() {
+    b = 0;
+    tile_base = 0;
+    ntiles = -1;
+  }
+
   __device__ __forceinline__ bool seek(long long ti) {
     while (b < num_seqs) {
       if (ntiles < 0) {
@@ -133,12 +140,27 @@ struct UnitWalker {
   }
 
   __device__ __forceinline__ bool unit(long long u, int& q0, int& h0) {
-    const long long ti = u / pairs;
+    // u < pairs x (query tiles + sequences) < 2^31 (the host bounds Hq x T); 32-bit division
+    const uint32_t uu = static_cast<uint32_t>(u), np = static_cast<uint32_t>(pairs);
+    const uint32_t ti = uu / np;
     if (!seek(ti)) return false;
-    const int local = static_cast<int>(ti - tile_base);
+    const int local = static_cast<int>(ti) - tile_base;
     const int qt = causal ? (ntiles - 1 - local) : local;
     q0 = qt * kBlockM;
-    h0 = 2 * static_cast<int>(u % pairs);
+    h0 = 2 * static_cast<int>(uu - ti * np);
+    return true;
+  }
+};
+
+// The units of one CTA as the pipelined kernel schedules them: unit blockIdx.x,
+// then every gridDim.x-th unit after it.  Every role builds the same iterator.
+struct StridedUnits {
+  UnitWalker W;
+  long long u;
+  __device__ __forceinline__ StridedUnits(const FwdParams& P, const void*) : W(P), u(blockIdx.x) {}
+  __device__ __forceinline__ bool next(int& q0, int& h0) {
+    if (!W.unit(u, q0, h0)) return false;
+    u += gridDim.x;
     return true;
   }
 };
@@ -271,11 +293,12 @@ __device__ __forceinline__ int unit_tiles(const FwdParams& P, int q0) {
   return kt_hi - kt_lo + 1;
 }
 
+template <class Units>
 __device__ void role_q_loader(uint8_t* smem, Ctrl* C, const CUtensorMap* tm_q, const FwdParams& P) {
-  UnitWalker W(P);
+  Units U(P, C);
+  const UnitWalker& W = U.W;
   int q0, h0;
-  uint32_t n_u = 0;
-  for (long long u = blockIdx.x; W.unit(u, q0, h0); u += gridDim.x, ++n_u) {
+  for (uint32_t n_u = 0; U.next(q0, h0); ++n_u) {
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
       if (n_u > 0 && !pwait(C, &C->q_empty[h], (n_u - 1) & 1, P.wait_limit_ns)) return;
@@ -539,17 +562,17 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
 }
 
 // RoPE warpgroup: thread r owns row r of each head's Q rope unit.
+template <class Units>
 __device__ void role_rope(uint8_t* smem, Ctrl* C, const FwdParams& P, int r) {
   const uint64_t lim = P.wait_limit_ns;
   float oc[32], os[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) rope_sincos(r, C->theta[i], os[i], oc[i]);
   float amax = 0.f;
-  UnitWalker W(P);
+  Units U(P, C);
   int q0, h0;
-  uint32_t n_u = 0;
   bool ok = true;
-  for (long long u = blockIdx.x; ok && W.unit(u, q0, h0); u += gridDim.x, ++n_u) {
+  for (uint32_t n_u = 0; ok && U.next(q0, h0); ++n_u) {
     if (r < 32) {
       float sn, cs;
       rope_sincos(q0, C->theta[r], sn, cs);
@@ -630,7 +653,7 @@ __global__ void __launch_bounds__(pipe::kThreads, 1)
   if (warp < 4) {
     setmaxnreg_dec<kRegsCtl>();
     if (lane == 0) {
-      if (warp == 0) role_q_loader(smem, C, &tm_q, P);
+      if (warp == 0) role_q_loader<StridedUnits>(smem, C, &tm_q, P);
       else if (warp == 1) role_mma(smem, C, tmem, P);
       else if (warp == 2) role_kv_loader(smem, C, &tm_kr, &tm_k, &tm_v, P);
     }
@@ -640,7 +663,7 @@ __global__ void __launch_bounds__(pipe::kThreads, 1)
     role_softmax(C, tmem, P, hw, tid - 128 * (1 + hw), warp & 3);
   } else {
     setmaxnreg_dec<kRegsRope>();
-    role_rope(smem, C, P, tid - 384);
+    role_rope<StridedUnits>(smem, C, P, tid - 384);
   }
   __syncwarp();
   tc_fence_before_sync();

@@ -17,6 +17,7 @@
 #include "../../include/mimo_attn.h"
 #include "attn_fwd_pipelined.cuh"
 #include "attn_fwd_simple.cuh"
+#include "attn_fwd_swa.cuh"
 #include "rope_k_prepass.cuh"
 #include "params.cuh"
 
@@ -74,6 +75,9 @@ int validate(const void* q, const void* k, const void* v, const float* sink, con
   if (layer_kind == MIMO_LAYER_SWA && window < 0) return MIMO_ERR_INVALID_ARG;
   if (layer_kind == MIMO_LAYER_GLOBAL && sink != nullptr) return MIMO_ERR_INVALID_ARG;
   if ((int64_t)d->num_q_heads * d->total_tokens > INT32_MAX) return MIMO_ERR_UNSUPPORTED;
+  // unit indices of the two-head kernels stay below 2^31
+  if ((int64_t)(d->num_q_heads / 2 + 1) * ((int64_t)d->total_tokens / kBlockM + 1 + d->num_seqs) > INT32_MAX)
+    return MIMO_ERR_UNSUPPORTED;
   if (!cu) return MIMO_ERR_INVALID_ARG;
   if (d->total_tokens > 0) {
     if (!q || !k || !v || !out || !lse) return MIMO_ERR_INVALID_ARG;
@@ -105,6 +109,44 @@ void fill_params(FwdParams& P, const float* sink, const int32_t* cu, const mimo_
 }
 
 std::atomic<int> g_kernel_choice{MIMO_KERNEL_AUTO};
+
+enum class Path { Simple, Pipelined, Window };
+
+// Chooses the kernel for one call from the process-wide choice and the shape.
+int select_path(const FwdParams& P, Path& path) {
+  const bool even = P.group % 2 == 0;
+  const bool short_window = P.window >= 0 && P.window <= kBlockN;
+  switch (g_kernel_choice.load()) {
+    case MIMO_KERNEL_SIMPLE: path = Path::Simple; return MIMO_OK;
+    case MIMO_KERNEL_PIPELINED: path = Path::Pipelined; return even ? MIMO_OK : MIMO_ERR_UNSUPPORTED;
+    case MIMO_KERNEL_WINDOW: path = Path::Window; return (even && short_window) ? MIMO_OK : MIMO_ERR_UNSUPPORTED;
+    default: path = !even ? Path::Simple : (short_window ? Path::Window : Path::Pipelined); return MIMO_OK;
+  }
+}
+
+// Raises the dynamic shared memory limit of every kernel (once per device).
+bool set_smem_attributes() {
+  return cudaFuncSetAttribute(attn_fwd_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              simple::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(attn_fwd_pipelined_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              pipe::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(attn_fwd_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              pipe::kSmemBytes) == cudaSuccess;
+}
+
+// Persistent grid of the two-head kernels: one CTA per SM, at most one per unit.
+int persistent_grid(const FwdParams& P, int sms) {
+  const long long units = (long long)(P.hq / 2) * ((P.total_tokens + kBlockM - 1) / kBlockM + P.num_seqs);
+  return (int)std::min<long long>(units, sms);
+}
+
+void launch_two_head(Path path, int grid, const CUtensorMap& tq, const CUtensorMap& tkr, const CUtensorMap& tk,
+                     const CUtensorMap& tv, const FwdParams& P, cudaStream_t stream) {
+  if (path == Path::Window)
+    attn_fwd_swa_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tkr, tk, tv, P);
+  else
+    attn_fwd_pipelined_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tkr, tk, tv, P);
+}
 
 // Kernel timing: while enabled, each forward records an event pair around its
 // attention kernel (library-owned events, per device, reused across sessions).
@@ -139,8 +181,7 @@ std::pair<cudaEvent_t, cudaEvent_t>* profile_slot(int dev) {
 
 struct DeviceInfo {
   int sms = 0;
-  bool simple_ready = false;
-  bool pipelined_ready = false;
+  bool kernels_ready = false;  // dynamic shared memory limits raised
   cudaMemPool_t pool = nullptr;  // stream-ordered scratch, kept by the library (never released to the OS)
 };
 
@@ -152,11 +193,7 @@ DeviceInfo* device_info(int dev) {
   DeviceInfo& d = infos[dev];
   if (d.sms == 0) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
-    d.simple_ready = cudaFuncSetAttribute(attn_fwd_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          simple::kSmemBytes) == cudaSuccess;
-    d.pipelined_ready = cudaFuncSetAttribute(attn_fwd_pipelined_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             pipe::kSmemBytes) == cudaSuccess;
+    d.kernels_ready = set_smem_attributes();
     cudaMemPoolProps props;
     std::memset(&props, 0, sizeof props);
     props.allocType = cudaMemAllocationTypePinned;
@@ -178,21 +215,21 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& P, cuda
   DeviceInfo* info = device_info(dev);
   if (!info) return MIMO_ERR_CUDA;
   if (P.max_seqlen == 0) return MIMO_OK;
-  const int choice = g_kernel_choice.load();
-  const bool pipelined = (choice == MIMO_KERNEL_PIPELINED) || (choice == MIMO_KERNEL_AUTO && P.group % 2 == 0);
-  if (pipelined && P.group % 2 != 0) return MIMO_ERR_UNSUPPORTED;
+  Path path;
+  if (const int sel = select_path(P, path); sel != MIMO_OK) return sel;
+  const bool two_head = path != Path::Simple;
   CUtensorMap tq, tk, tv;
   if (!encode_2d(&tq, q, (uint64_t)P.hq * kHeadDimQK, P.total_tokens) ||
       !encode_2d(&tk, k, (uint64_t)P.hkv * kHeadDimQK, P.total_tokens) ||
-      !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, P.total_tokens, pipelined ? 64 : 128))
+      !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, P.total_tokens, two_head ? 64 : 128))
     return MIMO_ERR_CUDA;
-  if (!pipelined) {
-    if (!info->simple_ready) return MIMO_ERR_CUDA;
+  if (!info->kernels_ready) return MIMO_ERR_CUDA;
+  if (!two_head) {
     dim3 grid((P.max_seqlen + kBlockM - 1) / kBlockM, P.num_seqs, P.hq);
     attn_fwd_simple_kernel<<<grid, simple::kThreads, simple::kSmemBytes, stream>>>(tq, tk, tv, P);
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
   }
-  if (!info->pipelined_ready || !info->pool) return MIMO_ERR_CUDA;
+  if (!info->pool) return MIMO_ERR_CUDA;
   // K's rope dims, rotated once: transient scratch from the library's stream-ordered pool
   const size_t kr_rows = (size_t)P.total_tokens * P.hkv;
   void* k_rope = nullptr;
@@ -215,11 +252,9 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& P, cuda
                                   CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     st = MIMO_ERR_CUDA;
   if (st == MIMO_OK) {
-    const long long units = (long long)(P.hq / 2) * ((P.total_tokens + kBlockM - 1) / kBlockM + P.num_seqs);
-    const int grid = (int)std::min<long long>(units, info->sms);
     auto* ev = profile_slot(dev);
     if (ev) cudaEventRecord(ev->first, stream);
-    attn_fwd_pipelined_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tkr, tk, tv, P);
+    launch_two_head(path, persistent_grid(P, info->sms), tq, tkr, tk, tv, P, stream);
     if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
     if (ev) cudaEventRecord(ev->second, stream);
   }
@@ -268,12 +303,7 @@ NoAllocInfo* noalloc_info(int dev) {
   NoAllocInfo& d = infos[dev];
   if (!d.ready) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
-    if (cudaFuncSetAttribute(attn_fwd_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             simple::kSmemBytes) != cudaSuccess)
-      return nullptr;
-    if (cudaFuncSetAttribute(attn_fwd_pipelined_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pipe::kSmemBytes) != cudaSuccess)
-      return nullptr;
+    if (!set_smem_attributes()) return nullptr;
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return nullptr;
     d.scratch = ptr;
@@ -285,9 +315,9 @@ NoAllocInfo* noalloc_info(int dev) {
 int launch_noalloc(const void* q, const void* k, const void* v, const FwdParams& P, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
-  const int choice = g_kernel_choice.load();
-  const bool pipelined = (choice == MIMO_KERNEL_PIPELINED) || (choice == MIMO_KERNEL_AUTO && P.group % 2 == 0);
-  if (pipelined && P.group % 2 != 0) return MIMO_ERR_UNSUPPORTED;
+  Path path;
+  if (const int sel = select_path(P, path); sel != MIMO_OK) return sel;
+  const bool pipelined = path != Path::Simple;
   const size_t kr_rows = (size_t)P.total_tokens * P.hkv;
   if (pipelined && kr_rows * kRopeDims * 2 > kNoAllocScratchBytes) return MIMO_ERR_SCRATCH_LIMIT;
   NoAllocInfo* info = noalloc_info(dev);
@@ -321,9 +351,7 @@ int launch_noalloc(const void* q, const void* k, const void* v, const FwdParams&
   if (!encode_2d(&tkr, info->scratch, (uint64_t)P.hkv * kRopeDims, P.total_tokens, 128,
                  CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MIMO_ERR_CUDA;
-  const long long units = (long long)(P.hq / 2) * ((P.total_tokens + kBlockM - 1) / kBlockM + P.num_seqs);
-  const int grid = (int)std::min<long long>(units, info->sms);
-  attn_fwd_pipelined_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tkr, tk, tv, P);
+  launch_two_head(path, persistent_grid(P, info->sms), tq, tkr, tk, tv, P, stream);
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 
@@ -477,7 +505,7 @@ int mimo_attn_profile_stop(int* launches, double* total_ms) {
   return MIMO_OK;
 }
 
-int mimo_attn_version(void) { return (1 << 16) | 1; }
+int mimo_attn_version(void) { return (1 << 16) | 2; }
 
 int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* sink,
                           const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind, int window,
@@ -493,7 +521,8 @@ int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, const flo
 size_t mimo_attn_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 int mimo_attn_set_kernel(int choice) {
-  if (choice != MIMO_KERNEL_AUTO && choice != MIMO_KERNEL_SIMPLE && choice != MIMO_KERNEL_PIPELINED)
+  if (choice != MIMO_KERNEL_AUTO && choice != MIMO_KERNEL_SIMPLE && choice != MIMO_KERNEL_PIPELINED &&
+      choice != MIMO_KERNEL_WINDOW)
     return MIMO_ERR_INVALID_ARG;
   g_kernel_choice.store(choice);
   return MIMO_OK;

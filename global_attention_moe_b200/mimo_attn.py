@@ -22,7 +22,7 @@ SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host
            "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_fwd_noalloc",
            "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_profile_start",
            "mimo_attn_profile_stop", "mimo_attn_version")
-KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED = 0, 1, 2
+KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED, KERNEL_WINDOW = 0, 1, 2, 3
 
 
 class Dims(ctypes.Structure):
@@ -83,7 +83,7 @@ def version() -> tuple[int, int]:
 
 
 def set_kernel(choice: int) -> None:
-    """Select the kernel mimo_attn_fwd launches (KERNEL_AUTO / KERNEL_SIMPLE / KERNEL_PIPELINED)."""
+    """Select the kernel mimo_attn_fwd launches (KERNEL_AUTO / _SIMPLE / _PIPELINED / _WINDOW)."""
     st = LIB.mimo_attn_set_kernel(int(choice))
     if st != OK:
         raise MimoAttnError(st, "mimo_attn_set_kernel")

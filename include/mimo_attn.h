@@ -102,7 +102,8 @@ typedef struct {
  * Rotated Q/K rope dims enter the tensor cores as FP16 (the pass-through dims
  * stay BF16), so |q|, |k| on the first 64 dims must stay below 2^15; a larger
  * rotated value is recorded as MIMO_ERR_RANGE for mimo_attn_check.
- * Scratch: when Hq/Hkv is even (the pipelined kernel), the call rotates K's
+ * Scratch: when a two-head kernel runs (Hq/Hkv even: the window or the
+ * pipelined kernel, see mimo_attn_set_kernel), the call rotates K's
  * rope dims once into T * Hkv * 128 bytes of transient device scratch taken
  * from a library-owned stream-ordered memory pool (cudaMallocFromPoolAsync on
  * `stream`, returned with cudaFreeAsync on the same stream; the pool keeps
@@ -186,22 +187,39 @@ MIMO_API int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, 
 /* Size in bytes of the fixed scratch array mimo_attn_fwd_noalloc uses. */
 MIMO_API size_t mimo_attn_noalloc_scratch_bytes(void);
 
-/* Kernel selection for mimo_attn_fwd (process-wide; default AUTO).
- *   MIMO_KERNEL_AUTO       pipelined kernel when Hq/Hkv is even, else the simple one
+/* Kernel selection for mimo_attn_fwd and mimo_attn_fwd_noalloc (process-wide;
+ * default AUTO).
+ *   MIMO_KERNEL_AUTO       WINDOW when Hq/Hkv is even and 0 <= window <= 128,
+ *                          PIPELINED when Hq/Hkv is even otherwise (the global
+ *                          layer, longer windows), else SIMPLE
  *   MIMO_KERNEL_SIMPLE     one CTA per (128-query tile, head), every step serialised;
  *                          any Hq/Hkv ratio (the cross-check path)
- *   MIMO_KERNEL_PIPELINED  warp-specialised persistent kernel, two heads per CTA;
- *                          Hq/Hkv must be even (else mimo_attn_fwd returns
- *                          MIMO_ERR_UNSUPPORTED)
- * Returns MIMO_ERR_INVALID_ARG for any other value.  Both kernels compute the
- * same operation with the same rounding steps. */
-typedef enum { MIMO_KERNEL_AUTO = 0, MIMO_KERNEL_SIMPLE = 1, MIMO_KERNEL_PIPELINED = 2 } mimo_kernel_choice;
+ *   MIMO_KERNEL_PIPELINED  warp-specialised persistent kernel, two heads per CTA,
+ *                          online softmax over any number of key tiles;
+ *                          Hq/Hkv must be even
+ *   MIMO_KERNEL_WINDOW     the same roles, specialised for sliding windows of at
+ *                          most 128 keys: both key tiles of a query tile are
+ *                          scored first and softmaxed in one pass; Hq/Hkv must be
+ *                          even and the call a sliding-window one with
+ *                          window <= 128
+ * A forced choice whose condition fails makes the call return
+ * MIMO_ERR_UNSUPPORTED.  Returns MIMO_ERR_INVALID_ARG for any other value.
+ * All kernels compute the same operation; they differ only in the order of
+ * floating-point rounding (where the softmax maximum is taken and when it is
+ * applied), well inside the stated tolerances. */
+typedef enum {
+  MIMO_KERNEL_AUTO = 0,
+  MIMO_KERNEL_SIMPLE = 1,
+  MIMO_KERNEL_PIPELINED = 2,
+  MIMO_KERNEL_WINDOW = 3
+} mimo_kernel_choice;
 MIMO_API int mimo_attn_set_kernel(int choice);
 
 /*
  * Kernel timing for measurement tools.  After mimo_attn_profile_start, every
- * forward that runs the pipelined kernel records a CUDA event pair (events
- * owned by the library) around that kernel on the call's stream.
+ * forward that runs a two-head kernel (window or pipelined) records a CUDA
+ * event pair (events owned by the library) around that kernel on the call's
+ * stream.
  * mimo_attn_profile_stop ends recording, waits for the recorded events, and
  * returns how many attention-kernel launches were recorded and their summed
  * duration in milliseconds (the K RoPE pre-pass is excluded).  Process-wide.

@@ -19,16 +19,36 @@ def _cuda():
     assert mimo_attn.check() == mimo_attn.OK
 
 
-@pytest.fixture(params=["auto", "simple"])
+KERNELS = {"auto": 0, "simple": 1, "pipelined": 2, "window": 3}
+_current = {"kernel": "auto"}
+
+
+@pytest.fixture(params=["auto", "simple", "pipelined"])
 def kernel(request):
-    """Run a test with the default kernel choice and again with the serialised cross-check kernel."""
+    """Run a test with the default kernel choice (the window kernel for short
+    sliding windows, the pipelined one otherwise), with the serialised
+    cross-check kernel, and with the pipelined kernel forced."""
     from global_attention_moe_b200 import mimo_attn
-    mimo_attn.set_kernel(mimo_attn.KERNEL_SIMPLE if request.param == "simple" else mimo_attn.KERNEL_AUTO)
+    mimo_attn.set_kernel(KERNELS[request.param])
+    _current["kernel"] = request.param
     yield request.param
     mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
+    _current["kernel"] = "auto"
+
+
+def kernel_supports(name: str, w) -> bool:
+    """Shapes a forced kernel choice accepts (the C ABI returns UNSUPPORTED otherwise)."""
+    even = (w.num_q_heads // w.num_kv_heads) % 2 == 0
+    if name == "pipelined":
+        return even
+    if name == "window":
+        return even and w.layer_kind == W.LAYER_SWA and 0 <= w.window <= 128
+    return True
 
 
 def full_parity(w):
+    if not kernel_supports(_current["kernel"], w):
+        pytest.skip(f"{_current['kernel']} kernel does not take this shape")
     x = W.make_inputs(w)
     out, lse = run_gpu(w, x)
     ref_out, ref_lse = run_oracle(w, x)
@@ -184,3 +204,62 @@ def test_kernels_agree_closely():
     o2, l2 = run_gpu(w, x, dev_inputs=dev)
     assert float((o1.float() - o2.float()).abs().max()) < 1e-2
     assert float((l1 - l2).abs().max()) < 2e-4
+
+
+def test_window_and_pipelined_kernels_agree():
+    """The window kernel (both key tiles scored, one softmax pass) and the
+    pipelined kernel (online softmax over key tiles) both meet the oracle
+    tolerances on the same inputs, and their mutual difference stays within
+    the same bounds.  (P is rounded to BF16 at different scales -- the row max
+    versus a lazily updated running max -- so they are not bit-identical.)"""
+    from global_attention_moe_b200 import mimo_attn
+    w = W.custom("agree_swa", W.LAYER_SWA, [700, 129, 1, 300], 8, 2, 128, 1e4, True, seed=12)
+    x = W.make_inputs(w)
+    dev = to_device(x)
+    ref_out, ref_lse = run_oracle(w, x)
+    res = {}
+    for name in ("pipelined", "window"):
+        mimo_attn.set_kernel(KERNELS[name])
+        try:
+            o, l = run_gpu(w, x, dev_inputs=dev)
+        finally:
+            mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
+        res[name] = (out_to_f64(o), l.cpu().numpy().astype(np.float64))
+        assert_within(errors(*res[name], ref_out, ref_lse), name)
+    mutual = errors(*res["window"], *res["pipelined"])
+    print("window vs pipelined:", mutual)
+    assert_within(mutual, "window vs pipelined")
+
+
+@pytest.mark.parametrize("layer,window,hq,hkv", [(W.LAYER_GLOBAL, -1, 8, 2), (W.LAYER_SWA, 129, 8, 2),
+                                                 (W.LAYER_SWA, 128, 8, 8)])
+def test_forced_window_kernel_rejects_other_shapes(layer, window, hq, hkv):
+    """Forcing the window kernel on a shape it does not take returns UNSUPPORTED
+    before anything is launched."""
+    from global_attention_moe_b200 import mimo_attn
+    w = W.custom("reject", layer, [300], hq, hkv, window, 1e4 if layer == W.LAYER_SWA else 1e7,
+                 layer == W.LAYER_SWA, seed=13)
+    x = W.make_inputs(w)
+    dev = to_device(x)
+    mimo_attn.set_kernel(mimo_attn.KERNEL_WINDOW)
+    try:
+        with pytest.raises(mimo_attn.MimoAttnError) as e:
+            run_gpu(w, x, dev_inputs=dev)
+        assert e.value.status == mimo_attn.ERR_UNSUPPORTED
+    finally:
+        mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
+    assert mimo_attn.check() == mimo_attn.OK
+
+
+@pytest.mark.parametrize("window", [0, 1, 31, 32, 33, 64, 96, 127, 128])
+@pytest.mark.parametrize("lengths", [[1000], [1, 128, 129, 383, 5]])
+def test_window_kernel_windows(window, lengths):
+    """The window kernel across windows that move the run's chunk boundaries."""
+    from global_attention_moe_b200 import mimo_attn
+    mimo_attn.set_kernel(mimo_attn.KERNEL_WINDOW)
+    try:
+        _current["kernel"] = "window"
+        full_parity(W.custom("wwin", W.LAYER_SWA, lengths, 4, 2, window, 1e4, window % 2 == 0, seed=14))
+    finally:
+        _current["kernel"] = "auto"
+        mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
