@@ -581,12 +581,12 @@ __device__ void role_rope(uint8_t* smem, Ctrl* C, const FwdParams& P, int r) {
     named_bar_sync(kRopeBarId, 128);
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
-      if (!pwait(C, &C->q_full[h], n_u & 1, lim)) ok = false;
-      if (ok) {
+      const bool got = pwait(C, &C->q_full[h], n_u & 1, lim);
+      if (got) {
         amax = fmaxf(amax, rope_row_rotate(smem + kQOff + 3 * h * kUnit, r, C->base_q, oc, os));
         fence_proxy_async_smem();
       }
-      named_bar_sync(kRopeBarId, 128);
+      ok = named_bar_and(kRopeBarId, 128, got);  // every thread leaves together once any wait fails
       if (!ok) break;
       if (r == 0) mbar_arrive(&C->q_roped[h]);
     }

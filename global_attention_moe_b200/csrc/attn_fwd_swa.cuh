@@ -71,16 +71,19 @@ struct BlockUnits {
     pair = tiles ? static_cast<uint32_t>(u0 / tiles) : 0u;
     ti = tiles ? static_cast<uint32_t>(u0 % tiles) : 0u;
   }
+  // After a call, W describes the returned unit's sequence (b, s_b, L) until the next call.
   __device__ __forceinline__ bool next(int& q0, int& h0) {
-    if (left == 0 || !W.seek(ti)) return false;
-    q0 = static_cast<int>(ti - W.tile_base) * kBlockM;
-    h0 = 2 * static_cast<int>(pair);
-    --left;
-    if (++ti == tiles) {  // next head pair: walk the sequences again
+    if (left == 0) return false;
+    if (ti == tiles) {  // next head pair: walk the sequences again
       ti = 0;
       ++pair;
       W.reset();
     }
+    if (!W.seek(ti)) return false;
+    q0 = static_cast<int>(ti - W.tile_base) * kBlockM;
+    h0 = 2 * static_cast<int>(pair);
+    --left;
+    ++ti;
     return true;
   }
 };
