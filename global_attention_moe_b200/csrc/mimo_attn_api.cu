@@ -18,6 +18,7 @@
 #include "attn_fwd_pipelined.cuh"
 #include "attn_fwd_simple.cuh"
 #include "attn_fwd_swa.cuh"
+#include "attn_decode.cuh"
 #include "rope_k_prepass.cuh"
 #include "params.cuh"
 
@@ -131,7 +132,9 @@ bool set_smem_attributes() {
          cudaFuncSetAttribute(attn_fwd_pipelined_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               pipe::kSmemBytes) == cudaSuccess &&
          cudaFuncSetAttribute(attn_fwd_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              pipe::kSmemBytes) == cudaSuccess;
+                              pipe::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(dec::attn_decode_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              dec::kSmemBytes) == cudaSuccess;
 }
 
 // Persistent grid of the two-head kernels: one CTA per SM, at most one per unit.
@@ -355,9 +358,115 @@ int launch_noalloc(const void* q, const void* k, const void* v, const FwdParams&
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 
+int validate_decode(const void* q, const void* kc, const void* vc, const int32_t* idx, const int32_t* indptr,
+                    const int32_t* cu_q, const float* sink, const mimo_decode_dims* d, int layer_kind, int window,
+                    double rope_base, int rope_dims, float v_scale, const void* out, const float* lse) {
+  if (!d) return MIMO_ERR_INVALID_ARG;
+  if (layer_kind != MIMO_LAYER_SWA && layer_kind != MIMO_LAYER_GLOBAL) return MIMO_ERR_INVALID_ARG;
+  if (d->num_seqs < 1 || d->total_q < 0 || d->total_kv < 0 || d->cache_rows < 0 || d->max_q_len < 0 ||
+      d->max_kv_len < 0 || d->num_q_heads < 1 || d->num_kv_heads < 1)
+    return MIMO_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads != 0) return MIMO_ERR_INVALID_ARG;
+  if (d->max_q_len > d->max_kv_len || d->max_q_len > d->total_q || d->max_kv_len > d->total_kv)
+    return MIMO_ERR_INVALID_ARG;
+  if (d->total_kv > 0 && d->cache_rows < 1) return MIMO_ERR_INVALID_ARG;
+  if (d->head_dim_qk < 1 || d->head_dim_v < 1) return MIMO_ERR_INVALID_ARG;
+  if (d->head_dim_qk != kHeadDimQK || d->head_dim_v != kHeadDimV) return MIMO_ERR_UNSUPPORTED;
+  if (rope_dims < 0 || rope_dims % 2 != 0 || rope_dims > d->head_dim_qk) return MIMO_ERR_INVALID_ARG;
+  if (rope_dims != kRopeDims) return MIMO_ERR_UNSUPPORTED;
+  if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return MIMO_ERR_INVALID_ARG;
+  if (!std::isfinite(v_scale)) return MIMO_ERR_INVALID_ARG;
+  if (layer_kind == MIMO_LAYER_SWA && window < 0) return MIMO_ERR_INVALID_ARG;
+  if (layer_kind == MIMO_LAYER_GLOBAL && sink != nullptr) return MIMO_ERR_INVALID_ARG;
+  if ((int64_t)d->max_q_len * (d->num_q_heads / d->num_kv_heads) > dec::kMaxRows) return MIMO_ERR_UNSUPPORTED;
+  if ((int64_t)d->cache_rows * d->num_kv_heads * kHeadDimQK > INT64_C(1) << 40) return MIMO_ERR_UNSUPPORTED;
+  if (!indptr || !cu_q) return MIMO_ERR_INVALID_ARG;
+  if (d->total_q > 0) {
+    if (!q || !out || !lse || (d->total_kv > 0 && (!kc || !vc || !idx))) return MIMO_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || (kc && !aligned16(kc)) || (vc && !aligned16(vc)))
+      return MIMO_ERR_INVALID_ARG;
+  }
+  if (sink && (reinterpret_cast<uintptr_t>(sink) & 3u)) return MIMO_ERR_INVALID_ARG;
+  return MIMO_OK;
+}
+
+int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* idx, const int32_t* indptr,
+                  const int32_t* cu_q, const float* sink, const mimo_decode_dims* d, int layer_kind, int window,
+                  double rope_base, float v_scale, void* out, float* lse, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
+  DeviceInfo* info = device_info(dev);
+  if (!info || !info->kernels_ready || !info->pool) return MIMO_ERR_CUDA;
+  dec::DecParams P;
+  std::memset(&P, 0, sizeof P);
+  P.q = static_cast<const uint16_t*>(q);
+  P.k_cache = static_cast<const uint16_t*>(kc);
+  P.v_cache = static_cast<const uint16_t*>(vc);
+  P.kv_indices = idx;
+  P.kv_indptr = indptr;
+  P.cu_q = cu_q;
+  P.sink = sink;
+  P.out = static_cast<uint16_t*>(out);
+  P.lse = lse;
+  P.num_seqs = d->num_seqs;
+  P.total_q = d->total_q;
+  P.total_kv = d->total_kv;
+  P.cache_rows = d->cache_rows;
+  P.hq = d->num_q_heads;
+  P.hkv = d->num_kv_heads;
+  P.group = d->num_q_heads / d->num_kv_heads;
+  P.window = (layer_kind == MIMO_LAYER_GLOBAL) ? -1 : window;
+  P.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDimQK)));
+  P.v_scale = v_scale;
+  for (int i = 0; i < kRopeDims / 2; ++i) P.theta[i] = std::pow(rope_base, -2.0 * i / kRopeDims);
+  // Keys one sequence's queries can see, at most; split them so that about two CTAs run per SM.
+  const long long span = (P.window >= 0) ? std::min<long long>(d->max_kv_len, (long long)P.window + d->max_q_len)
+                                         : (long long)d->max_kv_len;
+  const long long base_ctas = (long long)d->num_seqs * P.hkv;
+  long long splits = std::max<long long>(1, (2LL * info->sms + base_ctas - 1) / base_ctas);
+  splits = std::min<long long>(splits, std::max<long long>(1, (span + 63) / 64));
+  long long split_keys = (span + splits - 1) / splits;
+  split_keys = std::max<long long>(dec::kChunk, (split_keys + dec::kChunk - 1) / dec::kChunk * dec::kChunk);
+  splits = std::max<long long>(1, (span + split_keys - 1) / split_keys);
+  if (splits > 65535 || d->num_seqs > 65535 || P.hkv > 65535) return MIMO_ERR_UNSUPPORTED;  // grid limits
+  P.splits = (int)splits;
+  P.split_keys = (int)split_keys;
+  const size_t slots = (size_t)d->total_q * P.hq * splits;
+  void* part = nullptr;
+  if (cudaMallocFromPoolAsync(&part, slots * (kHeadDimV * 4 + 8), info->pool, stream) != cudaSuccess)
+    return MIMO_ERR_CUDA;
+  P.part_o = static_cast<float*>(part);
+  P.part_ml = P.part_o + slots * kHeadDimV;
+  int st = MIMO_OK;
+  dim3 grid((unsigned)splits, (unsigned)P.hkv, (unsigned)d->num_seqs);
+  dec::attn_decode_partial_kernel<<<grid, dec::kThreads, dec::kSmemBytes, stream>>>(P);
+  if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+  const long long warps = (long long)d->total_q * P.hq;
+  if (st == MIMO_OK) {
+    dec::attn_decode_combine_kernel<<<(unsigned)((warps * 32 + dec::kThreads - 1) / dec::kThreads), dec::kThreads,
+                                      0, stream>>>(P);
+    if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+  }
+  if (cudaFreeAsync(part, stream) != cudaSuccess) st = MIMO_ERR_CUDA;
+  return st;
+}
+
 }  // namespace
 
 extern "C" {
+
+int mimo_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_indices,
+                     const int32_t* kv_indptr, const int32_t* cu_q, const float* sink, const mimo_decode_dims* dims,
+                     int layer_kind, int window, double rope_base, int rope_dims, float v_scale, void* out,
+                     float* lse, void* stream) {
+  int st = validate_decode(q, k_cache, v_cache, kv_indices, kv_indptr, cu_q, sink, dims, layer_kind, window,
+                           rope_base, rope_dims, v_scale, out, lse);
+  if (st != MIMO_OK) return st;
+  if (dims->total_q == 0) return MIMO_OK;
+  return launch_decode(q, k_cache, v_cache, kv_indices, kv_indptr, cu_q, sink, dims, layer_kind, window, rope_base,
+                       v_scale, out, lse, static_cast<cudaStream_t>(stream));
+}
+
 
 int mimo_attn_fwd(const void* q, const void* k, const void* v, const float* sink, const int32_t* cu_seqlens,
                   const mimo_attn_dims* dims, int layer_kind, int window, double rope_base, int rope_dims,
@@ -505,7 +614,7 @@ int mimo_attn_profile_stop(int* launches, double* total_ms) {
   return MIMO_OK;
 }
 
-int mimo_attn_version(void) { return (1 << 16) | 2; }
+int mimo_attn_version(void) { return (1 << 16) | 3; }
 
 int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* sink,
                           const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind, int window,

@@ -21,12 +21,19 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BAD_
 SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host", "mimo_attn_check",
            "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_fwd_noalloc",
            "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_profile_start",
-           "mimo_attn_profile_stop", "mimo_attn_version")
+           "mimo_attn_profile_stop", "mimo_attn_decode", "mimo_attn_version")
 KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED, KERNEL_WINDOW = 0, 1, 2, 3
 
 
 class Dims(ctypes.Structure):
     _fields_ = [("num_seqs", ctypes.c_int32), ("total_tokens", ctypes.c_int32), ("max_seqlen", ctypes.c_int32),
+                ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim_qk", ctypes.c_int32), ("head_dim_v", ctypes.c_int32)]
+
+
+class DecodeDims(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("total_q", ctypes.c_int32), ("total_kv", ctypes.c_int32),
+                ("cache_rows", ctypes.c_int32), ("max_q_len", ctypes.c_int32), ("max_kv_len", ctypes.c_int32),
                 ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("head_dim_qk", ctypes.c_int32), ("head_dim_v", ctypes.c_int32)]
 
@@ -65,6 +72,8 @@ def _load():
     lib.mimo_attn_profile_stop.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
     lib.mimo_attn_set_kernel.restype = I
     lib.mimo_attn_set_kernel.argtypes = [I]
+    lib.mimo_attn_decode.restype = I
+    lib.mimo_attn_decode.argtypes = [P, P, P, P, P, P, P, ctypes.POINTER(DecodeDims), I, I, D, I, F, P, P, P]
     lib.mimo_attn_version.restype = I
     lib.mimo_attn_version.argtypes = []
     return lib
@@ -187,3 +196,42 @@ def check(stream=None) -> int:
 
 def selftest_wait_timeout(limit_ns: int, stream=None) -> int:
     return LIB.mimo_attn_selftest_wait_timeout(int(limit_ns), _stream_handle(stream))
+
+
+def make_decode_dims(num_seqs, total_q, total_kv, cache_rows, max_q_len, max_kv_len, hq, hkv, dqk=192,
+                     dv=128) -> DecodeDims:
+    return DecodeDims(int(num_seqs), int(total_q), int(total_kv), int(cache_rows), int(max_q_len),
+                      int(max_kv_len), int(hq), int(hkv), int(dqk), int(dv))
+
+
+def decode_raw(q_ptr, kc_ptr, vc_ptr, idx_ptr, indptr_ptr, cuq_ptr, sink_ptr, dims: DecodeDims, layer_kind, window,
+               rope_base, rope_dims, v_scale, out_ptr, lse_ptr, stream_handle) -> int:
+    """Direct C-ABI call of mimo_attn_decode with integer device pointers; returns the status code."""
+    return LIB.mimo_attn_decode(q_ptr, kc_ptr, vc_ptr, idx_ptr, indptr_ptr, cuq_ptr, sink_ptr, ctypes.byref(dims),
+                                int(layer_kind), int(window), float(rope_base), int(rope_dims), float(v_scale),
+                                out_ptr, lse_ptr, stream_handle)
+
+
+def decode(q, k_cache, v_cache, kv_indices, kv_indptr, cu_q, sink, max_q_len, max_kv_len, layer_kind, window,
+           rope_base, rope_dims=64, v_scale=0.707, out=None, lse=None, stream=None):
+    """New query tokens against a page-size-1 KV cache (CUDA tensors: bf16 q [Tq, Hq, 192], bf16 caches
+    [rows, Hkv, 192] / [rows, Hkv, 128], int32 kv_indices / kv_indptr / cu_q, fp32 sink or None).
+    Returns (out bf16 [Tq, Hq, 128], lse fp32 [Hq, Tq])."""
+    import torch
+    Tq, hq, dqk = q.shape
+    rows, hkv, dv = v_cache.shape
+    for t in (q, k_cache, v_cache):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("q and the caches must be contiguous bf16 CUDA tensors")
+    if out is None:
+        out = torch.empty((Tq, hq, dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((hq, Tq), dtype=torch.float32, device=q.device)
+    dims = make_decode_dims(cu_q.numel() - 1, Tq, kv_indices.numel(), rows, max_q_len, max_kv_len, hq, hkv, dqk, dv)
+    st = decode_raw(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), kv_indices.data_ptr(),
+                    kv_indptr.data_ptr(), cu_q.data_ptr(), sink.data_ptr() if sink is not None else None, dims,
+                    layer_kind, window, rope_base, rope_dims, v_scale, out.data_ptr(), lse.data_ptr(),
+                    _stream_handle(stream))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_attn_decode")
+    return out, lse

@@ -31,7 +31,7 @@ import numpy as np
 GOLDEN_GAMMA = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
-STREAM_LENGTHS, STREAM_Q, STREAM_K, STREAM_V, STREAM_SINK = 0, 1, 2, 3, 4
+STREAM_LENGTHS, STREAM_Q, STREAM_K, STREAM_V, STREAM_SINK, STREAM_PAGES = 0, 1, 2, 3, 4, 5
 _STREAM_SHIFT = 40
 _CHUNK = 1 << 22
 

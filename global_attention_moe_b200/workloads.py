@@ -150,3 +150,40 @@ def make_inputs(w: Workload, threads: int | None = None) -> Inputs:
 
 def custom(name, layer_kind, lengths, hq, hkv, window, rope_base, has_sink, seed=0, v_scale=V_SCALE) -> Workload:
     return Workload(name, layer_kind, list(lengths), hq, hkv, window, rope_base, has_sink, seed, v_scale=v_scale)
+
+
+# ---------------------------------------------------------------- KV-cache attention
+@dataclass
+class DecodeInputs:
+    """One batch of new tokens against a page-size-1 KV cache (host arrays).
+
+    Sequence b has kv_lens[b] cached tokens (the last q_lens[b] of them new), whose
+    cache rows are kv_indices[kv_indptr[b]:kv_indptr[b+1]] in position order; q holds
+    the new tokens' queries, THD-packed by cu_q."""
+    q: np.ndarray          # uint16 BF16 bits [Tq, Hq, 192]
+    k_cache: np.ndarray    # uint16 [rows, Hkv, 192]
+    v_cache: np.ndarray    # uint16 [rows, Hkv, 128]
+    kv_indices: np.ndarray  # int32 [total_kv]
+    kv_indptr: np.ndarray   # int32 [B+1]
+    cu_q: np.ndarray        # int32 [B+1]
+    sink: np.ndarray | None
+    q_lens: list
+    kv_lens: list
+
+
+def make_decode_inputs(kv_lens, q_lens, hq, hkv, has_sink, seed, spare_rows=64, threads=None) -> DecodeInputs:
+    """Seeded decode problem: cache rows are a random permutation (page size 1), with spare rows
+    that no sequence uses."""
+    kv_lens = [int(x) for x in kv_lens]
+    q_lens = [int(x) for x in q_lens]
+    total_kv = sum(kv_lens)
+    rows = total_kv + spare_rows
+    q = synth.normal_bf16(seed, synth.STREAM_Q, (sum(q_lens), hq, 192), threads)
+    k = synth.normal_bf16(seed, synth.STREAM_K, (rows, hkv, 192), threads)
+    v = synth.normal_bf16(seed, synth.STREAM_V, (rows, hkv, 128), threads)
+    perm = np.argsort(synth.uniforms(seed, synth.STREAM_PAGES, rows), kind="stable").astype(np.int32)
+    kv_indices = perm[:total_kv].copy()
+    kv_indptr = np.concatenate([[0], np.cumsum(kv_lens)]).astype(np.int32)
+    cu_q = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    sink = synth.normal_f32(seed, synth.STREAM_SINK, hq) if has_sink else None
+    return DecodeInputs(q, k, v, kv_indices, kv_indptr, cu_q, sink, q_lens, kv_lens)

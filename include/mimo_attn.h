@@ -227,6 +227,45 @@ MIMO_API int mimo_attn_set_kernel(int choice);
 MIMO_API int mimo_attn_profile_start(void);
 MIMO_API int mimo_attn_profile_stop(int* launches, double* total_ms);
 
+/*
+ * Attention of new query tokens against a KV cache with page size 1: decode,
+ * speculative-draft verification and chunked prefill for the same two layer
+ * kinds (miles docs "MiMo-V2.6-Flash" section 3.2 SGLang: page size 1,
+ * chunked prefill of up to 49152 tokens, 8 speculative draft tokens).
+ *
+ *   q           bf16 [total_q, Hq, 192]   (device) the new tokens of every
+ *               sequence, THD-packed by cu_q
+ *   k_cache     bf16 [cache_rows, Hkv, 192] (device) K as mimo_attn_fwd takes it
+ *               (not rotated); v_cache bf16 [cache_rows, Hkv, 128]
+ *   kv_indices  int32 [total_kv]          (device) cache row of every key:
+ *               sequence b's keys, in position order, are entries
+ *               kv_indptr[b] .. kv_indptr[b+1]-1; the new tokens' K and V
+ *               are already in the cache (the last q_len_b entries)
+ *   kv_indptr   int32 [num_seqs + 1]      (device) kv_indptr[0] = 0, nondecreasing
+ *   cu_q        int32 [num_seqs + 1]      (device) cu_q[0] = 0, cu_q[B] = total_q
+ *   sink, layer_kind, window, rope_base, rope_dims, v_scale: as mimo_attn_fwd
+ *   out         bf16 [total_q, Hq, 128]   (device); lse fp32 [Hq, total_q] (device)
+ * Query i of sequence b (1 <= q_len_b <= kv_len_b) sits at position
+ * kv_len_b - q_len_b + i and attends the keys mimo_attn_fwd would give it, so
+ * out and lse equal the forward's rows for those positions.  Needs
+ * max_q_len * Hq/Hkv <= 128 (else MIMO_ERR_UNSUPPORTED); every q_len_b,
+ * kv_len_b must be at most max_q_len, max_kv_len.  Inconsistent cu_q /
+ * kv_indptr, q_len_b > kv_len_b and cache rows outside [0, cache_rows) are
+ * recorded as MIMO_ERR_BAD_SEQLENS for mimo_attn_check (such rows are left
+ * unwritten; an index outside the cache is never dereferenced).  Scratch: a
+ * partial result per key split, total_q * Hq * splits * 520 bytes from the
+ * library's stream-ordered pool.  Does not synchronise.  (The pages give no
+ * interface; this one mirrors mimo_attn_fwd.)
+ */
+typedef struct {
+  int32_t num_seqs, total_q, total_kv, cache_rows, max_q_len, max_kv_len;
+  int32_t num_q_heads, num_kv_heads, head_dim_qk, head_dim_v;
+} mimo_decode_dims;
+MIMO_API int mimo_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_indices,
+                              const int32_t* kv_indptr, const int32_t* cu_q, const float* sink,
+                              const mimo_decode_dims* dims, int layer_kind, int window, double rope_base,
+                              int rope_dims, float v_scale, void* out, float* lse, void* stream);
+
 /* ABI version: (major << 16) | minor. */
 MIMO_API int mimo_attn_version(void);
 

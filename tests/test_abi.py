@@ -119,3 +119,27 @@ def test_kernel_choice_values(M):
             M.set_kernel(bad)
         assert e.value.status == M.ERR_INVALID_ARG
     M.set_kernel(M.KERNEL_AUTO)
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(hq=6, hkv=4), 1),                 # Hq % Hkv != 0
+    (dict(max_q_len=9, total_q=20, hq=64, hkv=4), 2),  # 9 x 16 rows per KV head > 128
+    (dict(max_q_len=20, max_kv_len=10), 1), # max_q_len > max_kv_len
+    (dict(cache_rows=0), 1),                # keys but no cache
+    (dict(dqk=128), 2),
+    (dict(rope_dims=32), 2),
+    (dict(window=-1), 1),
+    (dict(layer=1, sink=FAKE), 1),
+    (dict(q=FAKE + 8), 1),
+])
+def test_decode_validation_rejects(M, case, expect):
+    d = dict(num_seqs=2, total_q=4, total_kv=100, cache_rows=128, max_q_len=2, max_kv_len=60, hq=8, hkv=2,
+             dqk=192, dv=128)
+    args = dict(layer=0, window=128, rope_dims=64, sink=None, q=FAKE)
+    for key in list(case):
+        (d if key in d else args)[key] = case[key]
+    dims = M.make_decode_dims(d["num_seqs"], d["total_q"], d["total_kv"], d["cache_rows"], d["max_q_len"],
+                              d["max_kv_len"], d["hq"], d["hkv"], d["dqk"], d["dv"])
+    st = M.decode_raw(args["q"], FAKE, FAKE, FAKE, FAKE, FAKE, args["sink"], dims, args["layer"], args["window"],
+                      1e4, args["rope_dims"], 0.707, FAKE, FAKE, None)
+    assert st == expect
