@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--no-parity", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--ref-budget-s", type=float, default=90.0, help="reference arm: total CPU seconds to aim for")
+    ap.add_argument("--decode", choices=W.DECODE_KINDS, default=None,
+                    help="time the KV-cache path (64 requests x 8 new tokens) instead of the forward")
     return ap.parse_args()
 
 
@@ -461,8 +463,116 @@ def run_ours(args):
     return 0
 
 
+DECODE_METRIC = "KV-cache attention (page size 1) new tokens/s on 1 B200; % of HBM roofline"
+
+
+def decode_bytes_flops(x, window):
+    """Algorithmic bytes (K/V rows the queries can see, read once with their indices; q read, out
+    and lse written once) and FLOPs (640 per attended pair) of one KV-cache step."""
+    hq, hkv = x.q.shape[1], x.k_cache.shape[1]
+    keys = pairs = 0
+    for kv, q in zip(x.kv_lens, x.q_lens):
+        keys += min(kv, window + q) if window >= 0 else kv
+        for i in range(q):
+            p = kv - q + i
+            pairs += min(p + 1, window + 1) if window >= 0 else p + 1
+    Tq = x.q.shape[0]
+    nbytes = keys * (hkv * (192 + 128) * 2 + 4) + Tq * hq * (192 * 2 + 128 * 2 + 4)
+    return nbytes, FLOPS_PER_PAIR * pairs * hq
+
+
+def run_decode(args):
+    """The KV-cache path on a serving-shaped batch; one JSON line (single GPU)."""
+    import torch
+    import oracle
+    from global_attention_moe_b200 import mimo_attn
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    n_sets = 4 if args.decode == "swa" else 1  # the sliding layer's rows per step fit in L2: rotate
+    sets = []
+    for seed in range(n_sets):
+        x, layer, window, base = W.decode_batch(args.decode, seed=seed)
+        t = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+        dev = (t(x.q), t(x.k_cache), t(x.v_cache), i32(x.kv_indices), i32(x.kv_indptr), i32(x.cu_q),
+               None if x.sink is None else torch.from_numpy(x.sink).cuda())
+        out = torch.empty(x.q.shape[0], 64, 128, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(64, x.q.shape[0], dtype=torch.float32, device="cuda")
+        sets.append((x, dev, out, lse))
+    x0 = sets[0][0]
+    Tq = x0.q.shape[0]
+    set_bytes = sum(a.numel() * a.element_size() for a in sets[0][1] if a is not None)
+
+    def step(i):
+        x, (q, kc, vc, idx, indptr, cuq, sk), out, lse = sets[i % n_sets]
+        mimo_attn.decode(q, kc, vc, idx, indptr, cuq, sk, max(x.q_lens), max(x.kv_lens), layer, window, base,
+                         out=out, lse=lse)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    assert mimo_attn.check() == mimo_attn.OK
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.synchronize()
+        e0.record()
+        for i in range(args.steps):
+            step(i)
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    st = mimo_attn.check()
+    if st != mimo_attn.OK:
+        raise RuntimeError(mimo_attn.status_string(st))
+    # parity spot check and CPU baseline: the first two requests of set 0 through the oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from decode_helpers import decode_reference
+    sub = W.decode_subset(x0, [0, 1])
+    t0 = time.time()
+    ro, rl = decode_reference(sub, window, base)
+    cpu_s = time.time() - t0
+    step(0)
+    torch.cuda.synchronize()
+    rows = int(sub.q.shape[0])
+    g_out = sets[0][2][:rows].float().cpu().numpy().astype(np.float64)
+    g_lse = sets[0][3][:, :rows].cpu().numpy().astype(np.float64)
+    d = g_out - ro
+    parity = {"rows": rows, "max_abs": float(np.abs(d).max()), "rel_l2": float(np.linalg.norm(d) / np.linalg.norm(ro)),
+              "lse_max_abs": float(np.abs(g_lse - rl).max())}
+    nbytes, flops = decode_bytes_flops(x0, window)
+    peaks, peak_src = load_peaks()
+    ach = nbytes / (ms / 1e3) / 1e9
+    line = {
+        "metric": DECODE_METRIC, "value": Tq / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"decode_{args.decode}_B{len(x0.kv_lens)}_q{max(x0.q_lens)}_kv1024-8192",
+                   "layer": "swa_sink" if args.decode == "swa" else "global_causal", "requests": len(x0.kv_lens),
+                   "new_tokens": Tq, "context_tokens": int(sum(x0.kv_lens)), "q_heads": 64,
+                   "kv_heads": int(x0.k_cache.shape[1]), "page_size": 1,
+                   "l2": f"{n_sets} input sets rotated ({n_sets * set_bytes / 2**20:.0f} MiB on the device)"},
+        "tflops": flops / (ms / 1e3) / 1e12, "gbs": ach,
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peak_src} (burst)",
+                     "kernel": "attn_decode_partial_kernel + attn_decode_combine_kernel",
+                     "algorithmic_bytes": nbytes, "algorithmic_flops": flops},
+        "cpu_baseline": {"value": rows / cpu_s, "unit": "tokens/s", "cores": oracle.default_threads(),
+                         "kind": "oracle", "sample": f"the first two requests of the batch ({rows} new tokens)"},
+        "e2e": None,
+        "gpu_launches": args.steps * 2,
+        "clocks": clk.summary(),
+        "parity": parity,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.decode:
+        return run_decode(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -36,8 +36,9 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = 32;                        // keys per step, one per lane
 constexpr int kMaxRows = 128;                     // q_len x (Hq/Hkv) query rows per CTA
 constexpr int kRowsPerWarp = kMaxRows / kWarps;   // row r belongs to warp r % kWarps
-constexpr int kQStride = kHeadDimQK + 1;          // padded FP32 rows: lane-strided reads hit distinct banks
-constexpr int kKStride = kHeadDimQK + 1;
+constexpr int kQStride = kHeadDimQK;              // Q rows are read as broadcast 16-byte loads
+constexpr int kKStride = kHeadDimQK + 4;          // 16-byte aligned, lane stride of 4 banks: conflict-free
+constexpr int kDimsPerPass = 48;                  // key dims held in registers per pass of the score loop
 constexpr int kPStride = kChunk + 1;
 constexpr uint32_t kSmemBytes =
     (kMaxRows * kQStride + kChunk * kKStride + kChunk * kHeadDimV + kWarps * kRowsPerWarp * kPStride) * 4;
@@ -171,25 +172,47 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial_kernel(const __g
     }
     __syncthreads();
 
-    // scores: lane = key c0 + lane; the warp's rows
+    // scores: lane = key c0 + lane, against the warp's rows.  The key's dims sit in registers
+    // 48 at a time and every Q value comes from a broadcast 16-byte load, so the loop is bound by
+    // the FMA pipe rather than by shared-memory loads.
     const int j = c0 + lane;
-    const float* kr = sK + lane * kKStride;
+    float acc[kRowsPerWarp];
+#pragma unroll
+    for (int k = 0; k < kRowsPerWarp; ++k) acc[k] = 0.f;
+#pragma unroll 1
+    for (int d0 = 0; d0 < kHeadDimQK; d0 += kDimsPerPass) {
+      float4 kv[kDimsPerPass / 4];
+#pragma unroll
+      for (int c = 0; c < kDimsPerPass / 4; ++c)
+        kv[c] = *reinterpret_cast<const float4*>(sK + lane * kKStride + d0 + 4 * c);
+#pragma unroll
+      for (int k = 0; k < kRowsPerWarp; ++k) {
+        const int r = warp + kWarps * k;
+        if (r >= rows) break;  // warp-uniform
+        const float4* qr = reinterpret_cast<const float4*>(sQ + r * kQStride + d0);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < kDimsPerPass / 4; c += 2) {
+          const float4 x = qr[c], y = qr[c + 1];
+          a0 = fmaf(x.x, kv[c].x, a0);
+          a0 = fmaf(x.y, kv[c].y, a0);
+          a0 = fmaf(x.z, kv[c].z, a0);
+          a0 = fmaf(x.w, kv[c].w, a0);
+          a1 = fmaf(y.x, kv[c + 1].x, a1);
+          a1 = fmaf(y.y, kv[c + 1].y, a1);
+          a1 = fmaf(y.z, kv[c + 1].z, a1);
+          a1 = fmaf(y.w, kv[c + 1].w, a1);
+        }
+        acc[k] += a0 + a1;
+      }
+    }
 #pragma unroll
     for (int k = 0; k < kRowsPerWarp; ++k) {  // unrolled: the per-row state stays in registers
       const int r = warp + kWarps * k;
       if (r >= rows) break;  // warp-uniform
-      const float* qr = sQ + r * kQStride;
-      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll 4
-      for (int d = 0; d < kHeadDimQK; d += 4) {
-        acc0 = fmaf(qr[d], kr[d], acc0);
-        acc1 = fmaf(qr[d + 1], kr[d + 1], acc1);
-        acc2 = fmaf(qr[d + 2], kr[d + 2], acc2);
-        acc3 = fmaf(qr[d + 3], kr[d + 3], acc3);
-      }
       const int pos = p0 + r / P.group;
       const bool ok = lane < n && j <= pos && (P.window < 0 || pos - j <= P.window);
-      const float s = ok ? ((acc0 + acc1) + (acc2 + acc3)) * P.scale_log2 : -INFINITY;
+      const float s = ok ? acc[k] * P.scale_log2 : -INFINITY;
       float mx = s;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));

@@ -187,3 +187,54 @@ def make_decode_inputs(kv_lens, q_lens, hq, hkv, has_sink, seed, spare_rows=64, 
     cu_q = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
     sink = synth.normal_f32(seed, synth.STREAM_SINK, hq) if has_sink else None
     return DecodeInputs(q, k, v, kv_indices, kv_indptr, cu_q, sink, q_lens, kv_lens)
+
+
+DECODE_KINDS = ("swa", "global")
+
+
+def decode_batch(kind: str, seed: int = 0, num_seqs: int = 64, q_len: int = 8, kv_lo: int = 1024,
+                 kv_hi: int = 8192, threads=None):
+    """A serving-shaped batch for the KV-cache path: num_seqs requests (SGLang's cap of 64 running
+    requests), q_len = 8 new tokens each (8 speculative draft tokens), context lengths uniform in
+    [kv_lo, kv_hi].  The sliding-window layer (64 Q / 8 KV heads, window 128, sink, base 1e4) keeps
+    only each request's last window + q_len rows in its cache, as a sliding-window pool does; the
+    index entries of older positions point at row 0 and are never read.  The global layer (64 Q /
+    4 KV heads, base 1e7) keeps every row.  Returns (DecodeInputs, layer_kind, window, rope_base)."""
+    assert kind in DECODE_KINDS
+    kv = [int(x) for x in synth.seq_lengths(seed, num_seqs, kv_lo, kv_hi)]
+    ql = [min(q_len, x) for x in kv]
+    if kind == "swa":
+        hq, hkv, window, base, has_sink = 64, 8, SWA_WINDOW, ROPE_BASE_SWA, True
+        stored = [min(x, window + q) for x, q in zip(kv, ql)]
+    else:
+        hq, hkv, window, base, has_sink = 64, 4, -1, ROPE_BASE_GLOBAL, False
+        stored = list(kv)
+    rows = sum(stored) + 1
+    q = synth.normal_bf16(seed, synth.STREAM_Q, (sum(ql), hq, 192), threads)
+    k = synth.normal_bf16(seed, synth.STREAM_K, (rows, hkv, 192), threads)
+    v = synth.normal_bf16(seed, synth.STREAM_V, (rows, hkv, 128), threads)
+    perm = (1 + np.argsort(synth.uniforms(seed, synth.STREAM_PAGES, rows - 1), kind="stable")).astype(np.int32)
+    idx, used = [], 0
+    for x, st in zip(kv, stored):
+        idx.append(np.zeros(x - st, dtype=np.int32))
+        idx.append(perm[used:used + st])
+        used += st
+    kv_indices = np.concatenate(idx).astype(np.int32)
+    kv_indptr = np.concatenate([[0], np.cumsum(kv)]).astype(np.int32)
+    cu_q = np.concatenate([[0], np.cumsum(ql)]).astype(np.int32)
+    sink = synth.normal_f32(seed, synth.STREAM_SINK, hq) if has_sink else None
+    layer = LAYER_SWA if kind == "swa" else LAYER_GLOBAL
+    return DecodeInputs(q, k, v, kv_indices, kv_indptr, cu_q, sink, ql, kv), layer, window, base
+
+
+def decode_subset(x: DecodeInputs, seqs) -> DecodeInputs:
+    """The same problem restricted to the given sequences (for bounded reference checks)."""
+    qs, idx, kv, ql = [], [], [], []
+    for b in seqs:
+        qs.append(x.q[x.cu_q[b]:x.cu_q[b + 1]])
+        idx.append(x.kv_indices[x.kv_indptr[b]:x.kv_indptr[b + 1]])
+        kv.append(x.kv_lens[b])
+        ql.append(x.q_lens[b])
+    return DecodeInputs(np.concatenate(qs), x.k_cache, x.v_cache, np.concatenate(idx).astype(np.int32),
+                        np.concatenate([[0], np.cumsum(kv)]).astype(np.int32),
+                        np.concatenate([[0], np.cumsum(ql)]).astype(np.int32), x.sink, ql, kv)
