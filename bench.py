@@ -556,7 +556,7 @@ def run_decode(args):
         "tflops": flops / (ms / 1e3) / 1e12, "gbs": ach,
         "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peak_src} (burst)",
-                     "kernel": "attn_decode_partial_kernel + attn_decode_combine_kernel",
+                     "kernel": "attn_decode_tc_kernel + attn_decode_combine_kernel",
                      "algorithmic_bytes": nbytes, "algorithmic_flops": flops},
         "cpu_baseline": {"value": rows / cpu_s, "unit": "tokens/s", "cores": oracle.default_threads(),
                          "kind": "oracle", "sample": f"the first two requests of the batch ({rows} new tokens)"},

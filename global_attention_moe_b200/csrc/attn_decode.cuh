@@ -61,6 +61,7 @@ struct DecParams {
   int32_t splits, split_keys;
   float scale_log2;           // log2(e) / sqrt(192)
   float v_scale;
+  uint64_t wait_limit_ns;     // bound of every barrier wait (tensor-core kernel)
   double theta[kRopeDims / 2];
 };
 

@@ -1,0 +1,449 @@
+// attn_decode_tc.cuh -- tensor-core form of the KV-cache attention (decode,
+// speculative-draft verification, chunked prefill) with page size 1.
+//
+// The operation is the one attn_decode.cuh states: query i of sequence b sits
+// at position kv_len_b - q_len_b + i and attends the cache keys the forward
+// would give it; every CTA writes the same per-split partial (running max in
+// log2 units, sum, unnormalised O) that the combine kernel there merges with
+// the sink.
+//
+// One CTA per (sequence, KV head, key split).  The q_len x (Hq/Hkv) query rows
+// that share the KV head (row r = query r / group, head g*group + r % group)
+// form the M = 128 operand of tcgen05.mma (rows past q_len x group are zero and
+// never written out).  K/V rows are gathered by index with cp.async straight
+// into the 128-byte-swizzled K-major layout a TMA tile load would produce, so
+// the score and PV contractions use the same descriptors as the forward:
+//
+//   Q      : 3 units of 128 rows x 64 dims (dims 0..63 rotated, FP16; 64..191 BF16)
+//   stage  : 64 keys: K dims 0..63 (rotated in place, FP16), 64..127, 128..191
+//            (8 KB each, 64 rows x 128 B), then V as 64 keys x 128 dims in two
+//            8 KB halves (dims 0..63, 64..127); 4 stages in a ring
+//   TMEM   : S/P of chunk t in columns 64 (t & 1) .. +63 (P as BF16 pairs in
+//            the first 32), O in columns 128..255
+//
+// Warp roles (9 warps):
+//   warps 0-3  softmax (thread = query row = TMEM lane) and the partial write
+//   warps 4-7  loader: gathers Q once and the K/V chunks into the ring with
+//              cp.async, rotates the first 64 dims of Q and K at their
+//              positions (BF16 -> FP16 in place), then signals the chunk
+//   warp 8     TMEM owner; lane 0 issues the MMAs:
+//              S(0) | S(1) PV(0) | S(2) PV(1) | ... | PV(n-1)
+//              so the score of the next chunk overlaps the softmax of this one.
+// The loader keeps three chunks in flight: chunk k+3 is requested once PV(k-1)
+// has released its stage, which needs S(k), which needs chunk k -- so the
+// loader signals chunk k before it waits for that release.
+//
+// Softmax: lazy rescale as in the pipelined forward (the running max moves only
+// when a chunk's max exceeds it by more than 2^8); O is rescaled in TMEM after
+// PV(t-1) has completed.  Every wait is bounded (kErrTimeout); the softmax
+// warps take each wait's outcome warp-uniformly, since the TMEM loads and
+// stores that follow are warp-collective.
+#pragma once
+
+#include "attn_decode.cuh"
+#include "attn_fwd_swa.cuh"
+
+namespace mimo {
+namespace dtc {
+
+constexpr int kThreads = 288;
+constexpr int kChunk = 64;   // keys per step
+constexpr int kStages = 4;
+constexpr int kAhead = kStages - 1;  // chunks in flight ahead of the one being signalled
+constexpr uint32_t kQUnit = 16384;   // 128 rows x 64 dims x 2 B
+constexpr uint32_t kKUnit = 8192;    // 64 keys x 64 dims x 2 B
+constexpr uint32_t kVOff = 3 * kKUnit;
+constexpr uint32_t kStageBytes = 3 * kKUnit + 2 * kKUnit;  // 40 KB
+constexpr uint32_t kQOff = 0;
+constexpr uint32_t kStageOff = 3 * kQUnit;
+constexpr uint32_t kCtrlOff = kStageOff + kStages * kStageBytes;  // 212992
+constexpr uint32_t kCtrlBytes = 512;
+constexpr uint32_t kSmemBytes = kCtrlOff + kCtrlBytes;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColO = 128;
+constexpr uint32_t kLoaderBar = 2;  // named barrier of the loader warpgroup
+constexpr uint32_t kIdescSF16 = make_idesc_f32acc(0, 0, 128, kChunk);
+constexpr uint32_t kIdescSBF16 = make_idesc_f32acc(1, 0, 128, kChunk);
+static_assert(kStageBytes % 1024 == 0 && kStageOff % 1024 == 0 && kVOff % 1024 == 0, "swizzle atoms");
+
+struct Ctrl {
+  uint64_t q_ready;
+  uint64_t full[kStages], empty[kStages];
+  uint64_t s_full[2], p_full, pv_done, o_full;
+  uint32_t tmem_base;
+  int abort;
+  double theta[kRopeDims / 2];  // RoPE inverse frequencies, staged once per CTA
+};
+static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
+
+// The CTA's share of one sequence.
+struct Work {
+  int q_beg, rows, p0;      // first query row, q_len * group, position of query 0
+  int kv_beg, k_beg, k_end;  // index-list offset, key range [k_beg, k_end) of this split
+  int n;                     // chunks
+  int g;                     // KV head
+};
+
+// Bounded wait; gives up once another role has aborted (kept inline for the same
+// reason as the forward's: every role runs it).
+__device__ __forceinline__ bool dwait(Ctrl* C, uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSliceNs)) return true;
+    if (*reinterpret_cast<volatile int*>(&C->abort)) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *reinterpret_cast<volatile int*>(&C->abort) = 1;
+      atomicOr(&g_mimo_error, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// S = Q K^T for one 64-key chunk: 4 FP16 K-steps (rotated dims) + 8 BF16 K-steps.
+__device__ __forceinline__ void issue_s64(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
+  constexpr uint32_t kQStep = kQUnit >> 4, kKStep = kKUnit >> 4;
+#pragma unroll
+  for (int sub = 0; sub < 4; ++sub) mma_ss_lo(d_tmem, q_lo + 2 * sub, k_lo + 2 * sub, kIdescSF16, sub > 0 ? 1u : 0u);
+#pragma unroll
+  for (int u = 1; u < 3; ++u)
+#pragma unroll
+    for (int sub = 0; sub < 4; ++sub)
+      mma_ss_lo(d_tmem, q_lo + u * kQStep + 2 * sub, k_lo + u * kKStep + 2 * sub, kIdescSBF16, 1u);
+}
+
+// Cache-row indices of the four keys this loader thread copies in chunk c (-1: none / invalid).
+__device__ __forceinline__ void load_idx(const dec::DecParams& P, const Work& w, int c, int rsub, int (&idx)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int key = w.k_beg + c * kChunk + 16 * p + rsub;
+    idx[p] = key < w.k_end ? __ldg(P.kv_indices + w.kv_beg + key) : -1;
+  }
+}
+
+// Issues the copies of chunk c into stage c % kStages (8 lanes per key row, 16 rows per pass).
+__device__ __forceinline__ bool issue_chunk(uint8_t* smem, const dec::DecParams& P, const Work& w, int c, int l8,
+                                           int rsub, const int (&idx)[4]) {
+  const uint32_t st = smem_u32(smem + kStageOff + (c % kStages) * kStageBytes);
+  bool bad = false;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int j = 16 * p + rsub;  // key row within the chunk
+    const int key = w.k_beg + c * kChunk + j;
+    const int row = idx[p];
+    const bool in = row >= 0 && row < P.cache_rows;
+    bad |= key < w.k_end && !in;  // an index outside the cache: zeros, reported
+    const uint16_t* ks = in ? P.k_cache + (static_cast<size_t>(row) * P.hkv + w.g) * kHeadDimQK : P.k_cache;
+    const uint16_t* vs = in ? P.v_cache + (static_cast<size_t>(row) * P.hkv + w.g) * kHeadDimV : P.v_cache;
+    const uint32_t nb = in ? 16u : 0u;
+    const uint32_t sw = static_cast<uint32_t>(j * 128 + ((l8 ^ (j & 7)) << 4));
+#pragma unroll
+    for (int u = 0; u < 3; ++u) cp_async_16(st + u * kKUnit + sw, ks + 64 * u + 8 * l8, nb);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) cp_async_16(st + kVOff + h * kKUnit + sw, vs + 64 * h + 8 * l8, nb);
+  }
+  cp_async_commit();
+  return bad;
+}
+
+__device__ __forceinline__ void wait_pending(int n) {  // n = groups allowed to stay in flight (0..4)
+  if (n >= 4) cp_async_wait<4>();
+  else if (n == 3) cp_async_wait<3>();
+  else if (n == 2) cp_async_wait<2>();
+  else if (n == 1) cp_async_wait<1>();
+  else cp_async_wait<0>();
+}
+
+__device__ __forceinline__ void role_loader(uint8_t* smem, Ctrl* C, const dec::DecParams& P, const Work& w, int lt) {
+  const uint64_t lim = P.wait_limit_ns;
+  const int l8 = lt & 7, rsub = lt >> 3;
+  const int group = P.group;
+  // Q rows (zeros past q_len x group)
+#pragma unroll 1
+  for (int pass = 0; pass < 8; ++pass) {
+    const int r = 16 * pass + rsub;
+    const bool in = r < w.rows;
+    const int i = in ? r / group : 0, hh = in ? r % group : 0;
+    const uint16_t* src =
+        in ? P.q + (static_cast<size_t>(w.q_beg + i) * P.hq + w.g * group + hh) * kHeadDimQK : P.q;
+    const uint32_t sw = static_cast<uint32_t>(r * 128 + ((l8 ^ (r & 7)) << 4));
+#pragma unroll
+    for (int u = 0; u < 3; ++u) cp_async_16(smem_u32(smem + kQOff + u * kQUnit) + sw, src + 64 * u + 8 * l8, in ? 16u : 0u);
+  }
+  cp_async_commit();
+  // the first chunks, then their indices' successors
+  int idx[4];
+  bool bad = false;
+  const int first = min(w.n, kAhead + 1);
+#pragma unroll 1
+  for (int c = 0; c < first; ++c) {
+    load_idx(P, w, c, rsub, idx);
+    bad |= issue_chunk(smem, P, w, c, l8, rsub, idx);
+  }
+  if (first < w.n) load_idx(P, w, first, rsub, idx);
+  // Q: rotate once its copies (the oldest group) have landed
+  wait_pending(first);
+  named_bar_sync(kLoaderBar, 128);
+  float amax = 0.f;
+  {
+    const int r = lt;  // one row per thread
+    const int pos = r < w.rows ? w.p0 + r / group : 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) amax = fmaxf(amax, rope_rotate_chunk_pair(smem + kQOff, r, c, pos, C->theta));
+  }
+  fence_proxy_async_smem();
+  mbar_arrive(&C->q_ready);
+
+  bool ok = true;
+  int next = first;  // next chunk to request
+#pragma unroll 1
+  for (int k = 0; k < w.n; ++k) {
+    // chunk k: every copy landed (the ones requested after it may stay in flight)
+    wait_pending(next - k - 1);
+    ok = named_bar_and(kLoaderBar, 128, ok);
+    if (!ok) break;
+    {
+      uint8_t* kr = smem + kStageOff + (k % kStages) * kStageBytes;  // rotated dims of the 64 keys
+      const int r = lt & 63, c0 = 2 * (lt >> 6);
+      const int pos = w.k_beg + k * kChunk + r;
+      amax = fmaxf(amax, rope_rotate_chunk_pair(kr, r, c0, pos, C->theta));
+      amax = fmaxf(amax, rope_rotate_chunk_pair(kr, r, c0 + 1, pos, C->theta));
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&C->full[k % kStages]);
+    // request chunk k + kAhead into the stage PV(k - 1) releases (needs S(k): chunk k, signalled above)
+    if (k >= 1 && next < w.n) {
+      ok = dwait(C, &C->empty[(k - 1) % kStages], ((k - 1) / kStages) & 1, lim);
+      if (ok) {
+        bad |= issue_chunk(smem, P, w, next, l8, rsub, idx);
+        ++next;
+        if (next < w.n) load_idx(P, w, next, rsub, idx);
+      }
+    }
+  }
+  cp_async_wait<0>();  // nothing of ours stays in flight, on every path
+  if (bad) atomicOr(&g_mimo_error, kErrSeqlens);
+  if (amax > 65504.f) atomicOr(&g_mimo_error, kErrRange);
+}
+
+__device__ __forceinline__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, const dec::DecParams& P, const Work& w) {
+  const uint64_t lim = P.wait_limit_ns;
+  const uint32_t qd = sdesc_lo(smem_u32(smem + kQOff), 16);
+  if (!dwait(C, &C->q_ready, 0, lim)) return;
+  tc_fence_after_sync();
+#pragma unroll 1
+  for (int t = 0; t <= w.n; ++t) {
+    if (t < w.n) {
+      const int s = t % kStages;
+      if (!dwait(C, &C->full[s], (t / kStages) & 1, lim)) return;
+      tc_fence_after_sync();
+      issue_s64(tmem + 64u * (t & 1), qd, sdesc_lo(smem_u32(smem + kStageOff + s * kStageBytes), 16));
+      tc_commit(&C->s_full[t & 1]);
+    }
+    if (t >= 1) {
+      const int u = t - 1, s = u % kStages;
+      if (!dwait(C, &C->p_full, u & 1, lim)) return;
+      tc_fence_after_sync();
+      issue_pv_half(tmem + kColO, tmem + 64u * (u & 1),
+                    sdesc_lo(smem_u32(smem + kStageOff + s * kStageBytes + kVOff), kKUnit), u == 0);
+      tc_commit(&C->pv_done);
+      tc_commit(&C->empty[s]);
+    }
+  }
+  tc_commit(&C->o_full);
+}
+
+__device__ __forceinline__ void role_softmax(Ctrl* C, uint32_t tmem, const dec::DecParams& P, const Work& w, int r, int wq,
+                             int split) {
+  const uint64_t lim = P.wait_limit_ns;
+  const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+  const uint32_t tO = tmem + lane_base + kColO;
+  const float sl2 = P.scale_log2;
+  const bool valid = r < w.rows;
+  const int pos = valid ? w.p0 + r / P.group : -1;  // rows past the queries see no key
+  const int last = min(w.k_end - 1, pos);           // last key this row may see
+  const int first = P.window >= 0 ? pos - P.window : w.k_beg;
+  float m = -INFINITY, l = 0.f;
+#pragma unroll 1
+  for (int t = 0; t < w.n; ++t) {
+    const uint32_t tS = tmem + lane_base + 64u * (t & 1);
+    if (!__all_sync(0xffffffffu, dwait(C, &C->s_full[t & 1], (t >> 1) & 1, lim))) return;
+    tc_fence_after_sync();
+    uint32_t s[2][32];
+    tmem_ld32(tS, s[0]);
+    tmem_ld32(tS + 32, s[1]);
+    tmem_ld_wait(s[0]);
+    reg_fence(s[1]);
+    const int c0 = w.k_beg + t * kChunk;
+    const int hi = last - c0, lo = max(first - c0, 0);  // allowed columns lo..hi of this chunk
+    float mx[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {  // masked keys become -inf in place (their exp is 0)
+      const uint32_t run = swa::run_mask(lo - 32 * q, hi - 32 * q);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float x = ((run >> i) & 1u) ? __uint_as_float(s[q][i]) : -INFINITY;
+        s[q][i] = __float_as_uint(x);
+        mx[i & 7] = fmaxf(mx[i & 7], x);
+      }
+    }
+    const float mt =
+        fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+    const bool grow = mt > m + pipe::kRescaleThreshold;
+    const float m_new = grow ? mt : m;
+    const float corr = grow ? ex2_approx(m - m_new) : 1.f;  // m = -inf -> 0
+    const float base = (m_new == -INFINITY) ? 0.f : m_new;
+    float sm[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sm[k] = 0.f;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(s[q][i]), sl2, -base));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(s[q][i + 1]), sl2, -base));
+        sm[i & 7] += p0;
+        sm[(i + 1) & 7] += p1;
+        pk[i >> 1] = pack_bf16x2(p0, p1);
+      }
+      tmem_st16(tS + 16 * q, pk);
+    }
+    l = l * corr + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+    m = m_new;
+    if (t > 0) {
+      // O holds PV(0 .. t-1) once PV(t-1) has completed; rescale it if this row's max moved
+      if (!__all_sync(0xffffffffu, dwait(C, &C->pv_done, (t - 1) & 1, lim))) return;
+      tc_fence_after_sync();
+      if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * q, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+          tmem_st32(tO + 32 * q, o);
+        }
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before_sync();
+    mbar_arrive(&C->p_full);
+  }
+  if (!__all_sync(0xffffffffu, dwait(C, &C->o_full, 0, lim))) return;
+  tc_fence_after_sync();
+  const int i = valid ? r / P.group : 0, hh = valid ? r % P.group : 0;
+  const size_t slot = (static_cast<size_t>(w.q_beg + i) * P.hq + w.g * P.group + hh) * P.splits + split;
+  float4* dst = reinterpret_cast<float4*>(P.part_o + slot * kHeadDimV);
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {  // 32 columns at a time (the loads are warp-collective: every row takes part)
+    uint32_t o[32];
+    tmem_ld32(tO + 32 * q, o);
+    tmem_ld_wait(o);
+    if (valid) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        dst[8 * q + e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                     __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+    }
+  }
+  if (!valid) return;
+  P.part_ml[2 * slot] = m;
+  P.part_ml[2 * slot + 1] = l;
+}
+
+}  // namespace dtc
+
+__global__ void __launch_bounds__(dtc::kThreads, 1) attn_decode_tc_kernel(const __grid_constant__ dec::DecParams P) {
+  using namespace dtc;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  Ctrl* C = reinterpret_cast<Ctrl*>(smem + kCtrlOff);
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5;
+
+  int skip = 0;
+  if (tid == 0) {
+    skip = (*reinterpret_cast<volatile unsigned int*>(&g_mimo_error) & kErrTimeout) != 0;
+    if (smem_u32(smem) & 1023u) skip = 1;  // swizzled operands need a 1 KB aligned base
+  }
+  if (__syncthreads_or(skip)) return;
+
+  // the sequence, with the checks of the CUDA-core kernel (uniform over the CTA)
+  Work w;
+  w.g = g;
+  w.q_beg = __ldg(P.cu_q + b);
+  const int q_len = __ldg(P.cu_q + b + 1) - w.q_beg;
+  w.kv_beg = __ldg(P.kv_indptr + b);
+  const int kv_len = __ldg(P.kv_indptr + b + 1) - w.kv_beg;
+  w.rows = q_len * P.group;
+  if (q_len < 0 || kv_len < 0 || q_len > kv_len || w.rows > 128 || w.q_beg < 0 || w.q_beg + q_len > P.total_q ||
+      w.kv_beg < 0 || w.kv_beg + kv_len > P.total_kv) {
+    if (tid == 0 && split == 0 && g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
+    return;
+  }
+  if (w.rows == 0) return;
+  w.p0 = kv_len - q_len;
+  const int lo = dec::key_lo(kv_len, q_len, P.window);
+  if (kv_len - lo > P.splits * P.split_keys) {
+    if (tid == 0 && split == 0 && g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
+    return;
+  }
+  w.k_beg = lo + split * P.split_keys;
+  w.k_end = min(kv_len, w.k_beg + P.split_keys);
+  w.n = w.k_end > w.k_beg ? (w.k_end - w.k_beg + kChunk - 1) / kChunk : 0;
+  if (w.n == 0) {  // a split past the sequence's keys: an empty partial
+    if (tid < w.rows) {
+      const int i = tid / P.group, hh = tid % P.group;
+      const size_t slot = (static_cast<size_t>(w.q_beg + i) * P.hq + g * P.group + hh) * P.splits + split;
+      float4* dst = reinterpret_cast<float4*>(P.part_o + slot * kHeadDimV);
+      for (int e = 0; e < kHeadDimV / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      P.part_ml[2 * slot] = -INFINITY;
+      P.part_ml[2 * slot + 1] = 0.f;
+    }
+    return;
+  }
+
+  if (tid == 0) {
+    mbar_init(&C->q_ready, 128);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&C->full[s], 128);
+      mbar_init(&C->empty[s], 1);
+    }
+    mbar_init(&C->s_full[0], 1);
+    mbar_init(&C->s_full[1], 1);
+    mbar_init(&C->p_full, 128);
+    mbar_init(&C->pv_done, 1);
+    mbar_init(&C->o_full, 1);
+    C->abort = 0;
+    fence_barrier_init();
+  }
+  if (tid < kRopeDims / 2) C->theta[tid] = P.theta[tid];
+  if (warp == 8) {
+    tmem_alloc(&C->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = C->tmem_base;
+
+  if (warp < 4) {
+    role_softmax(C, tmem, P, w, tid, warp, split);
+  } else if (warp < 8) {
+    role_loader(smem, C, P, w, tid - 128);
+  } else if ((tid & 31) == 0) {
+    role_mma(smem, C, tmem, P, w);
+  }
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace mimo

@@ -19,6 +19,7 @@
 #include "attn_fwd_simple.cuh"
 #include "attn_fwd_swa.cuh"
 #include "attn_decode.cuh"
+#include "attn_decode_tc.cuh"
 #include "rope_k_prepass.cuh"
 #include "params.cuh"
 
@@ -134,8 +135,12 @@ bool set_smem_attributes() {
          cudaFuncSetAttribute(attn_fwd_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               pipe::kSmemBytes) == cudaSuccess &&
          cudaFuncSetAttribute(dec::attn_decode_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              dec::kSmemBytes) == cudaSuccess;
+                              dec::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              dtc::kSmemBytes) == cudaSuccess;
 }
+
+std::atomic<int> g_decode_choice{MIMO_DECODE_AUTO};
 
 // Persistent grid of the two-head kernels: one CTA per SM, at most one per unit.
 int persistent_grid(const FwdParams& P, int sms) {
@@ -418,15 +423,20 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   P.window = (layer_kind == MIMO_LAYER_GLOBAL) ? -1 : window;
   P.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDimQK)));
   P.v_scale = v_scale;
+  P.wait_limit_ns = kDefaultWaitLimitNs;
   for (int i = 0; i < kRopeDims / 2; ++i) P.theta[i] = std::pow(rope_base, -2.0 * i / kRopeDims);
-  // Keys one sequence's queries can see, at most; split them so that about two CTAs run per SM.
+  const bool tensor = g_decode_choice.load() != MIMO_DECODE_CUDA_CORES;
+  // Keys one sequence's queries can see, at most; split them so that the grid covers the SMs a few
+  // times over (tensor-core kernel: one CTA per SM, four waves; CUDA-core kernel: two CTAs per SM).
   const long long span = (P.window >= 0) ? std::min<long long>(d->max_kv_len, (long long)P.window + d->max_q_len)
                                          : (long long)d->max_kv_len;
   const long long base_ctas = (long long)d->num_seqs * P.hkv;
-  long long splits = std::max<long long>(1, (2LL * info->sms + base_ctas - 1) / base_ctas);
+  const long long chunk = tensor ? dtc::kChunk : dec::kChunk;
+  const long long target = (tensor ? 4LL : 2LL) * info->sms;
+  long long splits = std::max<long long>(1, (target + base_ctas - 1) / base_ctas);
   splits = std::min<long long>(splits, std::max<long long>(1, (span + 63) / 64));
   long long split_keys = (span + splits - 1) / splits;
-  split_keys = std::max<long long>(dec::kChunk, (split_keys + dec::kChunk - 1) / dec::kChunk * dec::kChunk);
+  split_keys = std::max<long long>(chunk, (split_keys + chunk - 1) / chunk * chunk);
   splits = std::max<long long>(1, (span + split_keys - 1) / split_keys);
   if (splits > 65535 || d->num_seqs > 65535 || P.hkv > 65535) return MIMO_ERR_UNSUPPORTED;  // grid limits
   P.splits = (int)splits;
@@ -439,7 +449,10 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   P.part_ml = P.part_o + slots * kHeadDimV;
   int st = MIMO_OK;
   dim3 grid((unsigned)splits, (unsigned)P.hkv, (unsigned)d->num_seqs);
-  dec::attn_decode_partial_kernel<<<grid, dec::kThreads, dec::kSmemBytes, stream>>>(P);
+  if (tensor)
+    attn_decode_tc_kernel<<<grid, dtc::kThreads, dtc::kSmemBytes, stream>>>(P);
+  else
+    dec::attn_decode_partial_kernel<<<grid, dec::kThreads, dec::kSmemBytes, stream>>>(P);
   if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
   const long long warps = (long long)d->total_q * P.hq;
   if (st == MIMO_OK) {
@@ -614,7 +627,7 @@ int mimo_attn_profile_stop(int* launches, double* total_ms) {
   return MIMO_OK;
 }
 
-int mimo_attn_version(void) { return (1 << 16) | 3; }
+int mimo_attn_version(void) { return (1 << 16) | 4; }
 
 int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* sink,
                           const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind, int window,
@@ -628,6 +641,13 @@ int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, const flo
 }
 
 size_t mimo_attn_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+int mimo_attn_set_decode_kernel(int choice) {
+  if (choice != MIMO_DECODE_AUTO && choice != MIMO_DECODE_CUDA_CORES && choice != MIMO_DECODE_TENSOR)
+    return MIMO_ERR_INVALID_ARG;
+  g_decode_choice.store(choice);
+  return MIMO_OK;
+}
 
 int mimo_attn_set_kernel(int choice) {
   if (choice != MIMO_KERNEL_AUTO && choice != MIMO_KERNEL_SIMPLE && choice != MIMO_KERNEL_PIPELINED &&

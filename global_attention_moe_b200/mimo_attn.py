@@ -21,8 +21,9 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BAD_
 SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host", "mimo_attn_check",
            "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_fwd_noalloc",
            "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_profile_start",
-           "mimo_attn_profile_stop", "mimo_attn_decode", "mimo_attn_version")
+           "mimo_attn_profile_stop", "mimo_attn_decode", "mimo_attn_set_decode_kernel", "mimo_attn_version")
 KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED, KERNEL_WINDOW = 0, 1, 2, 3
+DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR = 0, 1, 2
 
 
 class Dims(ctypes.Structure):
@@ -74,6 +75,8 @@ def _load():
     lib.mimo_attn_set_kernel.argtypes = [I]
     lib.mimo_attn_decode.restype = I
     lib.mimo_attn_decode.argtypes = [P, P, P, P, P, P, P, ctypes.POINTER(DecodeDims), I, I, D, I, F, P, P, P]
+    lib.mimo_attn_set_decode_kernel.restype = I
+    lib.mimo_attn_set_decode_kernel.argtypes = [I]
     lib.mimo_attn_version.restype = I
     lib.mimo_attn_version.argtypes = []
     return lib
@@ -96,6 +99,13 @@ def set_kernel(choice: int) -> None:
     st = LIB.mimo_attn_set_kernel(int(choice))
     if st != OK:
         raise MimoAttnError(st, "mimo_attn_set_kernel")
+
+
+def set_decode_kernel(choice: int) -> None:
+    """Select the kernel mimo_attn_decode launches (DECODE_AUTO / _CUDA_CORES / _TENSOR)."""
+    st = LIB.mimo_attn_set_decode_kernel(int(choice))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_attn_set_decode_kernel")
 
 
 def profile_start() -> None:

@@ -266,6 +266,22 @@ MIMO_API int mimo_attn_decode(const void* q, const void* k_cache, const void* v_
                               const mimo_decode_dims* dims, int layer_kind, int window, double rope_base,
                               int rope_dims, float v_scale, void* out, float* lse, void* stream);
 
+/*
+ * Selects the kernel mimo_attn_decode launches (process-wide; default AUTO):
+ *   MIMO_DECODE_AUTO        the tensor-core kernel
+ *   MIMO_DECODE_CUDA_CORES  FP32 on the CUDA cores, 32 keys per step (the
+ *                           cross-check path)
+ *   MIMO_DECODE_TENSOR      tcgen05: the query rows of one KV head as the
+ *                           M = 128 operand, K/V gathered by index into
+ *                           shared memory 64 keys per step, S and O in TMEM
+ * Both accept every call mimo_attn_decode accepts and compute the same
+ * operation; they differ in rounding order (the tensor-core kernel rounds P to
+ * BF16 and the rotated dims of Q and K to FP16, as the forward does).  Returns
+ * MIMO_ERR_INVALID_ARG for any other value.
+ */
+typedef enum { MIMO_DECODE_AUTO = 0, MIMO_DECODE_CUDA_CORES = 1, MIMO_DECODE_TENSOR = 2 } mimo_decode_choice;
+MIMO_API int mimo_attn_set_decode_kernel(int choice);
+
 /* ABI version: (major << 16) | minor. */
 MIMO_API int mimo_attn_version(void);
 

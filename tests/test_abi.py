@@ -121,6 +121,16 @@ def test_kernel_choice_values(M):
     M.set_kernel(M.KERNEL_AUTO)
 
 
+def test_decode_kernel_choice_values(M):
+    for choice in (M.DECODE_CUDA_CORES, M.DECODE_TENSOR, M.DECODE_AUTO):
+        M.set_decode_kernel(choice)
+    for bad in (-1, 3, 99):
+        with pytest.raises(M.MimoAttnError) as e:
+            M.set_decode_kernel(bad)
+        assert e.value.status == M.ERR_INVALID_ARG
+    M.set_decode_kernel(M.DECODE_AUTO)
+
+
 @pytest.mark.parametrize("case,expect", [
     (dict(hq=6, hkv=4), 1),                 # Hq % Hkv != 0
     (dict(max_q_len=9, total_q=20, hq=64, hkv=4), 2),  # 9 x 16 rows per KV head > 128

@@ -20,6 +20,15 @@ def _cuda():
     assert mimo_attn.check() == mimo_attn.OK
 
 
+@pytest.fixture(params=["tensor", "cuda_cores"], autouse=True)
+def dkernel(request):
+    """Every test runs on both decode kernels (tcgen05, and FP32 on the CUDA cores)."""
+    from global_attention_moe_b200 import mimo_attn
+    mimo_attn.set_decode_kernel(mimo_attn.DECODE_TENSOR if request.param == "tensor" else mimo_attn.DECODE_CUDA_CORES)
+    yield request.param
+    mimo_attn.set_decode_kernel(mimo_attn.DECODE_AUTO)
+
+
 def parity(x, layer, window, base):
     out, lse = decode_gpu(x, layer, window, base)
     ro, rl = decode_reference(x, window, base)
@@ -104,3 +113,41 @@ def test_rows_per_kv_head_limit():
     with pytest.raises(mimo_attn.MimoAttnError) as e:
         decode_gpu(x, W.LAYER_GLOBAL, -1, 1e7)
     assert e.value.status == mimo_attn.ERR_UNSUPPORTED
+
+
+def test_chunk_and_ring_boundaries():
+    """Contexts at and around the 64-key step of the tensor-core kernel, and long enough per CTA
+    (24 requests x 4 KV heads: few splits) that its 4-stage ring wraps several times."""
+    kv = [63, 64, 65, 128, 191, 192, 257, 320, 1500, 2000, 2600, 3100, 4000, 3500, 900, 1200,
+          2222, 3333, 1111, 777, 2048, 2049, 3999, 66]
+    ql = [1, 8, 2, 8, 3, 8, 4, 8, 5, 6, 7, 8, 1, 2, 3, 4, 5, 6, 7, 8, 8, 8, 8, 2]
+    parity(W.make_decode_inputs(kv, ql, 64, 4, False, seed=38), W.LAYER_GLOBAL, -1, 1e7)
+
+
+@pytest.mark.parametrize("kind", W.DECODE_KINDS)
+def test_serving_batch_sampled(kind):
+    """The bench's serving batch (64 requests, 8 new tokens, contexts 1024..8192) in its own launch
+    configuration: requests 0, 1 and the last against the oracle."""
+    x, layer, window, base = W.decode_batch(kind)
+    out, lse = decode_gpu(x, layer, window, base)
+    seqs = [0, 1, len(x.kv_lens) - 1]
+    ro, rl = decode_reference(W.decode_subset(x, seqs), window, base)
+    rows = np.concatenate([np.arange(x.cu_q[b], x.cu_q[b + 1]) for b in seqs])
+    assert_within(errors(out_to_f64(out)[rows], lse.cpu().numpy().astype(np.float64)[:, rows], ro, rl), kind)
+
+
+@pytest.mark.parametrize("kind", W.DECODE_KINDS)
+def test_kernels_agree_on_serving_batch(kind, dkernel):
+    """Every output row of the two decode kernels (written independently) agree on the full batch."""
+    from global_attention_moe_b200 import mimo_attn
+    if dkernel != "tensor":
+        pytest.skip("one comparison per batch")
+    x, layer, window, base = W.decode_batch(kind, seed=1)
+    out_t, lse_t = decode_gpu(x, layer, window, base)
+    mimo_attn.set_decode_kernel(mimo_attn.DECODE_CUDA_CORES)
+    out_c, lse_c = decode_gpu(x, layer, window, base)
+    a, b = out_t.float(), out_c.float()
+    assert bool(torch.isfinite(a).all())
+    assert float((a - b).abs().max()) <= 2e-2
+    assert float((a - b).norm() / b.norm()) <= 5e-3
+    assert float((lse_t - lse_c).abs().max()) <= 1e-3
