@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--ref-budget-s", type=float, default=90.0, help="reference arm: total CPU seconds to aim for")
     ap.add_argument("--decode", choices=W.DECODE_KINDS, default=None,
                     help="time the KV-cache path (64 requests x 8 new tokens) instead of the forward")
+    ap.add_argument("--decode-requests", type=int, default=64,
+                    help="requests in the KV-cache batch (fewer: a smaller case for profiling)")
     return ap.parse_args()
 
 
@@ -493,7 +495,7 @@ def run_decode(args):
     n_sets = 4 if args.decode == "swa" else 1  # the sliding layer's rows per step fit in L2: rotate
     sets = []
     for seed in range(n_sets):
-        x, layer, window, base = W.decode_batch(args.decode, seed=seed)
+        x, layer, window, base = W.decode_batch(args.decode, seed=seed, num_seqs=args.decode_requests)
         t = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
         i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
         dev = (t(x.q), t(x.k_cache), t(x.v_cache), i32(x.kv_indices), i32(x.kv_indptr), i32(x.cu_q),

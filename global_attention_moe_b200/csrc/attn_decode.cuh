@@ -53,6 +53,7 @@ struct DecParams {
   const float* sink;          // [hq] or nullptr
   float* part_o;              // [Tq, hq, splits, 128]
   float* part_ml;             // [Tq, hq, splits, 2]: running max (log2 units), sum
+  unsigned long long* item_counter;  // zero before the tensor-core kernel: items claimed so far
   uint16_t* out;              // bf16 [Tq, hq, 128]
   float* lse;                 // [hq, Tq]
   int32_t num_seqs, total_q, total_kv, cache_rows;
@@ -282,9 +283,10 @@ __global__ void __launch_bounds__(kThreads) attn_decode_combine_kernel(const __g
   if (q_len <= 0 || q_len > kv_len || q_len * P.group > kMaxRows || q_beg < 0 || q_beg + q_len > P.total_q ||
       kv_beg < 0 || kv_beg + kv_len > P.total_kv)
     return;
-  if (kv_len - key_lo(kv_len, q_len, P.window) > P.splits * P.split_keys) return;
+  const int n_keys = kv_len - key_lo(kv_len, q_len, P.window);
+  if (n_keys > P.splits * P.split_keys) return;
   const size_t base = (static_cast<size_t>(t) * P.hq + h) * P.splits;
-  const int used = P.splits;  // a split without keys wrote max -inf and sum 0
+  const int used = (n_keys + P.split_keys - 1) / P.split_keys;  // splits that hold keys (the others are not written)
   float M = P.sink != nullptr ? __ldg(P.sink + h) * kLog2e : -INFINITY;
   for (int s = 0; s < used; ++s) M = fmaxf(M, P.part_ml[2 * (base + s)]);
   const float mb = (M == -INFINITY) ? 0.f : M;

@@ -7,10 +7,14 @@
 // log2 units, sum, unnormalised O) that the combine kernel there merges with
 // the sink.
 //
-// One CTA per (sequence, KV head, key split).  The q_len x (Hq/Hkv) query rows
-// that share the KV head (row r = query r / group, head g*group + r % group)
-// form the M = 128 operand of tcgen05.mma (rows past q_len x group are zero and
-// never written out).  K/V rows are gathered by index with cp.async straight
+// Work items are (sequence, KV head, key split); the grid is persistent (at
+// most one CTA per SM) and the CTAs share the items through a global counter:
+// a producer warp claims the next item, skips items without keys, and
+// publishes it in a shared-memory ring that every role reads in the same order
+// (items are numbered split-major, so the full-length splits go first and the
+// short remainders last).  The q_len x (Hq/Hkv) query rows of an item (row r = query r / group, head
+// g*group + r % group) form the M = 128 operand of tcgen05.mma (rows past
+// q_len x group are zero and never written out).  K/V rows are gathered by index with cp.async straight
 // into the 128-byte-swizzled K-major layout a TMA tile load would produce, so
 // the score and PV contractions use the same descriptors as the forward:
 //
@@ -21,17 +25,25 @@
 //   TMEM   : S/P of chunk t in columns 64 (t & 1) .. +63 (P as BF16 pairs in
 //            the first 32), O in columns 128..255
 //
-// Warp roles (9 warps):
-//   warps 0-3  softmax (thread = query row = TMEM lane) and the partial write
-//   warps 4-7  loader: gathers Q once and the K/V chunks into the ring with
-//              cp.async, rotates the first 64 dims of Q and K at their
-//              positions (BF16 -> FP16 in place), then signals the chunk
-//   warp 8     TMEM owner; lane 0 issues the MMAs:
-//              S(0) | S(1) PV(0) | S(2) PV(1) | ... | PV(n-1)
-//              so the score of the next chunk overlaps the softmax of this one.
-// The loader keeps three chunks in flight: chunk k+3 is requested once PV(k-1)
-// has released its stage, which needs S(k), which needs chunk k -- so the
-// loader signals chunk k before it waits for that release.
+// Warp roles (14 warps):
+//   warps 0-3   softmax (thread = query row = TMEM lane) and the partial write
+//   warps 4-7   K/V fetcher: gathers the chunks of all items, in order, into
+//               the ring with cp.async as stages free up; each thread's copies
+//               of a chunk arrive on the stage's `landed` barrier when done
+//   warp 8      TMEM owner; lane 0 issues the MMAs over the CTA's chunk stream
+//               (t counts chunks over all items):
+//               S(0) | S(1) PV(0) | S(2) PV(1) | ... | PV(T-1)
+//               so the score of the next chunk overlaps the softmax of this one
+//   warps 9-12  lander: per item, once the previous item's last S has read Q,
+//               loads and rotates the item's Q (its own cp.async groups); then,
+//               per landed chunk, rotates the first 64 dims of K at the key
+//               positions (BF16 -> FP16 in place) and signals the MMA issuer
+//   warp 13     item producer (lane 0)
+// Fetching and landing are separate warps, so a chunk is signalled as soon as
+// it lands, whatever the fetcher is waiting for: chunk f waits for PV(f-4) to
+// release its stage, which needs S(f-3), which needs only chunks already
+// fetched.  PV of an item's first chunk (which overwrites O) waits until the
+// softmax warps have read the previous item's O.
 //
 // Softmax: lazy rescale as in the pipelined forward (the running max moves only
 // when a chunk's max exceeds it by more than 2^8); O is rescaled in TMEM after
@@ -46,7 +58,7 @@
 namespace mimo {
 namespace dtc {
 
-constexpr int kThreads = 288;
+constexpr int kThreads = 448;
 constexpr int kChunk = 64;   // keys per step
 constexpr int kStages = 4;
 constexpr int kAhead = kStages - 1;  // chunks in flight ahead of the one being signalled
@@ -57,32 +69,66 @@ constexpr uint32_t kStageBytes = 3 * kKUnit + 2 * kKUnit;  // 40 KB
 constexpr uint32_t kQOff = 0;
 constexpr uint32_t kStageOff = 3 * kQUnit;
 constexpr uint32_t kCtrlOff = kStageOff + kStages * kStageBytes;  // 212992
-constexpr uint32_t kCtrlBytes = 512;
+constexpr uint32_t kCtrlBytes = 2048;
+constexpr int kRing = 16;  // published items not yet read by every role
 constexpr uint32_t kSmemBytes = kCtrlOff + kCtrlBytes;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 128;
-constexpr uint32_t kLoaderBar = 2;  // named barrier of the loader warpgroup
+constexpr uint32_t kQBar = 3;  // named barrier of the lander warpgroup
 constexpr uint32_t kIdescSF16 = make_idesc_f32acc(0, 0, 128, kChunk);
 constexpr uint32_t kIdescSBF16 = make_idesc_f32acc(1, 0, 128, kChunk);
 static_assert(kStageBytes % 1024 == 0 && kStageOff % 1024 == 0 && kVOff % 1024 == 0, "swizzle atoms");
 
+
+
+// One work item: a key split of one (sequence, KV head).
+struct Work {
+  int q_beg, rows, p0;       // first query row, q_len * group, position of query 0
+  int kv_beg, k_beg, k_end;  // index-list offset, key range [k_beg, k_end) of this split
+  int n;                     // chunks (0: the split lies past the sequence's keys)
+  int g, split;              // KV head, split
+};
+
 struct Ctrl {
-  uint64_t q_ready;
+  uint64_t q_ready, q_empty;
   uint64_t full[kStages], empty[kStages];
-  uint64_t s_full[2], p_full, pv_done, o_full;
+  uint64_t s_full[2], p_full, pv_done, o_full, o_empty;
   uint32_t tmem_base;
   int abort;
+  uint64_t landed[kStages];  // the fetcher's copies of the stage's chunk are in
+  uint64_t item_full[kRing], item_empty[kRing];
+  Work ring[kRing];  // n < 0: no more items
   double theta[kRopeDims / 2];  // RoPE inverse frequencies, staged once per CTA
 };
 static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
 
-// The CTA's share of one sequence.
-struct Work {
-  int q_beg, rows, p0;      // first query row, q_len * group, position of query 0
-  int kv_beg, k_beg, k_end;  // index-list offset, key range [k_beg, k_end) of this split
-  int n;                     // chunks
-  int g;                     // KV head
-};
+// Fills w for item u (split-major: u = (split * num_seqs + b) * hkv + g); false when the item has no query rows or its sequence is
+// inconsistent (reported; the combine kernel skips the same rows).  The checks
+// are those of the CUDA-core kernel.
+__device__ __forceinline__ bool make_work(const dec::DecParams& P, long long u, Work& w) {
+  const long long per_split = static_cast<long long>(P.hkv) * P.num_seqs;
+  w.split = static_cast<int>(u / per_split);
+  const long long r = u % per_split;
+  w.g = static_cast<int>(r % P.hkv);
+  const int b = static_cast<int>(r / P.hkv);
+  w.q_beg = __ldg(P.cu_q + b);
+  const int q_len = __ldg(P.cu_q + b + 1) - w.q_beg;
+  w.kv_beg = __ldg(P.kv_indptr + b);
+  const int kv_len = __ldg(P.kv_indptr + b + 1) - w.kv_beg;
+  w.rows = q_len * P.group;
+  const int lo = dec::key_lo(kv_len, q_len, P.window);
+  if (q_len < 0 || kv_len < 0 || q_len > kv_len || w.rows > 128 || w.q_beg < 0 || w.q_beg + q_len > P.total_q ||
+      w.kv_beg < 0 || w.kv_beg + kv_len > P.total_kv || kv_len - lo > P.splits * P.split_keys) {
+    if (w.split == 0 && w.g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
+    return false;
+  }
+  if (w.rows == 0) return false;
+  w.p0 = kv_len - q_len;
+  w.k_beg = lo + w.split * P.split_keys;
+  w.k_end = min(kv_len, w.k_beg + P.split_keys);
+  w.n = w.k_end > w.k_beg ? (w.k_end - w.k_beg + kChunk - 1) / kChunk : 0;
+  return true;
+}
 
 // Bounded wait; gives up once another role has aborted (kept inline for the same
 // reason as the forward's: every role runs it).
@@ -97,6 +143,48 @@ __device__ __forceinline__ bool dwait(Ctrl* C, uint64_t* bar, uint32_t parity, u
       atomicOr(&g_mimo_error, kErrTimeout);
       return false;
     }
+  }
+}
+
+// Reader of the CTA's item ring; every role reads every published item once, in order.
+struct Items {
+  uint32_t k = 0;
+  // The next item (false at the end, or when the wait gave up: then failed is set).
+  __device__ __forceinline__ bool next(Ctrl* C, Work& w, bool& failed, uint64_t lim) {
+    const int slot = static_cast<int>(k % kRing);
+    if (!dwait(C, &C->item_full[slot], (k / kRing) & 1, lim)) {
+      failed = true;
+      return false;
+    }
+    w = C->ring[slot];
+    mbar_arrive(&C->item_empty[slot]);
+    ++k;
+    return w.n > 0;
+  }
+};
+constexpr uint32_t kItemReaders = 128 + 128 + 1 + 128;  // softmax, fetcher, MMA issuer, lander
+
+// Claims items from the global counter, skips those without keys (and reports
+// inconsistent sequences), and publishes the rest; ends with an n < 0 entry.
+__device__ __forceinline__ void role_producer(Ctrl* C, const dec::DecParams& P) {
+  const uint64_t lim = P.wait_limit_ns;
+  const long long total = static_cast<long long>(P.splits) * P.hkv * P.num_seqs;
+#pragma unroll 1
+  for (uint32_t k = 0;; ++k) {
+    const int slot = static_cast<int>(k % kRing);
+    if (k >= kRing && !dwait(C, &C->item_empty[slot], ((k / kRing) - 1) & 1, lim)) return;
+    Work w;
+    w.n = -1;
+#pragma unroll 1
+    while (true) {
+      const long long v = static_cast<long long>(atomicAdd(P.item_counter, 1ull));
+      if (v >= total) break;
+      if (make_work(P, v, w) && w.n > 0) break;
+      w.n = -1;
+    }
+    C->ring[slot] = w;
+    mbar_arrive(&C->item_full[slot]);
+    if (w.n < 0) return;
   }
 }
 
@@ -121,10 +209,10 @@ __device__ __forceinline__ void load_idx(const dec::DecParams& P, const Work& w,
   }
 }
 
-// Issues the copies of chunk c into stage c % kStages (8 lanes per key row, 16 rows per pass).
-__device__ __forceinline__ bool issue_chunk(uint8_t* smem, const dec::DecParams& P, const Work& w, int c, int l8,
-                                           int rsub, const int (&idx)[4]) {
-  const uint32_t st = smem_u32(smem + kStageOff + (c % kStages) * kStageBytes);
+// Issues the copies of chunk c of item w into ring stage `stage` (8 lanes per key row, 16 rows per pass).
+__device__ __forceinline__ bool issue_chunk(uint8_t* smem, const dec::DecParams& P, const Work& w, int c, int stage,
+                                           int l8, int rsub, const int (&idx)[4]) {
+  const uint32_t st = smem_u32(smem + kStageOff + stage * kStageBytes);
   bool bad = false;
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
@@ -146,213 +234,261 @@ __device__ __forceinline__ bool issue_chunk(uint8_t* smem, const dec::DecParams&
   return bad;
 }
 
-__device__ __forceinline__ void wait_pending(int n) {  // n = groups allowed to stay in flight (0..4)
-  if (n >= 4) cp_async_wait<4>();
-  else if (n == 3) cp_async_wait<3>();
-  else if (n == 2) cp_async_wait<2>();
-  else if (n == 1) cp_async_wait<1>();
-  else cp_async_wait<0>();
-}
-
-__device__ __forceinline__ void role_loader(uint8_t* smem, Ctrl* C, const dec::DecParams& P, const Work& w, int lt) {
+// K/V chunks of every item, in one stream over the ring.
+__device__ __forceinline__ void role_fetcher(uint8_t* smem, Ctrl* C, const dec::DecParams& P, int lt) {
   const uint64_t lim = P.wait_limit_ns;
   const int l8 = lt & 7, rsub = lt >> 3;
-  const int group = P.group;
-  // Q rows (zeros past q_len x group)
-#pragma unroll 1
-  for (int pass = 0; pass < 8; ++pass) {
-    const int r = 16 * pass + rsub;
-    const bool in = r < w.rows;
-    const int i = in ? r / group : 0, hh = in ? r % group : 0;
-    const uint16_t* src =
-        in ? P.q + (static_cast<size_t>(w.q_beg + i) * P.hq + w.g * group + hh) * kHeadDimQK : P.q;
-    const uint32_t sw = static_cast<uint32_t>(r * 128 + ((l8 ^ (r & 7)) << 4));
-#pragma unroll
-    for (int u = 0; u < 3; ++u) cp_async_16(smem_u32(smem + kQOff + u * kQUnit) + sw, src + 64 * u + 8 * l8, in ? 16u : 0u);
-  }
-  cp_async_commit();
-  // the first chunks, then their indices' successors
+  Items items;
+  Work fw;  // the item being fetched
+  bool failed = false, bad = false;
+  bool more = items.next(C, fw, failed, lim);
+  int fc = 0;  // its next chunk
   int idx[4];
-  bool bad = false;
-  const int first = min(w.n, kAhead + 1);
+  if (more) load_idx(P, fw, 0, rsub, idx);
 #pragma unroll 1
-  for (int c = 0; c < first; ++c) {
-    load_idx(P, w, c, rsub, idx);
-    bad |= issue_chunk(smem, P, w, c, l8, rsub, idx);
-  }
-  if (first < w.n) load_idx(P, w, first, rsub, idx);
-  // Q: rotate once its copies (the oldest group) have landed
-  wait_pending(first);
-  named_bar_sync(kLoaderBar, 128);
-  float amax = 0.f;
-  {
-    const int r = lt;  // one row per thread
-    const int pos = r < w.rows ? w.p0 + r / group : 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) amax = fmaxf(amax, rope_rotate_chunk_pair(smem + kQOff, r, c, pos, C->theta));
-  }
-  fence_proxy_async_smem();
-  mbar_arrive(&C->q_ready);
-
-  bool ok = true;
-  int next = first;  // next chunk to request
-#pragma unroll 1
-  for (int k = 0; k < w.n; ++k) {
-    // chunk k: every copy landed (the ones requested after it may stay in flight)
-    wait_pending(next - k - 1);
-    ok = named_bar_and(kLoaderBar, 128, ok);
-    if (!ok) break;
-    {
-      uint8_t* kr = smem + kStageOff + (k % kStages) * kStageBytes;  // rotated dims of the 64 keys
-      const int r = lt & 63, c0 = 2 * (lt >> 6);
-      const int pos = w.k_beg + k * kChunk + r;
-      amax = fmaxf(amax, rope_rotate_chunk_pair(kr, r, c0, pos, C->theta));
-      amax = fmaxf(amax, rope_rotate_chunk_pair(kr, r, c0 + 1, pos, C->theta));
+  for (uint32_t f = 0; more; ++f) {
+    const int stage = static_cast<int>(f % kStages);
+    // the stage's previous chunk f-4 is released by PV(f-4)
+    if (f >= kStages && !dwait(C, &C->empty[stage], ((f / kStages) - 1) & 1, lim)) break;
+    bad |= issue_chunk(smem, P, fw, fc, stage, l8, rsub, idx);
+    cp_async_mbar_arrive_noinc(&C->landed[stage]);
+    if (++fc == fw.n) {
+      more = items.next(C, fw, failed, lim);
+      fc = 0;
     }
-    fence_proxy_async_smem();
-    mbar_arrive(&C->full[k % kStages]);
-    // request chunk k + kAhead into the stage PV(k - 1) releases (needs S(k): chunk k, signalled above)
-    if (k >= 1 && next < w.n) {
-      ok = dwait(C, &C->empty[(k - 1) % kStages], ((k - 1) / kStages) & 1, lim);
-      if (ok) {
-        bad |= issue_chunk(smem, P, w, next, l8, rsub, idx);
-        ++next;
-        if (next < w.n) load_idx(P, w, next, rsub, idx);
-      }
-    }
+    if (more) load_idx(P, fw, fc, rsub, idx);  // in flight while this thread waits for the next stage
   }
   cp_async_wait<0>();  // nothing of ours stays in flight, on every path
   if (bad) atomicOr(&g_mimo_error, kErrSeqlens);
+}
+
+// Per item: Q (once the previous item's last S has read Q), then every chunk as it lands.
+__device__ __forceinline__ void role_lander(uint8_t* smem, Ctrl* C, const dec::DecParams& P, int qt) {
+  const uint64_t lim = P.wait_limit_ns;
+  const int l8 = qt & 7, rsub = qt >> 3;
+  const int group = P.group;
+  Items items;
+  Work w;
+  float amax = 0.f;
+  uint32_t landed = 0;
+  bool ok = true;
+#pragma unroll 1
+  for (uint32_t item = 0;; ++item) {
+    bool failed = false;
+    const bool have = items.next(C, w, failed, lim);
+    ok = ok && !failed && (!have || item == 0 || dwait(C, &C->q_empty, (item - 1) & 1, lim));
+    // every thread leaves here together: a failed wait anywhere ends the loop in all of them
+    if (!named_bar_and(kQBar, 128, ok) || !have) break;
+#pragma unroll 1
+    for (int pass = 0; pass < 8; ++pass) {  // zeros past q_len x group
+      const int r = 16 * pass + rsub;
+      const bool in = r < w.rows;
+      const int i = in ? r / group : 0, hh = in ? r % group : 0;
+      const uint16_t* src =
+          in ? P.q + (static_cast<size_t>(w.q_beg + i) * P.hq + w.g * group + hh) * kHeadDimQK : P.q;
+      const uint32_t sw = static_cast<uint32_t>(r * 128 + ((l8 ^ (r & 7)) << 4));
+#pragma unroll
+      for (int u = 0; u < 3; ++u)
+        cp_async_16(smem_u32(smem + kQOff + u * kQUnit) + sw, src + 64 * u + 8 * l8, in ? 16u : 0u);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    named_bar_sync(kQBar, 128);
+    const int pos = qt < w.rows ? w.p0 + qt / group : 0;  // one row per thread
+#pragma unroll
+    for (int c = 0; c < 4; ++c) amax = fmaxf(amax, rope_rotate_chunk_pair(smem + kQOff, qt, c, pos, C->theta));
+    fence_proxy_async_smem();
+    mbar_arrive(&C->q_ready);
+    // the item's chunks: rotated dims of the 64 keys, two chunk pairs per thread
+    const int r = qt & 63, c0 = 2 * (qt >> 6);
+#pragma unroll 1
+    for (int c = 0; c < w.n; ++c, ++landed) {
+      const int stage = static_cast<int>(landed % kStages);
+      if (ok) ok = dwait(C, &C->landed[stage], (landed / kStages) & 1, lim);
+      if (!ok) continue;  // the same trips as the others, without the work, up to the barrier above
+      uint8_t* kr = smem + kStageOff + stage * kStageBytes;
+      const int kpos = w.k_beg + c * kChunk + r;
+      amax = fmaxf(amax, rope_rotate_chunk_pair(kr, r, c0, kpos, C->theta));
+      amax = fmaxf(amax, rope_rotate_chunk_pair(kr, r, c0 + 1, kpos, C->theta));
+      fence_proxy_async_smem();  // the fetcher's copies and these writes, before the MMA reads the stage
+      mbar_arrive(&C->full[stage]);
+    }
+  }
+  cp_async_wait<0>();
   if (amax > 65504.f) atomicOr(&g_mimo_error, kErrRange);
 }
 
-__device__ __forceinline__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, const dec::DecParams& P, const Work& w) {
+__device__ __forceinline__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, const dec::DecParams& P) {
   const uint64_t lim = P.wait_limit_ns;
   const uint32_t qd = sdesc_lo(smem_u32(smem + kQOff), 16);
-  if (!dwait(C, &C->q_ready, 0, lim)) return;
-  tc_fence_after_sync();
+  Items items;
+  Work w;
+  w.n = 0;
+  int c = 0;
+  bool failed = false;
+  uint32_t item = 0;  // busy items started so far
+  bool prev = false, prev_first = false, prev_last = false;
+  uint32_t prev_item = 0;
 #pragma unroll 1
-  for (int t = 0; t <= w.n; ++t) {
-    if (t < w.n) {
-      const int s = t % kStages;
+  for (uint32_t t = 0;; ++t) {
+    bool have = true;
+    if (c == w.n) {
+      have = items.next(C, w, failed, lim);
+      if (failed) return;
+      c = 0;
+      if (have) ++item;
+    }
+    if (have) {
+      if (c == 0) {
+        if (!dwait(C, &C->q_ready, (item - 1) & 1, lim)) return;
+        tc_fence_after_sync();
+      }
+      const int s = static_cast<int>(t % kStages);
       if (!dwait(C, &C->full[s], (t / kStages) & 1, lim)) return;
       tc_fence_after_sync();
       issue_s64(tmem + 64u * (t & 1), qd, sdesc_lo(smem_u32(smem + kStageOff + s * kStageBytes), 16));
       tc_commit(&C->s_full[t & 1]);
+      if (c == w.n - 1) tc_commit(&C->q_empty);  // the item's last S has read Q
     }
-    if (t >= 1) {
-      const int u = t - 1, s = u % kStages;
+    if (prev) {
+      const uint32_t u = t - 1;
+      const int s = static_cast<int>(u % kStages);
       if (!dwait(C, &C->p_full, u & 1, lim)) return;
+      if (prev_first && prev_item > 1 && !dwait(C, &C->o_empty, (prev_item - 2) & 1, lim)) return;
       tc_fence_after_sync();
       issue_pv_half(tmem + kColO, tmem + 64u * (u & 1),
-                    sdesc_lo(smem_u32(smem + kStageOff + s * kStageBytes + kVOff), kKUnit), u == 0);
+                    sdesc_lo(smem_u32(smem + kStageOff + s * kStageBytes + kVOff), kKUnit), prev_first);
       tc_commit(&C->pv_done);
       tc_commit(&C->empty[s]);
+      if (prev_last) tc_commit(&C->o_full);
     }
+    if (!have) break;
+    prev = true;
+    prev_first = c == 0;
+    prev_last = c == w.n - 1;
+    prev_item = item;
+    ++c;
   }
-  tc_commit(&C->o_full);
 }
 
-__device__ __forceinline__ void role_softmax(Ctrl* C, uint32_t tmem, const dec::DecParams& P, const Work& w, int r, int wq,
-                             int split) {
+// Writes an item's partial for row r: (m, l) and the unnormalised O row.
+__device__ __forceinline__ float4* partial_row(const dec::DecParams& P, const Work& w, int r, size_t& slot) {
+  const int i = r / P.group, hh = r % P.group;
+  slot = (static_cast<size_t>(w.q_beg + i) * P.hq + w.g * P.group + hh) * P.splits + w.split;
+  return reinterpret_cast<float4*>(P.part_o + slot * kHeadDimV);
+}
+
+__device__ __forceinline__ void role_softmax(Ctrl* C, uint32_t tmem, const dec::DecParams& P, int r, int wq) {
   const uint64_t lim = P.wait_limit_ns;
   const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
   const uint32_t tO = tmem + lane_base + kColO;
   const float sl2 = P.scale_log2;
-  const bool valid = r < w.rows;
-  const int pos = valid ? w.p0 + r / P.group : -1;  // rows past the queries see no key
-  const int last = min(w.k_end - 1, pos);           // last key this row may see
-  const int first = P.window >= 0 ? pos - P.window : w.k_beg;
-  float m = -INFINITY, l = 0.f;
+  Items items;
+  Work w;
+  uint32_t t = 0, item = 0;  // chunks and items so far
 #pragma unroll 1
-  for (int t = 0; t < w.n; ++t) {
-    const uint32_t tS = tmem + lane_base + 64u * (t & 1);
-    if (!__all_sync(0xffffffffu, dwait(C, &C->s_full[t & 1], (t >> 1) & 1, lim))) return;
-    tc_fence_after_sync();
-    uint32_t s[2][32];
-    tmem_ld32(tS, s[0]);
-    tmem_ld32(tS + 32, s[1]);
-    tmem_ld_wait(s[0]);
-    reg_fence(s[1]);
-    const int c0 = w.k_beg + t * kChunk;
-    const int hi = last - c0, lo = max(first - c0, 0);  // allowed columns lo..hi of this chunk
-    float mx[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {  // masked keys become -inf in place (their exp is 0)
-      const uint32_t run = swa::run_mask(lo - 32 * q, hi - 32 * q);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float x = ((run >> i) & 1u) ? __uint_as_float(s[q][i]) : -INFINITY;
-        s[q][i] = __float_as_uint(x);
-        mx[i & 7] = fmaxf(mx[i & 7], x);
-      }
-    }
-    const float mt =
-        fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-    const bool grow = mt > m + pipe::kRescaleThreshold;
-    const float m_new = grow ? mt : m;
-    const float corr = grow ? ex2_approx(m - m_new) : 1.f;  // m = -inf -> 0
-    const float base = (m_new == -INFINITY) ? 0.f : m_new;
-    float sm[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) sm[k] = 0.f;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(s[q][i]), sl2, -base));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(s[q][i + 1]), sl2, -base));
-        sm[i & 7] += p0;
-        sm[(i + 1) & 7] += p1;
-        pk[i >> 1] = pack_bf16x2(p0, p1);
-      }
-      tmem_st16(tS + 16 * q, pk);
-    }
-    l = l * corr + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
-    m = m_new;
-    if (t > 0) {
-      // O holds PV(0 .. t-1) once PV(t-1) has completed; rescale it if this row's max moved
-      if (!__all_sync(0xffffffffu, dwait(C, &C->pv_done, (t - 1) & 1, lim))) return;
+  while (true) {
+    bool failed = false;
+    const bool have = items.next(C, w, failed, lim);
+    if (!__all_sync(0xffffffffu, !failed) || !have) break;
+    const bool valid = r < w.rows;
+    const int pos = valid ? w.p0 + r / P.group : -1;  // rows past the queries see no key
+    const int last = min(w.k_end - 1, pos);           // last key this row may see
+    const int first = P.window >= 0 ? pos - P.window : w.k_beg;
+    float m = -INFINITY, l = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < w.n; ++c, ++t) {
+      const uint32_t tS = tmem + lane_base + 64u * (t & 1);
+      if (!__all_sync(0xffffffffu, dwait(C, &C->s_full[t & 1], (t >> 1) & 1, lim))) return;
       tc_fence_after_sync();
-      if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * q, o);
-          tmem_ld_wait(o);
+      uint32_t s[2][32];
+      tmem_ld32(tS, s[0]);
+      tmem_ld32(tS + 32, s[1]);
+      tmem_ld_wait(s[0]);
+      reg_fence(s[1]);
+      const int c0 = w.k_beg + c * kChunk;
+      const int hi = last - c0, lo = max(first - c0, 0);  // allowed columns lo..hi of this chunk
+      float mx[8];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-          tmem_st32(tO + 32 * q, o);
+      for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {  // masked keys become -inf in place (their exp is 0)
+        const uint32_t run = swa::run_mask(lo - 32 * q, hi - 32 * q);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x = ((run >> i) & 1u) ? __uint_as_float(s[q][i]) : -INFINITY;
+          s[q][i] = __float_as_uint(x);
+          mx[i & 7] = fmaxf(mx[i & 7], x);
         }
       }
-    }
-    tmem_st_wait();
-    tc_fence_before_sync();
-    mbar_arrive(&C->p_full);
-  }
-  if (!__all_sync(0xffffffffu, dwait(C, &C->o_full, 0, lim))) return;
-  tc_fence_after_sync();
-  const int i = valid ? r / P.group : 0, hh = valid ? r % P.group : 0;
-  const size_t slot = (static_cast<size_t>(w.q_beg + i) * P.hq + w.g * P.group + hh) * P.splits + split;
-  float4* dst = reinterpret_cast<float4*>(P.part_o + slot * kHeadDimV);
-#pragma unroll 1
-  for (int q = 0; q < 4; ++q) {  // 32 columns at a time (the loads are warp-collective: every row takes part)
-    uint32_t o[32];
-    tmem_ld32(tO + 32 * q, o);
-    tmem_ld_wait(o);
-    if (valid) {
+      const float mt =
+          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+      const bool grow = mt > m + pipe::kRescaleThreshold;
+      const float m_new = grow ? mt : m;
+      const float corr = grow ? ex2_approx(m - m_new) : 1.f;  // m = -inf -> 0
+      const float base = (m_new == -INFINITY) ? 0.f : m_new;
+      float sm[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        dst[8 * q + e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                                     __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+      for (int k = 0; k < 8; ++k) sm[k] = 0.f;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(s[q][i]), sl2, -base));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(s[q][i + 1]), sl2, -base));
+          sm[i & 7] += p0;
+          sm[(i + 1) & 7] += p1;
+          pk[i >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + 16 * q, pk);
+      }
+      l = l * corr + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+      m = m_new;
+      if (c > 0) {
+        // O holds PV of chunks 0 .. c-1 once PV(c-1) has completed; rescale it if this row's max moved
+        if (!__all_sync(0xffffffffu, dwait(C, &C->pv_done, (t - 1) & 1, lim))) return;
+        tc_fence_after_sync();
+        if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * q, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+            tmem_st32(tO + 32 * q, o);
+          }
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      mbar_arrive(&C->p_full);
     }
+    if (!__all_sync(0xffffffffu, dwait(C, &C->o_full, item & 1, lim))) return;
+    tc_fence_after_sync();
+    size_t slot = 0;
+    float4* dst = valid ? partial_row(P, w, r, slot) : nullptr;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {  // 32 columns at a time (the loads are warp-collective: every row takes part)
+      uint32_t o[32];
+      tmem_ld32(tO + 32 * q, o);
+      tmem_ld_wait(o);
+      if (valid) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          dst[8 * q + e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                       __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+      }
+    }
+    tc_fence_before_sync();
+    mbar_arrive(&C->o_empty);  // the next item's first PV may overwrite O
+    if (valid) {
+      P.part_ml[2 * slot] = m;
+      P.part_ml[2 * slot + 1] = l;
+    }
+    ++item;
   }
-  if (!valid) return;
-  P.part_ml[2 * slot] = m;
-  P.part_ml[2 * slot + 1] = l;
 }
 
 }  // namespace dtc
@@ -361,7 +497,6 @@ __global__ void __launch_bounds__(dtc::kThreads, 1) attn_decode_tc_kernel(const 
   using namespace dtc;
   extern __shared__ __align__(1024) uint8_t smem[];
   Ctrl* C = reinterpret_cast<Ctrl*>(smem + kCtrlOff);
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5;
 
   int skip = 0;
@@ -371,44 +506,11 @@ __global__ void __launch_bounds__(dtc::kThreads, 1) attn_decode_tc_kernel(const 
   }
   if (__syncthreads_or(skip)) return;
 
-  // the sequence, with the checks of the CUDA-core kernel (uniform over the CTA)
-  Work w;
-  w.g = g;
-  w.q_beg = __ldg(P.cu_q + b);
-  const int q_len = __ldg(P.cu_q + b + 1) - w.q_beg;
-  w.kv_beg = __ldg(P.kv_indptr + b);
-  const int kv_len = __ldg(P.kv_indptr + b + 1) - w.kv_beg;
-  w.rows = q_len * P.group;
-  if (q_len < 0 || kv_len < 0 || q_len > kv_len || w.rows > 128 || w.q_beg < 0 || w.q_beg + q_len > P.total_q ||
-      w.kv_beg < 0 || w.kv_beg + kv_len > P.total_kv) {
-    if (tid == 0 && split == 0 && g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
-    return;
-  }
-  if (w.rows == 0) return;
-  w.p0 = kv_len - q_len;
-  const int lo = dec::key_lo(kv_len, q_len, P.window);
-  if (kv_len - lo > P.splits * P.split_keys) {
-    if (tid == 0 && split == 0 && g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
-    return;
-  }
-  w.k_beg = lo + split * P.split_keys;
-  w.k_end = min(kv_len, w.k_beg + P.split_keys);
-  w.n = w.k_end > w.k_beg ? (w.k_end - w.k_beg + kChunk - 1) / kChunk : 0;
-  if (w.n == 0) {  // a split past the sequence's keys: an empty partial
-    if (tid < w.rows) {
-      const int i = tid / P.group, hh = tid % P.group;
-      const size_t slot = (static_cast<size_t>(w.q_beg + i) * P.hq + g * P.group + hh) * P.splits + split;
-      float4* dst = reinterpret_cast<float4*>(P.part_o + slot * kHeadDimV);
-      for (int e = 0; e < kHeadDimV / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-      P.part_ml[2 * slot] = -INFINITY;
-      P.part_ml[2 * slot + 1] = 0.f;
-    }
-    return;
-  }
-
   if (tid == 0) {
     mbar_init(&C->q_ready, 128);
+    mbar_init(&C->q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
+      mbar_init(&C->landed[s], 128);  // one cp.async arrival per fetcher thread
       mbar_init(&C->full[s], 128);
       mbar_init(&C->empty[s], 1);
     }
@@ -417,6 +519,11 @@ __global__ void __launch_bounds__(dtc::kThreads, 1) attn_decode_tc_kernel(const 
     mbar_init(&C->p_full, 128);
     mbar_init(&C->pv_done, 1);
     mbar_init(&C->o_full, 1);
+    mbar_init(&C->o_empty, 128);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&C->item_full[i], 1);
+      mbar_init(&C->item_empty[i], kItemReaders);
+    }
     C->abort = 0;
     fence_barrier_init();
   }
@@ -431,11 +538,15 @@ __global__ void __launch_bounds__(dtc::kThreads, 1) attn_decode_tc_kernel(const 
   const uint32_t tmem = C->tmem_base;
 
   if (warp < 4) {
-    role_softmax(C, tmem, P, w, tid, warp, split);
+    role_softmax(C, tmem, P, tid, warp);
   } else if (warp < 8) {
-    role_loader(smem, C, P, w, tid - 128);
+    role_fetcher(smem, C, P, tid - 128);
+  } else if (warp == 8) {
+    if ((tid & 31) == 0) role_mma(smem, C, tmem, P);
+  } else if (warp < 13) {
+    role_lander(smem, C, P, tid - 288);
   } else if ((tid & 31) == 0) {
-    role_mma(smem, C, tmem, P, w);
+    role_producer(C, P);
   }
   __syncwarp();
   tc_fence_before_sync();

@@ -426,15 +426,17 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   P.wait_limit_ns = kDefaultWaitLimitNs;
   for (int i = 0; i < kRopeDims / 2; ++i) P.theta[i] = std::pow(rope_base, -2.0 * i / kRopeDims);
   const bool tensor = g_decode_choice.load() != MIMO_DECODE_CUDA_CORES;
-  // Keys one sequence's queries can see, at most; split them so that the grid covers the SMs a few
-  // times over (tensor-core kernel: one CTA per SM, four waves; CUDA-core kernel: two CTAs per SM).
+  // Keys one sequence's queries can see, at most; split them so that the work covers the SMs a few
+  // times over (tensor-core kernel: persistent, one CTA per SM walking about six (sequence, KV head,
+  // split) items; CUDA-core kernel: one CTA per item, about two per SM).
   const long long span = (P.window >= 0) ? std::min<long long>(d->max_kv_len, (long long)P.window + d->max_q_len)
                                          : (long long)d->max_kv_len;
   const long long base_ctas = (long long)d->num_seqs * P.hkv;
   const long long chunk = tensor ? dtc::kChunk : dec::kChunk;
-  const long long target = (tensor ? 4LL : 2LL) * info->sms;
+  const long long target = (tensor ? 6LL : 2LL) * info->sms;
   long long splits = std::max<long long>(1, (target + base_ctas - 1) / base_ctas);
-  splits = std::min<long long>(splits, std::max<long long>(1, (span + 63) / 64));
+  const long long min_split = tensor ? 256 : 64;  // fewer keys per CTA do not pay for its set-up
+  splits = std::min<long long>(splits, std::max<long long>(1, (span + min_split - 1) / min_split));
   long long split_keys = (span + splits - 1) / splits;
   split_keys = std::max<long long>(chunk, (split_keys + chunk - 1) / chunk * chunk);
   splits = std::max<long long>(1, (span + split_keys - 1) / split_keys);
@@ -442,18 +444,26 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   P.splits = (int)splits;
   P.split_keys = (int)split_keys;
   const size_t slots = (size_t)d->total_q * P.hq * splits;
+  const size_t part_bytes = align256(slots * (kHeadDimV * 4 + 8));
   void* part = nullptr;
-  if (cudaMallocFromPoolAsync(&part, slots * (kHeadDimV * 4 + 8), info->pool, stream) != cudaSuccess)
-    return MIMO_ERR_CUDA;
+  if (cudaMallocFromPoolAsync(&part, part_bytes + 256, info->pool, stream) != cudaSuccess) return MIMO_ERR_CUDA;
   P.part_o = static_cast<float*>(part);
   P.part_ml = P.part_o + slots * kHeadDimV;
+  P.item_counter = reinterpret_cast<unsigned long long*>(static_cast<char*>(part) + part_bytes);
   int st = MIMO_OK;
-  dim3 grid((unsigned)splits, (unsigned)P.hkv, (unsigned)d->num_seqs);
-  if (tensor)
-    attn_decode_tc_kernel<<<grid, dtc::kThreads, dtc::kSmemBytes, stream>>>(P);
-  else
-    dec::attn_decode_partial_kernel<<<grid, dec::kThreads, dec::kSmemBytes, stream>>>(P);
-  if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+  if (tensor && cudaMemsetAsync(P.item_counter, 0, sizeof(unsigned long long), stream) != cudaSuccess)
+    st = MIMO_ERR_CUDA;
+  if (st == MIMO_OK) {
+    if (tensor) {  // persistent: at most one CTA per SM, items from the shared counter
+      const long long items = splits * P.hkv * (long long)d->num_seqs;
+      attn_decode_tc_kernel<<<(unsigned)std::min<long long>(items, info->sms), dtc::kThreads, dtc::kSmemBytes,
+                              stream>>>(P);
+    } else {
+      dim3 grid((unsigned)splits, (unsigned)P.hkv, (unsigned)d->num_seqs);
+      dec::attn_decode_partial_kernel<<<grid, dec::kThreads, dec::kSmemBytes, stream>>>(P);
+    }
+    if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+  }
   const long long warps = (long long)d->total_q * P.hq;
   if (st == MIMO_OK) {
     dec::attn_decode_combine_kernel<<<(unsigned)((warps * 32 + dec::kThreads - 1) / dec::kThreads), dec::kThreads,

@@ -337,6 +337,12 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src, 
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Arrives on `bar` once every cp.async this thread has issued so far has landed
+// (without raising the barrier's pending count: the barrier expects one such
+// arrival per issuing thread and phase).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 // Waits until at most N of this thread's committed groups are still in flight.
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
