@@ -47,7 +47,9 @@
 //
 // Softmax: lazy rescale as in the pipelined forward (the running max moves only
 // when a chunk's max exceeds it by more than 2^8); O is rescaled in TMEM after
-// PV(t-1) has completed.  Every wait is bounded (kErrTimeout); the softmax
+// PV(t-1) has completed, and only a warp that rescales waits for that, so the
+// softmax of chunk t otherwise hands its P over without a round trip through
+// PV(t-1).  Every wait is bounded (kErrTimeout); the softmax
 // warps take each wait's outcome warp-uniformly, since the TMEM loads and
 // stores that follow are warp-collective.
 #pragma once
@@ -92,7 +94,7 @@ struct Work {
 struct Ctrl {
   uint64_t q_ready, q_empty;
   uint64_t full[kStages], empty[kStages];
-  uint64_t s_full[2], p_full, pv_done, o_full, o_empty;
+  uint64_t s_full[2], p_full[2], pv_done, o_full, o_empty;  // p_full by chunk parity: a warp may run a chunk ahead
   uint32_t tmem_base;
   int abort;
   uint64_t landed[kStages];  // the fetcher's copies of the stage's chunk are in
@@ -353,7 +355,7 @@ __device__ __forceinline__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, 
     if (prev) {
       const uint32_t u = t - 1;
       const int s = static_cast<int>(u % kStages);
-      if (!dwait(C, &C->p_full, u & 1, lim)) return;
+      if (!dwait(C, &C->p_full[u & 1], (u >> 1) & 1, lim)) return;
       if (prev_first && prev_item > 1 && !dwait(C, &C->o_empty, (prev_item - 2) & 1, lim)) return;
       tc_fence_after_sync();
       issue_pv_half(tmem + kColO, tmem + 64u * (u & 1),
@@ -445,25 +447,25 @@ __device__ __forceinline__ void role_softmax(Ctrl* C, uint32_t tmem, const dec::
       }
       l = l * corr + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
       m = m_new;
-      if (c > 0) {
-        // O holds PV of chunks 0 .. c-1 once PV(c-1) has completed; rescale it if this row's max moved
+      if (c > 0 && __any_sync(0xffffffffu, grow)) {
+        // O holds PV of chunks 0 .. c-1 once PV(c-1) has completed: rescale it.  Only a warp that
+        // rescales waits; pv_done cannot run two phases ahead of any waiter, since PV(t) needs
+        // this chunk's P.
         if (!__all_sync(0xffffffffu, dwait(C, &C->pv_done, (t - 1) & 1, lim))) return;
         tc_fence_after_sync();
-        if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-          for (int q = 0; q < 4; ++q) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * q, o);
-            tmem_ld_wait(o);
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * q, o);
+          tmem_ld_wait(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-            tmem_st32(tO + 32 * q, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+          tmem_st32(tO + 32 * q, o);
         }
       }
       tmem_st_wait();
       tc_fence_before_sync();
-      mbar_arrive(&C->p_full);
+      mbar_arrive(&C->p_full[t & 1]);
     }
     if (!__all_sync(0xffffffffu, dwait(C, &C->o_full, item & 1, lim))) return;
     tc_fence_after_sync();
@@ -516,7 +518,8 @@ __global__ void __launch_bounds__(dtc::kThreads, 1) attn_decode_tc_kernel(const 
     }
     mbar_init(&C->s_full[0], 1);
     mbar_init(&C->s_full[1], 1);
-    mbar_init(&C->p_full, 128);
+    mbar_init(&C->p_full[0], 128);
+    mbar_init(&C->p_full[1], 128);
     mbar_init(&C->pv_done, 1);
     mbar_init(&C->o_full, 1);
     mbar_init(&C->o_empty, 128);
