@@ -13,13 +13,13 @@
 // first 64 dims of Q and K at their positions.  The result equals the
 // forward's output rows for those positions.
 //
-// The path is bound by reading K and V (640 bytes per cache row and KV head)
-// and does little arithmetic per byte, so it runs on the CUDA cores in FP32:
-// one CTA per (sequence, KV head, key split) holds the q_len x (Hq/Hkv) query
-// rows that share the KV head, walks its keys 32 at a time (one key per lane,
-// rows spread over the warps) with an online softmax, and writes a partial
-// (max, sum, O) per row; a second kernel merges the splits with the sink and
-// writes BF16 out and the FP32 LSE.
+// This file holds the FP32 CUDA-core form of the per-split kernel (the
+// cross-check of the tensor-core kernel in attn_decode_tc.cuh) and the combine
+// kernel both use: one CTA per (sequence, KV head, key split) holds the
+// q_len x (Hq/Hkv) query rows that share the KV head, walks its keys 32 at a
+// time (one key per lane, rows spread over the warps) with an online softmax,
+// and writes a partial (max, sum, O) per row; the combine kernel merges the
+// splits that hold keys with the sink and writes BF16 out and the FP32 LSE.
 #pragma once
 
 #include "params.cuh"

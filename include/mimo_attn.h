@@ -253,8 +253,8 @@ MIMO_API int mimo_attn_profile_stop(int* launches, double* total_ms);
  * kv_indptr, q_len_b > kv_len_b and cache rows outside [0, cache_rows) are
  * recorded as MIMO_ERR_BAD_SEQLENS for mimo_attn_check (such rows are left
  * unwritten; an index outside the cache is never dereferenced).  Scratch: a
- * partial result per key split, total_q * Hq * splits * 520 bytes from the
- * library's stream-ordered pool.  Does not synchronise.  (The pages give no
+ * partial result per key split, total_q * Hq * splits * 520 bytes (plus 512
+ * bytes) from the library's stream-ordered pool.  Does not synchronise.  (The pages give no
  * interface; this one mirrors mimo_attn_fwd.)
  */
 typedef struct {
