@@ -62,6 +62,8 @@ def parse():
                     help="time the KV-cache path (64 requests x 8 new tokens) instead of the forward")
     ap.add_argument("--decode-requests", type=int, default=64,
                     help="requests in the KV-cache batch (fewer: a smaller case for profiling)")
+    ap.add_argument("--decode-contiguous", action="store_true",
+                    help="each request's cache rows in order instead of a random permutation")
     return ap.parse_args()
 
 
@@ -495,7 +497,8 @@ def run_decode(args):
     n_sets = 4 if args.decode == "swa" else 1  # the sliding layer's rows per step fit in L2: rotate
     sets = []
     for seed in range(n_sets):
-        x, layer, window, base = W.decode_batch(args.decode, seed=seed, num_seqs=args.decode_requests)
+        x, layer, window, base = W.decode_batch(args.decode, seed=seed, num_seqs=args.decode_requests,
+                                                contiguous=args.decode_contiguous)
         t = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
         i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
         dev = (t(x.q), t(x.k_cache), t(x.v_cache), i32(x.kv_indices), i32(x.kv_indptr), i32(x.cu_q),
@@ -554,6 +557,7 @@ def run_decode(args):
                    "layer": "swa_sink" if args.decode == "swa" else "global_causal", "requests": len(x0.kv_lens),
                    "new_tokens": Tq, "context_tokens": int(sum(x0.kv_lens)), "q_heads": 64,
                    "kv_heads": int(x0.k_cache.shape[1]), "page_size": 1,
+                   "cache_rows": "in request order" if args.decode_contiguous else "random permutation",
                    "l2": f"{n_sets} input sets rotated ({n_sets * set_bytes / 2**20:.0f} MiB on the device)"},
         "tflops": flops / (ms / 1e3) / 1e12, "gbs": ach,
         "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",

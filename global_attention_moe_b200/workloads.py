@@ -193,13 +193,15 @@ DECODE_KINDS = ("swa", "global")
 
 
 def decode_batch(kind: str, seed: int = 0, num_seqs: int = 64, q_len: int = 8, kv_lo: int = 1024,
-                 kv_hi: int = 8192, threads=None):
+                 kv_hi: int = 8192, threads=None, contiguous: bool = False):
     """A serving-shaped batch for the KV-cache path: num_seqs requests (SGLang's cap of 64 running
     requests), q_len = 8 new tokens each (8 speculative draft tokens), context lengths uniform in
     [kv_lo, kv_hi].  The sliding-window layer (64 Q / 8 KV heads, window 128, sink, base 1e4) keeps
     only each request's last window + q_len rows in its cache, as a sliding-window pool does; the
     index entries of older positions point at row 0 and are never read.  The global layer (64 Q /
-    4 KV heads, base 1e7) keeps every row.  Returns (DecodeInputs, layer_kind, window, rope_base)."""
+    4 KV heads, base 1e7) keeps every row.  Cache rows are a seeded random permutation (a
+    fragmented page-size-1 pool), or, with ``contiguous``, each request's rows in order (a pool
+    filled request by request).  Returns (DecodeInputs, layer_kind, window, rope_base)."""
     assert kind in DECODE_KINDS
     kv = [int(x) for x in synth.seq_lengths(seed, num_seqs, kv_lo, kv_hi)]
     ql = [min(q_len, x) for x in kv]
@@ -213,7 +215,10 @@ def decode_batch(kind: str, seed: int = 0, num_seqs: int = 64, q_len: int = 8, k
     q = synth.normal_bf16(seed, synth.STREAM_Q, (sum(ql), hq, 192), threads)
     k = synth.normal_bf16(seed, synth.STREAM_K, (rows, hkv, 192), threads)
     v = synth.normal_bf16(seed, synth.STREAM_V, (rows, hkv, 128), threads)
-    perm = (1 + np.argsort(synth.uniforms(seed, synth.STREAM_PAGES, rows - 1), kind="stable")).astype(np.int32)
+    if contiguous:
+        perm = np.arange(1, rows, dtype=np.int32)
+    else:
+        perm = (1 + np.argsort(synth.uniforms(seed, synth.STREAM_PAGES, rows - 1), kind="stable")).astype(np.int32)
     idx, used = [], 0
     for x, st in zip(kv, stored):
         idx.append(np.zeros(x - st, dtype=np.int32))

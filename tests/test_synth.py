@@ -1,6 +1,7 @@
 """The seeded input generator: SplitMix64 against its scalar definition, BF16
 rounding against torch, chunking and stream independence."""
 import numpy as np
+import pytest
 import torch
 
 from global_attention_moe_b200 import synth, workloads
@@ -64,3 +65,24 @@ def test_workload_pair_counts():
     assert workloads.attended_pairs([4096], 128, 1) == 129 * 4096 - 8256
     assert workloads.attended_pairs([8192, 8192], -1, 1) == 8192 * 8193
     assert workloads.attended_pairs([512], 128, 4) == 4 * (129 * 512 - 8256)
+
+
+@pytest.mark.parametrize("kind", workloads.DECODE_KINDS)
+@pytest.mark.parametrize("contiguous", [False, True])
+def test_decode_batch_rows(kind, contiguous):
+    """Every stored cache row is used by exactly one key; the sliding layer's older positions
+    point at row 0 (never read); the contiguous layout keeps each request's rows in order."""
+    x, layer, window, base = workloads.decode_batch(kind, seed=3, num_seqs=5, kv_lo=100, kv_hi=400, contiguous=contiguous)
+    stored = []
+    for b, kv in enumerate(x.kv_lens):
+        idx = x.kv_indices[x.kv_indptr[b]:x.kv_indptr[b + 1]]
+        assert len(idx) == kv
+        keep = min(kv, window + x.q_lens[b]) if window >= 0 else kv
+        assert np.all(idx[:kv - keep] == 0)
+        live = idx[kv - keep:]
+        assert np.all((live >= 1) & (live < x.k_cache.shape[0]))
+        if contiguous:
+            assert np.all(np.diff(live) == 1)
+        stored.append(live)
+    allrows = np.concatenate(stored)
+    assert len(np.unique(allrows)) == len(allrows) == x.k_cache.shape[0] - 1
