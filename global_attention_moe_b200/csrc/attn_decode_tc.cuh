@@ -56,6 +56,7 @@
 
 #include "attn_decode.cuh"
 #include "attn_fwd_swa.cuh"
+#include "cp_async.cuh"
 
 namespace mimo {
 namespace dtc {
