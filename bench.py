@@ -62,6 +62,8 @@ def parse():
                     help="time the KV-cache path (64 requests x 8 new tokens) instead of the forward")
     ap.add_argument("--decode-requests", type=int, default=64,
                     help="requests in the KV-cache batch (fewer: a smaller case for profiling)")
+    ap.add_argument("--step", choices=("bwd", "dequant", "split", "route"), default=None,
+                    help="time a step beside the forward instead (backward, FP8 dequant, QKV split, MoE routing)")
     ap.add_argument("--decode-contiguous", action="store_true",
                     help="each request's cache rows in order instead of a random permutation")
     return ap.parse_args()
@@ -575,10 +577,100 @@ def run_decode(args):
     return 0
 
 
+STEP_KINDS = ("bwd", "dequant", "split", "route")
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core FP32 FMA peak at the maximum SM clock
+
+
+def run_step(args):
+    """One of the steps beside the forward (backward, FP8 dequant, fused-QKV split, MoE routing) on a
+    layer-shaped synthetic input; one JSON line (single GPU)."""
+    import torch
+    from global_attention_moe_b200 import mimo_attn, synth
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    rng = np.random.default_rng(0)
+    peaks, peak_src = load_peaks()
+    kind = args.step
+    if kind == "bwd":
+        w = W.WORKLOADS["swa4096"]()
+        x = W.make_inputs(w)
+        dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+        q, k, v = dev(x.q), dev(x.k), dev(x.v)
+        sk = torch.from_numpy(x.sink).cuda()
+        cu = torch.from_numpy(x.cu_seqlens).cuda()
+        out, lse = mimo_attn.fwd(q, k, v, sk, cu, w.max_seqlen, w.layer_kind, w.window, w.rope_base)
+        go = dev(synth.f32_to_bf16_bits(rng.standard_normal((w.total_tokens, w.num_q_heads, 128)).astype(np.float32)))
+        call = lambda: mimo_attn.bwd(q, k, v, sk, cu, w.max_seqlen, w.layer_kind, w.window, w.rope_base, out, lse, go)
+        flops = W.attended_pairs(w.lengths, w.window, w.num_q_heads) * (2 * 192 * 3 + 2 * 128 * 2)  # S, dQ, dK; dP, dV
+        nbytes = w.total_tokens * (w.num_q_heads * (192 * 2 + 128 * 2 * 2 + 4 + 192 * 4)
+                                   + w.num_kv_heads * (192 * 2 + 128 * 2 + 192 * 4 + 128 * 4))
+        units, unit, config = w.total_tokens, "tokens/s", {"workload": "bwd_" + w.name, "grads": "fp32"}
+        bound = "alu"  # FP32 FMAs on the CUDA cores
+    elif kind == "dequant":
+        # a fused qkv_proj weight of the sliding layer (hidden 4096, synthetic): 61 MB of codes, 122 MB out
+        M_, N_ = 8 * (8 * 192 + 320), 4096
+        codes = rng.integers(0, 256, size=(M_, N_)).astype(np.uint8)
+        codes[(codes & 0x7F) == 0x7F] = 0x3F
+        scale = rng.uniform(0.5, 2.0, size=(-(-M_ // 128), -(-N_ // 128))).astype(np.float32)
+        ct, st = torch.from_numpy(codes).cuda(), torch.from_numpy(scale).cuda()
+        call = lambda: mimo_attn.fp8_dequant_blockwise(ct, st)
+        flops, nbytes = 0, M_ * N_ * 3 + scale.size * 4
+        units, unit, config, bound = M_ * N_, "elements/s", {"workload": f"fp8_dequant_{M_}x{N_}_block128"}, "hbm"
+    elif kind == "split":
+        T, hq, hkv = 16384, 64, 8  # 486 MB in, 486 MB out: larger than L2
+        fused = torch.from_numpy(rng.integers(0, 1 << 16, size=(T, hkv * (hq // hkv * 192 + 320))).astype(np.uint16)
+                                 .view(np.int16)).cuda().view(torch.bfloat16)
+        call = lambda: mimo_attn.qkv_split(fused, hq, hkv)
+        flops, nbytes = 0, fused.numel() * 2 * 2
+        units, unit, config, bound = T, "tokens/s", {"workload": f"qkv_split_T{T}_hq{hq}_hkv{hkv}"}, "hbm"
+    else:
+        T, E = 262144, 256  # 268 MB of logits: larger than L2
+        lg = torch.from_numpy((rng.standard_normal((T, E)) * 2).astype(np.float32)).cuda()
+        bias = torch.from_numpy((rng.standard_normal(E) * 0.1).astype(np.float32)).cuda()
+        call = lambda: mimo_attn.moe_route(lg, bias, 8)
+        flops, nbytes = 0, T * E * 4 + E * 4 + T * 8 * 8
+        units, unit, config, bound = T, "tokens/s", {"workload": f"moe_route_T{T}_E{E}_top8"}, "hbm"
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    assert mimo_attn.check() == mimo_attn.OK
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = args.steps
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(steps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    assert mimo_attn.check() == mimo_attn.OK
+    if bound == "hbm":
+        ach, peak, runit = nbytes / (ms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        ach, peak, runit = flops / (ms / 1e3) / 1e12, FP32_ALU_TFLOPS, "TFLOP/s"
+        peak_src = "derived: 148 SMs x 128 FP32 lanes x 2 FLOP per FMA x 1965 MHz"
+    line = {
+        "metric": f"{kind} throughput on 1 B200; % of roofline", "value": units / (ms / 1e3), "unit": unit,
+        "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if kind != "route" else "f32", "data": "synthetic",
+        "config": dict(config, l2="inputs larger than L2"),
+        "roofline": {"bound": bound, "achieved": ach, "peak": peak, "unit": runit, "frac": ach / peak, "traffic": None,
+                     "peak_source": peak_src if bound == "alu" else f"{peak_src} (burst)", "algorithmic_bytes": nbytes, "algorithmic_flops": flops},
+        "e2e": None, "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.decode:
         return run_decode(args)
+    if args.step:
+        return run_step(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

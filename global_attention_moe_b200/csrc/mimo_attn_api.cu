@@ -20,6 +20,8 @@
 #include "attn_fwd_swa.cuh"
 #include "attn_decode.cuh"
 #include "attn_decode_tc.cuh"
+#include "attn_bwd_simple.cuh"
+#include "neighbors.cuh"
 #include "rope_k_prepass.cuh"
 #include "params.cuh"
 
@@ -137,7 +139,9 @@ bool set_smem_attributes() {
          cudaFuncSetAttribute(dec::attn_decode_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               dec::kSmemBytes) == cudaSuccess &&
          cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              dtc::kSmemBytes) == cudaSuccess;
+                              dtc::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(bwd::bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              bwd::kSmemBytes) == cudaSuccess;
 }
 
 std::atomic<int> g_decode_choice{MIMO_DECODE_AUTO};
@@ -474,6 +478,62 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   return st;
 }
 
+int launch_bwd(const void* q, const void* k, const void* v, const float* sink, const int32_t* cu,
+               const mimo_attn_dims* d, int layer_kind, int window, double rope_base, float v_scale,
+               const void* out, const float* lse, const void* dout, const float* dlse, float* dq, float* dk,
+               float* dv, float* dsink, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
+  DeviceInfo* info = device_info(dev);
+  if (!info || !info->kernels_ready || !info->pool) return MIMO_ERR_CUDA;
+  bwd::BwdParams P;
+  std::memset(&P, 0, sizeof P);
+  P.q = static_cast<const uint16_t*>(q);
+  P.k = static_cast<const uint16_t*>(k);
+  P.v = static_cast<const uint16_t*>(v);
+  P.sink = sink;
+  P.cu_seqlens = cu;
+  P.out = static_cast<const uint16_t*>(out);
+  P.lse = lse;
+  P.dout = static_cast<const uint16_t*>(dout);
+  P.dlse = dlse;
+  P.dq = dq;
+  P.dk = dk;
+  P.dv = dv;
+  P.dsink = dsink;
+  P.num_seqs = d->num_seqs;
+  P.total_tokens = d->total_tokens;
+  P.max_seqlen = d->max_seqlen;
+  P.hq = d->num_q_heads;
+  P.hkv = d->num_kv_heads;
+  P.group = d->num_q_heads / d->num_kv_heads;
+  P.window = (layer_kind == MIMO_LAYER_GLOBAL) ? -1 : window;
+  P.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDimQK)));
+  P.v_scale = v_scale;
+  for (int i = 0; i < kRopeDims / 2; ++i) P.theta[i] = std::pow(rope_base, -2.0 * i / kRopeDims);
+  if (d->num_seqs > 65535 || d->num_q_heads > 65535) return MIMO_ERR_UNSUPPORTED;  // grid limits
+  void* scratch = nullptr;
+  const size_t n_d = (size_t)d->total_tokens * d->num_q_heads;
+  if (cudaMallocFromPoolAsync(&scratch, n_d * sizeof(float), info->pool, stream) != cudaSuccess) return MIMO_ERR_CUDA;
+  P.D = static_cast<float*>(scratch);
+  int st = MIMO_OK;
+  bwd::bwd_prep_kernel<<<info->sms * 8, bwd::kThreads, 0, stream>>>(P);
+  if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+  if (st == MIMO_OK && d->max_seqlen > 0) {
+    dim3 grid((unsigned)((d->max_seqlen + bwd::kRows - 1) / bwd::kRows), (unsigned)d->num_seqs, (unsigned)d->num_q_heads);
+    bwd::bwd_main_kernel<<<grid, bwd::kThreads, bwd::kSmemBytes, stream>>>(P);
+    if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+  }
+  if (st == MIMO_OK) {
+    const long long n = (long long)d->total_tokens * d->num_kv_heads * (kRopeDims / 2);
+    if (n > 0) {
+      bwd::bwd_finalize_kernel<<<(unsigned)((n + bwd::kThreads - 1) / bwd::kThreads), bwd::kThreads, 0, stream>>>(P);
+      if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+    }
+  }
+  if (cudaFreeAsync(scratch, stream) != cudaSuccess) st = MIMO_ERR_CUDA;
+  return st;
+}
 }  // namespace
 
 extern "C" {
@@ -637,7 +697,81 @@ int mimo_attn_profile_stop(int* launches, double* total_ms) {
   return MIMO_OK;
 }
 
-int mimo_attn_version(void) { return (1 << 16) | 4; }
+int mimo_attn_bwd(const void* q, const void* k, const void* v, const float* sink, const int32_t* cu_seqlens,
+                  const mimo_attn_dims* dims, int layer_kind, int window, double rope_base, int rope_dims,
+                  float v_scale, const void* out, const float* lse, const void* dout, const float* dlse, float* dq,
+                  float* dk, float* dv, float* dsink, void* stream) {
+  int st = validate(q, k, v, sink, cu_seqlens, dims, layer_kind, window, rope_base, rope_dims, v_scale, out, lse);
+  if (st != MIMO_OK) return st;
+  if ((sink != nullptr) != (dsink != nullptr)) return MIMO_ERR_INVALID_ARG;
+  if (dims->total_tokens == 0) {
+    if (dsink) cudaMemsetAsync(dsink, 0, sizeof(float) * dims->num_q_heads, static_cast<cudaStream_t>(stream));
+    return MIMO_OK;
+  }
+  if (!dout || !dq || !dk || !dv || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return MIMO_ERR_INVALID_ARG;
+  if (dlse && (reinterpret_cast<uintptr_t>(dlse) & 3u)) return MIMO_ERR_INVALID_ARG;
+  return launch_bwd(q, k, v, sink, cu_seqlens, dims, layer_kind, window, rope_base, v_scale, out, lse, dout, dlse, dq,
+                    dk, dv, dsink, static_cast<cudaStream_t>(stream));
+}
+
+int mimo_fp8_dequant_blockwise(const void* codes, const float* scale_inv, int64_t rows, int64_t cols, int block_rows,
+                               int block_cols, void* out, void* stream) {
+  if (rows < 0 || cols < 0 || block_rows < 1 || block_cols < 1) return MIMO_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return MIMO_ERR_UNSUPPORTED;
+  if (rows == 0 || cols == 0) return MIMO_OK;
+  if (!codes || !scale_inv || !out || !aligned16(codes) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(scale_inv) & 3u))
+    return MIMO_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
+  DeviceInfo* info = device_info(dev);
+  if (!info) return MIMO_ERR_CUDA;
+  const long long work = rows * (cols / 16);
+  const unsigned grid = (unsigned)std::min<long long>((work + nb::kThreads - 1) / nb::kThreads, 8LL * info->sms);
+  nb::fp8_dequant_kernel<<<grid, nb::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(codes), scale_inv, static_cast<uint16_t*>(out), rows, cols, block_rows, block_cols);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
+int mimo_qkv_split(const void* fused, int64_t tokens, int num_q_heads, int num_kv_heads, void* q, void* k, void* v,
+                   void* stream) {
+  if (tokens < 0 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads != 0)
+    return MIMO_ERR_INVALID_ARG;
+  if (tokens == 0) return MIMO_OK;
+  if (!fused || !q || !k || !v || !aligned16(fused) || !aligned16(q) || !aligned16(k) || !aligned16(v))
+    return MIMO_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
+  DeviceInfo* info = device_info(dev);
+  if (!info) return MIMO_ERR_CUDA;
+  const long long chunks = tokens * (long long)num_kv_heads * ((num_q_heads / num_kv_heads) * 24 + 40);
+  const unsigned grid = (unsigned)std::min<long long>((chunks + nb::kThreads - 1) / nb::kThreads, 8LL * info->sms);
+  nb::qkv_split_kernel<<<grid, nb::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(fused), static_cast<uint16_t*>(q), static_cast<uint16_t*>(k),
+      static_cast<uint16_t*>(v), tokens, num_q_heads, num_kv_heads);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
+int mimo_moe_route(const float* logits, const float* bias, int64_t tokens, int num_experts, int top_k, int normalize,
+                   int32_t* ids, float* weights, void* stream) {
+  if (tokens < 0 || num_experts < 32 || num_experts % 32 != 0 || top_k < 1 || top_k > 32 || top_k > num_experts)
+    return MIMO_ERR_INVALID_ARG;
+  if (num_experts > 256) return MIMO_ERR_UNSUPPORTED;
+  if (tokens == 0) return MIMO_OK;
+  if (!logits || !bias || !ids || !weights) return MIMO_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
+  DeviceInfo* info = device_info(dev);
+  if (!info) return MIMO_ERR_CUDA;
+  const long long warps_per_cta = nb::kThreads / 32;
+  const unsigned grid = (unsigned)std::min<long long>((tokens + warps_per_cta - 1) / warps_per_cta, 16LL * info->sms);
+  nb::route_kernel<8><<<grid, nb::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      logits, bias, ids, weights, tokens, num_experts, top_k, normalize ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
+int mimo_attn_version(void) { return (1 << 16) | 5; }
 
 int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* sink,
                           const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind, int window,

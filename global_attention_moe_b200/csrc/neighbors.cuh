@@ -1,0 +1,170 @@
+// neighbors.cuh -- the steps on either side of the MiMo-V2 attention kernel:
+// FP8 blockwise dequant of a weight (out = fp8 * scale_inv per block), the
+// split of the kv-head-interleaved fused QKV output into q, k, v, and top-8
+// sigmoid routing with a score-correction bias.  All three are bound by HBM.
+//
+// Sources (page title and section): miles docs "MiMo-V2.6-Flash", section 1
+// Model Introduction (FP8 block-quantized weights, fused kv-head-interleaved
+// qkv_proj; 256 routed experts, top-8 sigmoid routing with a fixed
+// score-correction bias) and section 3.1 (split into q/k/v in head order);
+// Megatron-Bridge API doc "mimo_v2_flash_bridge" (_dequant_fp8_blockwise:
+// out = fp8 value times scale_inv; MiMoV2FlashQKVMapping: 192-dim Q/K, 128-dim
+// V); SGLang cookbook "MiMo-V2.6", section 2 (router logits in FP32).
+// Readings where the pages are silent: E4M3 elements; 128 x 128 scale blocks
+// (a parameter); per KV group the fused row holds its query heads, then its K
+// head, then its V head; the bias enters the choice only and the weights are
+// the chosen sigmoid scores normalised to sum to one; ties go to the lower
+// expert index.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace mimo {
+namespace nb {
+
+constexpr int kThreads = 256;
+
+// ---------------------------------------------------------------- FP8 dequant
+// Thread = 16 consecutive codes of one row (N % 16 == 0: 16-byte loads, 32-byte stores).
+// out = bf16_rne(decode(code) * scale_inv[block]) with the product formed exactly in FP64.
+__global__ void __launch_bounds__(kThreads) fp8_dequant_kernel(const uint8_t* __restrict__ codes,
+                                                               const float* __restrict__ scale_inv,
+                                                               uint16_t* __restrict__ out, int64_t M, int64_t N,
+                                                               int block_m, int block_n) {
+  const int64_t per_row = N / 16;
+  const int64_t n_vec = M * per_row;
+  const int64_t scale_cols = (N + block_n - 1) / block_n;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; e < n_vec;
+       e += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const int64_t i = e / per_row, j0 = (e % per_row) * 16;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(codes + i * N + j0));
+    const uint8_t* c = reinterpret_cast<const uint8_t*>(&u);
+    uint32_t w[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      float f[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = static_cast<int>(j0) + 2 * p + h;
+        const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c[2 * p + h]), __NV_E4M3);
+        const float x = __half2float(__half(hr));
+        const double s = static_cast<double>(__ldg(scale_inv + (i / block_m) * scale_cols + j / block_n));
+        const __nv_bfloat16 b = __double2bfloat16(static_cast<double>(x) * s);
+        f[h] = __bfloat162float(b);
+      }
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(f[0], f[1]);  // exact: both are bf16 values
+      w[p] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + i * N + j0);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+// ---------------------------------------------------------------- fused QKV split
+// Thread = one 16-byte chunk (8 bf16) of the fused row; every head boundary is a multiple of 8.
+__global__ void __launch_bounds__(kThreads) qkv_split_kernel(const uint16_t* __restrict__ fused,
+                                                             uint16_t* __restrict__ q, uint16_t* __restrict__ k,
+                                                             uint16_t* __restrict__ v, int64_t T, int hq, int hkv) {
+  const int group = hq / hkv;
+  const int per_group = group * 192 + 192 + 128;  // elements
+  const int chunks_per_group = per_group / 8;
+  const int64_t chunks_per_row = static_cast<int64_t>(hkv) * chunks_per_group;
+  const int64_t n = T * chunks_per_row;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const int64_t t = e / chunks_per_row;
+    const int rem = static_cast<int>(e % chunks_per_row);
+    const int g = rem / chunks_per_group;
+    const int o = (rem % chunks_per_group) * 8;  // element offset inside the group
+    const uint4 val = __ldg(reinterpret_cast<const uint4*>(fused) + e);
+    uint16_t* dst;
+    if (o < group * 192) {
+      dst = q + (t * hq + g * group + o / 192) * 192 + o % 192;
+    } else if (o < group * 192 + 192) {
+      dst = k + (t * hkv + g) * 192 + (o - group * 192);
+    } else {
+      dst = v + (t * hkv + g) * 128 + (o - group * 192 - 192);
+    }
+    *reinterpret_cast<uint4*>(dst) = val;
+  }
+}
+
+// ---------------------------------------------------------------- MoE router
+// One warp per token (E <= 256, E % 32 == 0): lane holds experts lane + 32 m.  The choice is taken on
+// FP32 keys fp32(sigmoid) + bias with the sigmoid formed in FP64; the weights are the chosen FP64
+// scores normalised in FP64, stored as FP32.
+template <int kMaxPerLane>
+__global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                                                         int32_t* __restrict__ ids, float* __restrict__ weights,
+                                                         int64_t T, int E, int top_k, int normalize) {
+  const int lane = threadIdx.x & 31;
+  const int per_lane = E / 32;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  for (int64_t t = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5; t < T; t += warps) {
+    double sc[kMaxPerLane];
+    float key[kMaxPerLane];
+#pragma unroll
+    for (int m = 0; m < kMaxPerLane; ++m) {
+      if (m < per_lane) {
+        const int e = lane + 32 * m;
+        const double x = static_cast<double>(__ldg(logits + t * E + e));
+        sc[m] = x >= 0 ? 1.0 / (1.0 + exp(-x)) : exp(x) / (1.0 + exp(x));
+        key[m] = static_cast<float>(sc[m]) + __ldg(bias + e);
+      } else {
+        sc[m] = 0.0;
+        key[m] = -INFINITY;
+      }
+    }
+    double chosen = 0.0, total = 0.0;
+    int my_id = -1;  // lane k keeps choice k
+    uint32_t taken = 0;
+#pragma unroll 1
+    for (int c = 0; c < top_k; ++c) {
+      // this lane's best remaining (largest key, then lowest expert)
+      float bk = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int m = 0; m < kMaxPerLane; ++m) {
+        const int e = lane + 32 * m;
+        if (m < per_lane && !((taken >> m) & 1u) && (key[m] > bk || (key[m] == bk && e < be))) {
+          bk = key[m];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ok > bk || (ok == bk && oe < be)) {
+          bk = ok;
+          be = oe;
+        }
+      }
+      // the owner marks it and broadcasts its score
+      double s = 0.0;
+      if ((be & 31) == lane) {
+        const int m = be >> 5;
+#pragma unroll
+        for (int mm = 0; mm < kMaxPerLane; ++mm)
+          if (mm == m) s = sc[mm];
+        taken |= 1u << m;
+      }
+      s = __shfl_sync(0xffffffffu, s, be & 31);
+      total += s;
+      if (lane == c) {
+        my_id = be;
+        chosen = s;
+      }
+    }
+    if (lane < top_k) {
+      ids[t * top_k + lane] = my_id;
+      weights[t * top_k + lane] = static_cast<float>(normalize ? chosen / total : chosen);
+    }
+  }
+}
+
+}  // namespace nb
+}  // namespace mimo

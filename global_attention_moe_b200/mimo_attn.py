@@ -21,7 +21,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BAD_
 SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host", "mimo_attn_check",
            "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_fwd_noalloc",
            "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_profile_start",
-           "mimo_attn_profile_stop", "mimo_attn_decode", "mimo_attn_set_decode_kernel", "mimo_attn_version")
+           "mimo_attn_profile_stop", "mimo_attn_decode", "mimo_attn_set_decode_kernel", "mimo_attn_version",
+           "mimo_attn_bwd", "mimo_fp8_dequant_blockwise", "mimo_qkv_split", "mimo_moe_route")
 KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED, KERNEL_WINDOW = 0, 1, 2, 3
 DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR = 0, 1, 2
 
@@ -75,6 +76,15 @@ def _load():
     lib.mimo_attn_set_kernel.argtypes = [I]
     lib.mimo_attn_decode.restype = I
     lib.mimo_attn_decode.argtypes = [P, P, P, P, P, P, P, ctypes.POINTER(DecodeDims), I, I, D, I, F, P, P, P]
+    lib.mimo_attn_bwd.restype = I
+    lib.mimo_attn_bwd.argtypes = [P, P, P, P, P, ctypes.POINTER(Dims), I, I, D, I, F, P, P, P, P, P, P, P, P, P]
+    L = ctypes.c_int64
+    lib.mimo_fp8_dequant_blockwise.restype = I
+    lib.mimo_fp8_dequant_blockwise.argtypes = [P, P, L, L, I, I, P, P]
+    lib.mimo_qkv_split.restype = I
+    lib.mimo_qkv_split.argtypes = [P, L, I, I, P, P, P, P]
+    lib.mimo_moe_route.restype = I
+    lib.mimo_moe_route.argtypes = [P, P, L, I, I, I, P, P, P]
     lib.mimo_attn_set_decode_kernel.restype = I
     lib.mimo_attn_set_decode_kernel.argtypes = [I]
     lib.mimo_attn_version.restype = I
@@ -106,6 +116,69 @@ def set_decode_kernel(choice: int) -> None:
     st = LIB.mimo_attn_set_decode_kernel(int(choice))
     if st != OK:
         raise MimoAttnError(st, "mimo_attn_set_decode_kernel")
+
+
+def bwd(q, k, v, sink, cu_seqlens, max_seqlen, layer_kind, window, rope_base, out, lse, dout, dlse=None,
+        rope_dims=64, v_scale=0.707, stream=None):
+    """Gradients of the forward: q/k/v/out/dout bf16 CUDA tensors, lse / dlse fp32 [Hq, T] (dlse may be
+    None).  Returns (dq fp32 [T, Hq, 192], dk fp32 [T, Hkv, 192], dv fp32 [T, Hkv, 128], dsink fp32 [Hq] or
+    None)."""
+    import torch
+    T, hq, dqk = q.shape
+    hkv, dv_ = v.shape[1], v.shape[2]
+    dq = torch.empty((T, hq, dqk), dtype=torch.float32, device=q.device)
+    dk = torch.empty((T, hkv, dqk), dtype=torch.float32, device=q.device)
+    dv = torch.empty((T, hkv, dv_), dtype=torch.float32, device=q.device)
+    dsink = None if sink is None else torch.empty((hq,), dtype=torch.float32, device=q.device)
+    dims = make_dims(cu_seqlens.numel() - 1, T, max_seqlen, hq, hkv)
+    ptr = lambda t: None if t is None else t.data_ptr()
+    st = LIB.mimo_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), ptr(sink), cu_seqlens.data_ptr(),
+                           ctypes.byref(dims), int(layer_kind), int(window), float(rope_base), int(rope_dims),
+                           float(v_scale), out.data_ptr(), lse.data_ptr(), dout.data_ptr(), ptr(dlse),
+                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ptr(dsink), _stream_handle(stream))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_attn_bwd")
+    return dq, dk, dv, dsink
+
+
+def fp8_dequant_blockwise(codes, scale_inv, block=(128, 128), out=None, stream=None):
+    """uint8 E4M3 codes [rows, cols] and fp32 scale_inv [ceil(rows/b0), ceil(cols/b1)] (CUDA) -> bf16."""
+    import torch
+    rows, cols = codes.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=codes.device)
+    st = LIB.mimo_fp8_dequant_blockwise(codes.data_ptr(), scale_inv.data_ptr(), rows, cols, int(block[0]),
+                                        int(block[1]), out.data_ptr(), _stream_handle(stream))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_fp8_dequant_blockwise")
+    return out
+
+
+def qkv_split(fused, num_q_heads, num_kv_heads, stream=None):
+    """bf16 fused [T, Hkv * (Hq/Hkv*192 + 320)] (CUDA) -> q [T, Hq, 192], k [T, Hkv, 192], v [T, Hkv, 128]."""
+    import torch
+    T = fused.shape[0]
+    q = torch.empty((T, num_q_heads, 192), dtype=torch.bfloat16, device=fused.device)
+    k = torch.empty((T, num_kv_heads, 192), dtype=torch.bfloat16, device=fused.device)
+    v = torch.empty((T, num_kv_heads, 128), dtype=torch.bfloat16, device=fused.device)
+    st = LIB.mimo_qkv_split(fused.data_ptr(), T, int(num_q_heads), int(num_kv_heads), q.data_ptr(), k.data_ptr(),
+                            v.data_ptr(), _stream_handle(stream))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_qkv_split")
+    return q, k, v
+
+
+def moe_route(logits, bias, top_k=8, normalize=True, stream=None):
+    """fp32 logits [T, E] and bias [E] (CUDA) -> ids int32 [T, top_k], weights fp32 [T, top_k]."""
+    import torch
+    T, E = logits.shape
+    ids = torch.empty((T, top_k), dtype=torch.int32, device=logits.device)
+    w = torch.empty((T, top_k), dtype=torch.float32, device=logits.device)
+    st = LIB.mimo_moe_route(logits.data_ptr(), bias.data_ptr(), T, int(E), int(top_k), int(bool(normalize)),
+                            ids.data_ptr(), w.data_ptr(), _stream_handle(stream))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_moe_route")
+    return ids, w
 
 
 def profile_start() -> None:

@@ -9,8 +9,8 @@ section 5.4 Notable quirks; miles PR #3648 "add MiMo-V2.6-Flash-RL support",
 Design Notes): sliding-window layers attend the query plus 128 previous keys
 with a learnable sink, 8 KV heads and RoPE base 1e4; global layers are causal
 with 4 KV heads, RoPE base 1e7 and no sink; Q/K are 192-dim, V is 128-dim and
-scaled by 0.707; RoPE covers 64 of the 192 Q/K dims.  The 64 query heads are a
-choice of this build (the pages do not state the query-head count).
+scaled by 0.707; RoPE covers 64 of the 192 Q/K dims.  The query-head count
+is not stated there; 64 query heads (8 per KV head on the sliding layer) is a chosen value.
 """
 from __future__ import annotations
 

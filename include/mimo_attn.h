@@ -282,6 +282,61 @@ MIMO_API int mimo_attn_decode(const void* q, const void* k_cache, const void* v_
 typedef enum { MIMO_DECODE_AUTO = 0, MIMO_DECODE_CUDA_CORES = 1, MIMO_DECODE_TENSOR = 2 } mimo_decode_choice;
 MIMO_API int mimo_attn_set_decode_kernel(int choice);
 
+/*
+ * Backward of mimo_attn_fwd (miles PR #3648 trains this layer; the LSE with the
+ * sink included is the convention it needs).  Inputs as mimo_attn_fwd, plus the
+ * forward's out (bf16 [T, Hq, 128]) and lse (fp32 [Hq, T]), dout = dL/dout
+ * (bf16 [T, Hq, 128]) and dlse = dL/dlse (fp32 [Hq, T], NULL = 0), all device.
+ * Outputs (device, fp32, overwritten): dq [T, Hq, 192], dk [T, Hkv, 192],
+ * dv [T, Hkv, 128] and dsink [Hq] (required iff sink is given).  dL/ds_j =
+ * P_j (dout . v_scale v_j - D + dlse) with D = dout . out; the rotation of the
+ * first 64 dims is taken back by its transpose.  FP32 on the CUDA cores
+ * (accumulation with atomics: the result is not bit-reproducible run to run).
+ * Scratch: Hq * T * 4 bytes from the library's pool.  Does not synchronise.
+ */
+MIMO_API int mimo_attn_bwd(const void* q, const void* k, const void* v, const float* sink,
+                           const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind,
+                           int window, double rope_base, int rope_dims, float v_scale, const void* out,
+                           const float* lse, const void* dout, const float* dlse, float* dq, float* dk,
+                           float* dv, float* dsink, void* stream);
+
+/*
+ * FP8 blockwise dequant of a weight matrix (Megatron-Bridge API doc
+ * "mimo_v2_flash_bridge", _dequant_fp8_blockwise: out = fp8 value times
+ * scale_inv; miles docs section 3.1: each kv-head shard of the fused qkv_proj
+ * has its own block scales).  codes: E4M3 bytes [rows, cols] (device, 16-byte
+ * aligned, cols a multiple of 16); scale_inv: fp32 [ceil(rows / block_rows),
+ * ceil(cols / block_cols)] (device); out: bf16 [rows, cols] (device), each the
+ * round-to-nearest-even of the exact product.  The pages do not give the block
+ * size (128 x 128 is the usual one).  Does not synchronise.
+ */
+MIMO_API int mimo_fp8_dequant_blockwise(const void* codes, const float* scale_inv, int64_t rows, int64_t cols,
+                                        int block_rows, int block_cols, void* out, void* stream);
+
+/*
+ * Split of the kv-head-interleaved fused QKV output (miles docs section 1 and
+ * 3.1) into the q, k, v this library's attention takes: fused bf16
+ * [T, Hkv * (Hq/Hkv * 192 + 192 + 128)], where KV group g holds its query heads,
+ * then its K head, then its V head; q bf16 [T, Hq, 192], k [T, Hkv, 192],
+ * v [T, Hkv, 128].  All device, 16-byte aligned.  Does not synchronise.
+ */
+MIMO_API int mimo_qkv_split(const void* fused, int64_t tokens, int num_q_heads, int num_kv_heads, void* q,
+                            void* k, void* v, void* stream);
+
+/*
+ * MoE routing (miles docs section 1: 256 routed experts, top-8 sigmoid routing
+ * with a fixed score-correction bias; router logits in FP32 per the SGLang
+ * cookbook section 2).  logits fp32 [T, E], bias fp32 [E] (E a multiple of 32,
+ * at most 256); ids int32 [T, top_k] in descending score + bias (ties to the
+ * lower expert), weights fp32 [T, top_k]: the chosen experts' sigmoid scores,
+ * normalised to sum to one when normalize != 0.  The choice is taken on FP32
+ * keys fp32(sigmoid) + bias.  The pages do not say where the bias enters or
+ * whether the weights are normalised: this is the plain reading.  Device
+ * pointers.  Does not synchronise.
+ */
+MIMO_API int mimo_moe_route(const float* logits, const float* bias, int64_t tokens, int num_experts, int top_k,
+                            int normalize, int32_t* ids, float* weights, void* stream);
+
 /* ABI version: (major << 16) | minor. */
 MIMO_API int mimo_attn_version(void);
 

@@ -21,14 +21,14 @@ def M():
 
 def header_functions():
     src = open(os.path.join(ROOT, "include", "mimo_attn.h")).read()
-    return sorted(set(re.findall(r"MIMO_API\s+[\w\s\*]*?\b(mimo_attn_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"MIMO_API\s+[\w\s\*]*?\b(mimo_\w+)\s*\(", src)))
 
 
 def test_exports_every_declared_symbol(M):
     declared = header_functions()
     assert declared and sorted(M.SYMBOLS) == declared
     nm = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True, text=True, check=True).stdout
-    exported = set(re.findall(r"\bT (mimo_attn_\w+)", nm))
+    exported = set(re.findall(r"\bT (mimo_\w+)", nm))
     assert set(declared) <= exported
     for name in declared:
         assert getattr(M.LIB, name) is not None

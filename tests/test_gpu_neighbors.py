@@ -1,0 +1,71 @@
+"""GPU parity of the steps beside the attention kernel (FP8 blockwise dequant, fused-QKV split, MoE
+router) against the numpy oracle: bit-exact for the dequant and the split; the router's choice equal
+where the FP32 keys are not tied, weights to FP32 rounding."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import neighbors as NB
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def f64_to_bf16_bits(x):
+    """Round-to-nearest-even of FP64 values to BF16 (one rounding; finite values in FP32 range)."""
+    b = np.asarray(x, dtype=np.float64).view(np.uint64)
+    lsb = (b >> np.uint64(45)) & np.uint64(1)
+    r = (b + np.uint64((1 << 44) - 1) + lsb) & ~np.uint64((1 << 45) - 1)  # 8 significant bits left
+    f32 = r.view(np.float64).astype(np.float32)  # exact: at most 8 significant bits
+    return (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+@pytest.mark.parametrize("shape,block", [((300, 512), (128, 128)), ((128, 16), (128, 128)), ((77, 96), (32, 48))])
+def test_fp8_dequant_bit_exact(shape, block):
+    from global_attention_moe_b200 import mimo_attn as M
+    rng = np.random.default_rng(51)
+    codes = rng.integers(0, 256, size=shape).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3F  # no NaN codes
+    gs = (-(-shape[0] // block[0]), -(-shape[1] // block[1]))
+    scale = (np.exp2(rng.integers(-8, 8, size=gs)) * rng.uniform(1, 2, size=gs)).astype(np.float32)
+    out = M.fp8_dequant_blockwise(torch.from_numpy(codes).cuda(), torch.from_numpy(scale).cuda(), block)
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    want = f64_to_bf16_bits(NB.dequant_fp8_blockwise(codes, scale.astype(np.float64), block))
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("hq,hkv,T", [(64, 8, 257), (64, 4, 100), (8, 8, 3), (6, 2, 9)])
+def test_qkv_split_bit_exact(hq, hkv, T):
+    from global_attention_moe_b200 import mimo_attn as M
+    rng = np.random.default_rng(52)
+    width = hkv * (hq // hkv * 192 + 192 + 128)
+    fused = rng.integers(0, 1 << 16, size=(T, width)).astype(np.uint16)
+    q, k, v = M.qkv_split(torch.from_numpy(fused.view(np.int16)).cuda().view(torch.bfloat16), hq, hkv)
+    rq, rk, rv = NB.split_qkv(fused, hq, hkv)
+    for a, r in ((q, rq), (k, rk), (v, rv)):
+        assert np.array_equal(a.view(torch.int16).cpu().numpy().view(np.uint16), r)
+
+
+@pytest.mark.parametrize("E,k,T", [(256, 8, 4099), (64, 8, 33), (32, 1, 7)])
+def test_route(E, k, T):
+    from global_attention_moe_b200 import mimo_attn as M
+    rng = np.random.default_rng(53)
+    logits = (rng.standard_normal((T, E)) * 2).astype(np.float32)
+    bias = (rng.standard_normal(E) * 0.1).astype(np.float32)
+    ids, w = M.moe_route(torch.from_numpy(logits).cuda(), torch.from_numpy(bias).cuda(), k)
+    ids, w = ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+    rid, rw, key = NB.route(logits, bias, k)
+    same = np.all(ids == rid, axis=1)
+    # rows that differ must be a different order of FP32 keys that tie within one rounding of the sigmoid
+    for t in np.nonzero(~same)[0]:
+        kk = key[t, ids[t]]
+        assert len(set(ids[t].tolist())) == k
+        assert np.all(np.abs(np.sort(kk)[::-1] - key[t, rid[t]]) <= 2 * np.spacing(np.abs(key[t, rid[t]])))
+    assert same.mean() > 0.999
+    assert np.max(np.abs(w[same] - rw[same])) <= 1e-6
+    assert np.allclose(w.sum(1), 1.0, atol=1e-6)
