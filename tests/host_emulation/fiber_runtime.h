@@ -1,0 +1,270 @@
+// fiber_runtime.h -- host emulation of the CUDA features that the CUDA-core kernels (backward, FP8
+// dequant, fused-QKV split, MoE router) use, so that their unchanged source runs on the CPU in tests:
+//   - one fiber (ucontext) per CUDA thread, a cooperative scheduler per block, blocks one after another;
+//   - __syncthreads / __syncwarp as barriers over the block's / warp's live fibers (exited threads do
+//     not count, as on the GPU); a barrier that can never complete is reported as a deadlock;
+//   - warp shuffles through an exchange array, with an error if a lane of the warp has exited;
+//   - atomics as plain read-modify-write (a single OS thread runs every fiber);
+//   - every buffer, and the block's dynamic shared memory, sits against a PROT_NONE guard page (at its
+//     end in mode 0, at its start in mode 1), so an out-of-range access faults on the host.
+// Device math: __sincosf is taken as the host's sinf/cosf (the GPU's is an approximation with an
+// absolute error near 2^-21 on [-pi, pi]); exp2f, fmaf and the BF16/FP8 conversions are the host forms.
+// Test infrastructure only: nothing in the library includes or calls it.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <sys/mman.h>
+#include <ucontext.h>
+#include <unistd.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <functional>
+#include <vector>
+
+#undef __global__
+#define __global__
+#undef __device__
+#define __device__
+#undef __host__
+#define __host__
+#define __launch_bounds__(...)
+#define __grid_constant__
+#undef __shared__
+#define __shared__ static
+
+using std::max;
+using std::min;
+
+namespace hemu {
+
+inline int g_mode = 0;  // 0: buffers end at a guard page; 1: buffers start right after one
+inline long g_page = sysconf(_SC_PAGESIZE);
+
+struct Alloc {
+  void* map;
+  size_t map_bytes;
+};
+inline std::vector<std::pair<void*, Alloc>> g_allocs;
+
+inline void* guarded_alloc(size_t nbytes) {
+  const size_t n16 = (nbytes + 15) & ~size_t(15);
+  const size_t body = (n16 + g_page - 1) / g_page * g_page;
+  const size_t total = body + 2 * g_page;
+  uint8_t* m = static_cast<uint8_t*>(mmap(nullptr, total, PROT_READ | PROT_WRITE, MAP_PRIVATE | MAP_ANONYMOUS, -1, 0));
+  if (m == MAP_FAILED) return nullptr;
+  mprotect(m, g_page, PROT_NONE);
+  mprotect(m + g_page + body, g_page, PROT_NONE);
+  uint8_t* p = g_mode == 0 ? m + g_page + body - n16 : m + g_page;
+  std::memset(p, 0xA5, n16);
+  g_allocs.push_back({p, {m, total}});
+  return p;
+}
+
+inline void guarded_free(void* p) {
+  for (size_t i = 0; i < g_allocs.size(); ++i)
+    if (g_allocs[i].first == p) {
+      munmap(g_allocs[i].second.map, g_allocs[i].second.map_bytes);
+      g_allocs.erase(g_allocs.begin() + i);
+      return;
+    }
+}
+
+struct Fiber {
+  ucontext_t ctx;
+  bool done;
+  int wait;  // 0 runnable, 1 block barrier, 2 warp barrier
+  uint64_t gen;
+};
+
+inline uint3 g_tid_cur, g_bid_cur;
+inline dim3 g_grid_dim, g_block_dim;
+inline std::vector<Fiber> g_fibers;
+inline std::vector<uint8_t*> g_stacks;
+inline constexpr size_t kStack = 256 * 1024;
+inline ucontext_t g_sched;
+inline int g_cur = -1;
+inline uint64_t g_block_gen;
+inline int g_block_arrived;
+inline std::vector<uint64_t> g_warp_gen;
+inline std::vector<int> g_warp_arrived;
+inline std::function<void()> g_body;
+inline uint8_t* g_smem = nullptr;
+inline uint64_t g_xch[64][32];
+inline int g_errors = 0;
+
+inline int lin_tid() { return static_cast<int>(g_tid_cur.x + g_block_dim.x * (g_tid_cur.y + g_block_dim.y * g_tid_cur.z)); }
+
+inline void syncthreads() {
+  Fiber& f = g_fibers[g_cur];
+  f.wait = 1;
+  f.gen = g_block_gen;
+  ++g_block_arrived;
+  swapcontext(&f.ctx, &g_sched);
+}
+
+inline void syncwarp() {
+  Fiber& f = g_fibers[g_cur];
+  const int w = lin_tid() / 32;
+  f.wait = 2;
+  f.gen = g_warp_gen[w];
+  ++g_warp_arrived[w];
+  swapcontext(&f.ctx, &g_sched);
+}
+
+template <class T>
+inline T shfl_idx(T v, int src) {
+  static_assert(sizeof(T) <= 8, "shuffle width");
+  const int t = lin_tid(), w = t / 32, l = t % 32;
+  std::memcpy(&g_xch[w][l], &v, sizeof(T));
+  syncwarp();
+  T r;
+  std::memcpy(&r, &g_xch[w][src & 31], sizeof(T));
+  syncwarp();
+  return r;
+}
+
+inline void trampoline() {
+  g_body();
+  g_fibers[g_cur].done = true;
+}
+
+inline uint8_t* g_smem_map = nullptr;
+inline size_t g_smem_map_bytes = 0;
+
+inline void set_smem(size_t bytes) {
+  if (g_smem_map) munmap(g_smem_map, g_smem_map_bytes);
+  const size_t n16 = (bytes + 15) & ~size_t(15);
+  const size_t body = (n16 + g_page - 1) / g_page * g_page + g_page;
+  g_smem_map_bytes = body + 2 * g_page;
+  g_smem_map = static_cast<uint8_t*>(
+      mmap(nullptr, g_smem_map_bytes, PROT_READ | PROT_WRITE, MAP_PRIVATE | MAP_ANONYMOUS, -1, 0));
+  mprotect(g_smem_map, g_page, PROT_NONE);
+  mprotect(g_smem_map + g_page + body, g_page, PROT_NONE);
+  g_smem = g_mode == 0 ? g_smem_map + g_page + body - n16 : g_smem_map + g_page;
+}
+
+// Runs fn (the kernel call) for every thread of every block.  Returns false on a barrier deadlock or a
+// shuffle with exited lanes.
+inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function<void()>& fn) {
+  g_grid_dim = grid;
+  g_block_dim = block;
+  const int nt = static_cast<int>(block.x * block.y * block.z);
+  const int nw = (nt + 31) / 32;
+  if (nw > 64) return false;
+  if (smem_bytes > 227 * 1024) {
+    std::fprintf(stderr, "emu: dynamic shared memory %zu above the per-block limit\n", smem_bytes);
+    return false;
+  }
+  set_smem(smem_bytes > 0 ? smem_bytes : 16);
+  while (static_cast<int>(g_stacks.size()) < nt) g_stacks.push_back(static_cast<uint8_t*>(std::malloc(kStack)));
+  g_fibers.assign(nt, Fiber{});
+  g_warp_gen.assign(nw, 0);
+  g_warp_arrived.assign(nw, 0);
+  g_body = fn;
+  for (unsigned bz = 0; bz < grid.z; ++bz)
+    for (unsigned by = 0; by < grid.y; ++by)
+      for (unsigned bx = 0; bx < grid.x; ++bx) {
+        g_bid_cur = make_uint3(bx, by, bz);
+        std::memset(g_smem, 0xCD, smem_bytes);
+        g_block_gen = 0;
+        g_block_arrived = 0;
+        std::fill(g_warp_arrived.begin(), g_warp_arrived.end(), 0);
+        for (int i = 0; i < nt; ++i) {
+          Fiber& f = g_fibers[i];
+          f.done = false;
+          f.wait = 0;
+          f.gen = 0;
+          getcontext(&f.ctx);
+          f.ctx.uc_stack.ss_sp = g_stacks[i];
+          f.ctx.uc_stack.ss_size = kStack;
+          f.ctx.uc_link = &g_sched;
+          makecontext(&f.ctx, trampoline, 0);
+        }
+        for (;;) {
+          bool progress = false;
+          int alive = 0;
+          std::vector<int> alive_w(nw, 0);
+          for (int i = 0; i < nt; ++i) {
+            Fiber& f = g_fibers[i];
+            if (f.done) continue;
+            if (f.wait == 1 && f.gen == g_block_gen) continue;
+            if (f.wait == 2 && f.gen == g_warp_gen[i / 32]) continue;
+            f.wait = 0;
+            g_cur = i;
+            g_tid_cur = make_uint3(i % block.x, (i / block.x) % block.y, i / (block.x * block.y));
+            swapcontext(&g_sched, &f.ctx);
+            progress = true;
+          }
+          for (int i = 0; i < nt; ++i)
+            if (!g_fibers[i].done) {
+              ++alive;
+              ++alive_w[i / 32];
+            }
+          if (alive == 0) break;
+          if (g_block_arrived > 0 && g_block_arrived == alive) {
+            ++g_block_gen;
+            g_block_arrived = 0;
+            progress = true;
+          }
+          for (int w = 0; w < nw; ++w)
+            if (g_warp_arrived[w] > 0 && g_warp_arrived[w] == alive_w[w]) {
+              if (alive_w[w] != std::min(32, nt - 32 * w)) {
+                std::fprintf(stderr, "emu: warp-collective with exited lanes (block %u,%u,%u warp %d)\n", bx, by, bz, w);
+                ++g_errors;
+              }
+              ++g_warp_gen[w];
+              g_warp_arrived[w] = 0;
+              progress = true;
+            }
+          if (!progress) {
+            std::fprintf(stderr, "emu: barrier deadlock in block %u,%u,%u (alive %d, at block barrier %d)\n", bx, by,
+                         bz, alive, g_block_arrived);
+            ++g_errors;
+            return false;
+          }
+        }
+      }
+  return g_errors == 0;
+}
+
+}  // namespace hemu
+
+#define threadIdx (hemu::g_tid_cur)
+#define blockIdx (hemu::g_bid_cur)
+#define gridDim (hemu::g_grid_dim)
+#define blockDim (hemu::g_block_dim)
+#define __syncthreads() hemu::syncthreads()
+#define __syncwarp(...) hemu::syncwarp()
+
+template <class T>
+inline T __ldg(const T* p) { return *p; }
+template <class T>
+inline T __shfl_xor_sync(unsigned, T v, int o) { return hemu::shfl_idx(v, (hemu::lin_tid() % 32) ^ o); }
+template <class T>
+inline T __shfl_sync(unsigned, T v, int src) { return hemu::shfl_idx(v, src); }
+inline float atomicAdd(float* p, float v) {
+  const float o = *p;
+  *p = o + v;
+  return o;
+}
+inline unsigned atomicOr(unsigned* p, unsigned v) {
+  const unsigned o = *p;
+  *p = o | v;
+  return o;
+}
+inline float __uint_as_float(uint32_t u) {
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+inline void __sincosf(float x, float* s, float* c) {
+  *s = std::sin(x);
+  *c = std::cos(x);
+}

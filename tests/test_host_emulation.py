@@ -1,0 +1,56 @@
+"""The CUDA-core kernels (backward, FP8 blockwise dequant, fused-QKV split, MoE router) and their C entry
+points, compiled unchanged for the CPU against a fiber runtime (tests/host_emulation), compared with
+the oracle.  Every buffer and the shared-memory block sit against guard pages, once at their end and
+once at their start, so any out-of-range index faults; barriers and warp shuffles are checked for
+deadlock and exited lanes.  This checks the kernels' index arithmetic, masks and block-level
+protocol on the CPU; the GPU parity tests check them on the device."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+EMU = os.path.join(HERE, "host_emulation")
+sys.path.insert(0, EMU)
+import build_host  # noqa: E402
+from cases import CASES  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def host_lib(tmp_path_factory):
+    return build_host.build(str(tmp_path_factory.mktemp("host_kernels")))
+
+
+def run_cases(lib, mode, names):
+    r = subprocess.run([sys.executable, os.path.join(EMU, "cases.py"), lib, str(mode), *names],
+                       capture_output=True, text=True, timeout=600)
+    return r.returncode, (r.stdout + r.stderr)[-2000:]
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_kernels_match_oracle(host_lib, mode):
+    rc, log = run_cases(host_lib, mode, list(CASES))
+    assert rc == 0, log
+
+
+# Mistakes planted in the host copy of the kernels, each of which the cases above must catch.
+PLANTED = [
+    ("one vector read past the end of the codes", "e < n_vec;", "e <= n_vec;", "dequant"),
+    ("shared-memory block one row-vector short", "kRows * kPS + 2 * kRows) * 4;", "kRows * kPS + kRows) * 4;",
+     "bwd_window0"),
+    ("barrier between the K/V load and its rotation dropped",
+     "    __syncthreads();\n    for (int e = tid; e < kChunk * (kRopeDims / 2); e += kThreads) {",
+     "    for (int e = tid; e < kChunk * (kRopeDims / 2); e += kThreads) {", "bwd_window0"),
+    ("window mask one key short", "pos - kpos <= P.window", "pos - kpos < P.window", "bwd_window31_mqa"),
+    ("router ties to the higher expert", "(ok == bk && oe < be)", "(ok == bk && oe > be)", "route"),
+]
+
+
+@pytest.mark.parametrize("what,old,new,case", PLANTED, ids=[p[0] for p in PLANTED])
+def test_planted_mistake_is_caught(tmp_path, what, old, new, case):
+    src = build_host.generate()
+    assert src.count(old) == 1, what
+    lib = build_host.build(str(tmp_path), src.replace(old, new))
+    rc = max(run_cases(lib, m, [case])[0] != 0 for m in (0, 1))
+    assert rc, f"not caught: {what}"
