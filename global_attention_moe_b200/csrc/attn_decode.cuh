@@ -14,12 +14,15 @@
 // forward's output rows for those positions.
 //
 // This file holds the FP32 CUDA-core form of the per-split kernel (the
-// cross-check of the tensor-core kernel in attn_decode_tc.cuh) and the combine
-// kernel both use: one CTA per (sequence, KV head, key split) holds the
-// q_len x (Hq/Hkv) query rows that share the KV head, walks its keys 32 at a
-// time (one key per lane, rows spread over the warps) with an online softmax,
-// and writes a partial (max, sum, O) per row; the combine kernel merges the
-// splits that hold keys with the sink and writes BF16 out and the FP32 LSE.
+// cross-check of the tensor-core kernel in attn_decode_tc.cuh, and the kernel
+// for chunked prefill) and the combine kernel both use.  The q_len x (Hq/Hkv)
+// query rows that share a KV head are cut into tiles of 128 rows; one CTA per
+// (key split, row tile, KV head, sequence) holds the tile's rows, walks the
+// split's keys that those rows may see 32 at a time (one key per lane, rows
+// spread over the warps) with an online softmax, and writes a partial (max,
+// sum, O) per row.  The combine kernel merges, per token and head, the splits
+// that overlap its tile's keys with the sink and writes BF16 out and the FP32
+// LSE.
 #pragma once
 
 #include "params.cuh"
@@ -34,7 +37,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = 32;                        // keys per step, one per lane
-constexpr int kMaxRows = 128;                     // q_len x (Hq/Hkv) query rows per CTA
+constexpr int kMaxRows = 128;                     // query rows per CTA (one row tile)
 constexpr int kRowsPerWarp = kMaxRows / kWarps;   // row r belongs to warp r % kWarps
 constexpr int kQStride = kHeadDimQK;              // Q rows are read as broadcast 16-byte loads
 constexpr int kKStride = kHeadDimQK + 4;          // 16-byte aligned, lane stride of 4 banks: conflict-free
@@ -60,6 +63,7 @@ struct DecParams {
   int32_t hq, hkv, group;
   int32_t window;             // < 0: global causal layer
   int32_t splits, split_keys;
+  int32_t qtiles;             // row tiles per sequence and KV head (CUDA-core kernel; 1 for the tensor-core one)
   float scale_log2;           // log2(e) / sqrt(192)
   float v_scale;
   uint64_t wait_limit_ns;     // bound of every barrier wait (tensor-core kernel)
@@ -70,6 +74,14 @@ struct DecParams {
 __device__ __forceinline__ int key_lo(int kv_len, int q_len, int window) {
   const int p0 = kv_len - q_len;  // first query's position
   return (window >= 0 && p0 - window > 0) ? p0 - window : 0;
+}
+
+// Keys [lo_t, hi_t) that the query rows row0 .. row0 + rows - 1 of a sequence may see (row r is query
+// r / group, at position p0 + r / group).
+__device__ __forceinline__ void tile_keys(int p0, int row0, int rows, int group, int window, int& lo_t, int& hi_t) {
+  const int pos_first = p0 + row0 / group, pos_last = p0 + (row0 + rows - 1) / group;
+  lo_t = (window >= 0 && pos_first - window > 0) ? pos_first - window : 0;
+  hi_t = pos_last + 1;
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
@@ -97,32 +109,40 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial_kernel(const __g
   float* sK = sQ + kMaxRows * kQStride;          // [kChunk][kKStride]
   float* sV = sK + kChunk * kKStride;            // [kChunk][128]
   float* sP = sV + kChunk * kHeadDimV;           // [kWarps][kRowsPerWarp][kPStride]
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x % P.splits, qt = blockIdx.x / P.splits, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const int q_beg = __ldg(P.cu_q + b), q_len = __ldg(P.cu_q + b + 1) - q_beg;
   const int kv_beg = __ldg(P.kv_indptr + b), kv_len = __ldg(P.kv_indptr + b + 1) - kv_beg;
-  const int rows = q_len * P.group;
+  const int all_rows = q_len * P.group;
   // Inconsistent bounds: report and touch nothing (the combine kernel skips the same rows).
-  if (q_len < 0 || kv_len < 0 || q_len > kv_len || rows > kMaxRows || q_beg < 0 || q_beg + q_len > P.total_q ||
-      kv_beg < 0 || kv_beg + kv_len > P.total_kv) {
-    if (tid == 0 && split == 0 && g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
+  if (q_len < 0 || kv_len < 0 || q_len > kv_len || all_rows > kMaxRows * P.qtiles || q_beg < 0 ||
+      q_beg + q_len > P.total_q || kv_beg < 0 || kv_beg + kv_len > P.total_kv) {
+    if (tid == 0 && split == 0 && qt == 0 && g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
     return;
   }
-  if (rows == 0) return;
+  const int row0 = kMaxRows * qt;  // the tile's rows: row0 .. row0 + rows - 1 of the sequence's
+  const int rows = min(kMaxRows, all_rows - row0);
+  if (rows <= 0) return;
   const int p0 = kv_len - q_len;
   const int lo = key_lo(kv_len, q_len, P.window);
   if (kv_len - lo > P.splits * P.split_keys) {  // more keys than the launch covers (max_kv_len too small)
-    if (tid == 0 && split == 0 && g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
+    if (tid == 0 && split == 0 && qt == 0 && g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
     return;
   }
-  const int k_beg = lo + split * P.split_keys;
-  const int k_end = min(kv_len, k_beg + P.split_keys);
+  // the split's keys, clipped to those the tile's rows may see; a split with none is not read back
+  int lo_t, hi_t;
+  tile_keys(p0, row0, rows, P.group, P.window, lo_t, hi_t);
+  const int s_beg = lo + split * P.split_keys;
+  const int k_beg = max(s_beg, lo_t);
+  const int k_end = min(min(kv_len, s_beg + P.split_keys), hi_t);
+  if (k_end <= k_beg) return;
 
-  // Q rows r = i * group + hh (query i of the sequence, head g * group + hh), rotated at p0 + i.
+  // Q rows r = row0 + tile row = i * group + hh (query i of the sequence, head g * group + hh), rotated
+  // at p0 + i.
   for (int e = tid; e < rows * (kHeadDimQK / 8); e += kThreads) {
     const int r = e / (kHeadDimQK / 8), c = e % (kHeadDimQK / 8);
-    const int i = r / P.group, hh = r % P.group;
+    const int i = (row0 + r) / P.group, hh = (row0 + r) % P.group;
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(
         P.q + (static_cast<size_t>(q_beg + i) * P.hq + g * P.group + hh) * kHeadDimQK) + c);
     bf16x8_to_f32(u, sQ + r * kQStride + 8 * c);
@@ -130,7 +150,7 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial_kernel(const __g
   __syncthreads();
   for (int e = tid; e < rows * (kRopeDims / 2); e += kThreads) {
     const int r = e / (kRopeDims / 2), i = e % (kRopeDims / 2);
-    rope_pair_f32(sQ + r * kQStride, i, p0 + r / P.group, P.theta[i]);
+    rope_pair_f32(sQ + r * kQStride, i, p0 + (row0 + r) / P.group, P.theta[i]);
   }
 
   // Per-row state of this warp's rows r = warp + kWarps * k.
@@ -212,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial_kernel(const __g
     for (int k = 0; k < kRowsPerWarp; ++k) {  // unrolled: the per-row state stays in registers
       const int r = warp + kWarps * k;
       if (r >= rows) break;  // warp-uniform
-      const int pos = p0 + r / P.group;
+      const int pos = p0 + (row0 + r) / P.group;
       const bool ok = lane < n && j <= pos && (P.window < 0 || pos - j <= P.window);
       const float s = ok ? acc[k] * P.scale_log2 : -INFINITY;
       float mx = s;
@@ -254,7 +274,7 @@ __global__ void __launch_bounds__(kThreads) attn_decode_partial_kernel(const __g
   for (int k = 0; k < kRowsPerWarp; ++k) {
     const int r = warp + kWarps * k;
     if (r >= rows) break;
-    const int i = r / P.group, hh = r % P.group;
+    const int i = (row0 + r) / P.group, hh = (row0 + r) % P.group;
     const size_t slot = (static_cast<size_t>(q_beg + i) * P.hq + g * P.group + hh) * P.splits + split;
 #pragma unroll
     for (int d = 0; d < 4; ++d) P.part_o[slot * kHeadDimV + lane + 32 * d] = o[k][d];
@@ -280,19 +300,25 @@ __global__ void __launch_bounds__(kThreads) attn_decode_combine_kernel(const __g
   const int q_beg = __ldg(P.cu_q + lo_b), q_len = __ldg(P.cu_q + lo_b + 1) - q_beg;
   const int kv_beg = __ldg(P.kv_indptr + lo_b), kv_len = __ldg(P.kv_indptr + lo_b + 1) - kv_beg;
   // the partial kernel's checks: such rows were reported there and stay unwritten
-  if (q_len <= 0 || q_len > kv_len || q_len * P.group > kMaxRows || q_beg < 0 || q_beg + q_len > P.total_q ||
-      kv_beg < 0 || kv_beg + kv_len > P.total_kv)
+  if (q_len <= 0 || q_len > kv_len || q_len * P.group > kMaxRows * P.qtiles || q_beg < 0 ||
+      q_beg + q_len > P.total_q || kv_beg < 0 || kv_beg + kv_len > P.total_kv)
     return;
-  const int n_keys = kv_len - key_lo(kv_len, q_len, P.window);
-  if (n_keys > P.splits * P.split_keys) return;
+  const int lo = key_lo(kv_len, q_len, P.window);
+  if (kv_len - lo > P.splits * P.split_keys) return;
+  // The token's row tile and the keys its rows may see: exactly the splits overlapping [lo_t, hi_t)
+  // hold written partials for the tile (one tile: every split that holds keys).
+  const int row = (t - q_beg) * P.group + h % P.group;
+  const int row0 = row / kMaxRows * kMaxRows;
+  int lo_t, hi_t;
+  tile_keys(kv_len - q_len, row0, min(kMaxRows, q_len * P.group - row0), P.group, P.window, lo_t, hi_t);
+  const int s_lo = (lo_t - lo) / P.split_keys, s_hi = (hi_t - 1 - lo) / P.split_keys;
   const size_t base = (static_cast<size_t>(t) * P.hq + h) * P.splits;
-  const int used = (n_keys + P.split_keys - 1) / P.split_keys;  // splits that hold keys (the others are not written)
   float M = P.sink != nullptr ? __ldg(P.sink + h) * kLog2e : -INFINITY;
-  for (int s = 0; s < used; ++s) M = fmaxf(M, P.part_ml[2 * (base + s)]);
+  for (int s = s_lo; s <= s_hi; ++s) M = fmaxf(M, P.part_ml[2 * (base + s)]);
   const float mb = (M == -INFINITY) ? 0.f : M;
   float L = P.sink != nullptr ? ex2_approx(__ldg(P.sink + h) * kLog2e - mb) : 0.f;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < used; ++s) {
+  for (int s = s_lo; s <= s_hi; ++s) {
     const float w = ex2_approx(P.part_ml[2 * (base + s)] - mb);
     L += P.part_ml[2 * (base + s) + 1] * w;
 #pragma unroll

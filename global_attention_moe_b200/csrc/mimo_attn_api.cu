@@ -367,6 +367,10 @@ int launch_noalloc(const void* q, const void* k, const void* v, const FwdParams&
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 
+// Query rows per KV head (q_len x Hq/Hkv) that one decode call accepts: 8192 row tiles of the CUDA-core
+// kernel (prefill chunks of up to 65536 tokens at 16 query heads per KV head).
+constexpr int64_t kMaxDecodeRows = INT64_C(1) << 20;
+
 int validate_decode(const void* q, const void* kc, const void* vc, const int32_t* idx, const int32_t* indptr,
                     const int32_t* cu_q, const float* sink, const mimo_decode_dims* d, int layer_kind, int window,
                     double rope_base, int rope_dims, float v_scale, const void* out, const float* lse) {
@@ -387,7 +391,7 @@ int validate_decode(const void* q, const void* kc, const void* vc, const int32_t
   if (!std::isfinite(v_scale)) return MIMO_ERR_INVALID_ARG;
   if (layer_kind == MIMO_LAYER_SWA && window < 0) return MIMO_ERR_INVALID_ARG;
   if (layer_kind == MIMO_LAYER_GLOBAL && sink != nullptr) return MIMO_ERR_INVALID_ARG;
-  if ((int64_t)d->max_q_len * (d->num_q_heads / d->num_kv_heads) > dec::kMaxRows) return MIMO_ERR_UNSUPPORTED;
+  if ((int64_t)d->max_q_len * (d->num_q_heads / d->num_kv_heads) > kMaxDecodeRows) return MIMO_ERR_UNSUPPORTED;
   if ((int64_t)d->cache_rows * d->num_kv_heads * kHeadDimQK > INT64_C(1) << 40) return MIMO_ERR_UNSUPPORTED;
   if (!indptr || !cu_q) return MIMO_ERR_INVALID_ARG;
   if (d->total_q > 0) {
@@ -429,13 +433,19 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   P.v_scale = v_scale;
   P.wait_limit_ns = kDefaultWaitLimitNs;
   for (int i = 0; i < kRopeDims / 2; ++i) P.theta[i] = std::pow(rope_base, -2.0 * i / kRopeDims);
-  const bool tensor = g_decode_choice.load() != MIMO_DECODE_CUDA_CORES;
+  // Query rows per KV head above 128 (chunked prefill) run on the CUDA-core kernel in 128-row tiles;
+  // the tensor-core kernel holds one tile (its M = 128 accumulator).
+  const long long all_rows = (long long)d->max_q_len * P.group;
+  const int choice = g_decode_choice.load();
+  if (choice == MIMO_DECODE_TENSOR && all_rows > dec::kMaxRows) return MIMO_ERR_UNSUPPORTED;
+  const bool tensor = choice == MIMO_DECODE_TENSOR || (choice == MIMO_DECODE_AUTO && all_rows <= dec::kMaxRows);
+  P.qtiles = tensor ? 1 : (int)std::max<long long>(1, (all_rows + dec::kMaxRows - 1) / dec::kMaxRows);
   // Keys one sequence's queries can see, at most; split them so that the work covers the SMs a few
   // times over (tensor-core kernel: persistent, one CTA per SM walking about six (sequence, KV head,
-  // split) items; CUDA-core kernel: one CTA per item, about two per SM).
+  // split) items; CUDA-core kernel: one CTA per (split, row tile) item, about two per SM).
   const long long span = (P.window >= 0) ? std::min<long long>(d->max_kv_len, (long long)P.window + d->max_q_len)
                                          : (long long)d->max_kv_len;
-  const long long base_ctas = (long long)d->num_seqs * P.hkv;
+  const long long base_ctas = (long long)d->num_seqs * P.hkv * P.qtiles;
   const long long chunk = tensor ? dtc::kChunk : dec::kChunk;
   const long long target = (tensor ? 6LL : 2LL) * info->sms;
   long long splits = std::max<long long>(1, (target + base_ctas - 1) / base_ctas);
@@ -463,7 +473,7 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
       attn_decode_tc_kernel<<<(unsigned)std::min<long long>(items, info->sms), dtc::kThreads, dtc::kSmemBytes,
                               stream>>>(P);
     } else {
-      dim3 grid((unsigned)splits, (unsigned)P.hkv, (unsigned)d->num_seqs);
+      dim3 grid((unsigned)(splits * P.qtiles), (unsigned)P.hkv, (unsigned)d->num_seqs);
       dec::attn_decode_partial_kernel<<<grid, dec::kThreads, dec::kSmemBytes, stream>>>(P);
     }
     if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;

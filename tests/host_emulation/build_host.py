@@ -1,11 +1,14 @@
-"""Compiles the library's CUDA-core kernels (backward, FP8 dequant, fused-QKV split, MoE router) and
-their host entry points for the CPU against fiber_runtime.h, into a shared library for the tests.
+"""Compiles the library's CUDA-core kernels (backward, FP8 dequant, fused-QKV split, MoE router, the
+KV-cache partial and combine kernels) and their host entry points for the CPU against
+fiber_runtime.h, into a shared library for the tests.
 
 The kernel files are taken as they are; the only source transforms are: project includes removed
 (their few definitions are pulled in by name: params.cuh whole, the error bits of sm100.cuh, the
-rope_sincos of rope_smem.cuh), the dynamic shared-memory declaration pointed at the runtime's guarded
-block, `kernel<<<grid, block, smem, stream>>>(args)` turned into a runtime launch, and in the host
-functions the device query, the pool allocation and cudaGetLastError replaced by host forms.
+rope_sincos of rope_smem.cuh, ex2_approx as the host exp2f), the dynamic shared-memory declaration
+pointed at the runtime's guarded block, the tensor-core KV-cache kernel replaced by a stub that
+records an error if it is ever launched, `kernel<<<grid, block, smem, stream>>>(args)` turned into a
+runtime launch, and in the host functions the device query, the pool allocation, the stream-ordered
+memset and cudaGetLastError replaced by host forms.
 Test infrastructure only."""
 import os
 import re
@@ -16,7 +19,8 @@ ROOT = os.path.dirname(os.path.dirname(HERE))
 CS = os.path.join(ROOT, "global_attention_moe_b200", "csrc")
 SMS = 148  # grid sizes of the grid-stride kernels follow the B200's SM count
 
-ENTRY_POINTS = ("mimo_attn_bwd", "mimo_fp8_dequant_blockwise", "mimo_qkv_split", "mimo_moe_route")
+ENTRY_POINTS = ("mimo_attn_bwd", "mimo_fp8_dequant_blockwise", "mimo_qkv_split", "mimo_moe_route",
+                "mimo_attn_decode", "mimo_attn_set_decode_kernel")
 
 
 def _read(name):
@@ -39,9 +43,23 @@ def _kernel(name):
     return s
 
 
+def _split_top(cfg):
+    """Splits a launch configuration at the commas outside parentheses."""
+    parts, depth, cur = [], 0, ""
+    for ch in cfg:
+        if ch == "," and depth == 0:
+            parts.append(cur.strip())
+            cur = ""
+            continue
+        depth += ch == "("
+        depth -= ch == ")"
+        cur += ch
+    return parts + [cur.strip()]
+
+
 def _launches(s):
     def rep(m):
-        parts = [p.strip() for p in m.group(2).split(",")]
+        parts = _split_top(m.group(2))
         smem = parts[2] if len(parts) > 2 else "0"
         return f"g_launch_ok = hemu::launch(dim3({parts[0]}), dim3({parts[1]}), {smem}, [&] {{ {m.group(1)}({m.group(3)}); }});"
     return re.subn(r"([\w:]+(?:<\d+>)?)<<<(.*?)>>>\((.*?)\);", rep, s, flags=re.S)
@@ -53,8 +71,10 @@ HOST_FORMS = [
     (r"  if \(!info \|\| !info->kernels_ready \|\| !info->pool\) return MIMO_ERR_CUDA;\n", ""),
     (r"  if \(!info\) return MIMO_ERR_CUDA;\n", ""),
     (r"info->sms", "kSms"),
-    (r"cudaMallocFromPoolAsync\(&scratch, ([^,]+), info->pool, stream\)", r"host_malloc(&scratch, \1)"),
-    (r"cudaFreeAsync\(scratch, stream\)", "(hemu::guarded_free(scratch), cudaSuccess)"),
+    (r"cudaMallocFromPoolAsync\(&(\w+), ([^,]+), info->pool, stream\)", r"host_malloc(&\1, \2)"),
+    (r"cudaFreeAsync\((\w+), stream\)", r"(hemu::guarded_free(\1), cudaSuccess)"),
+    (r"cudaMemsetAsync\(P\.item_counter, 0, sizeof\(unsigned long long\), stream\)",
+     "(std::memset(P.item_counter, 0, sizeof(unsigned long long)), cudaSuccess)"),
     (r"cudaGetLastError\(\)", "(g_launch_ok ? cudaSuccess : cudaErrorUnknown)"),
     (r"cudaMemsetAsync\(dsink, 0, ([^,]+), [^;]+\);", r"std::memset(dsink, 0, \1);"),
 ]
@@ -62,18 +82,27 @@ HOST_FORMS = [
 
 def generate() -> str:
     api = _read("mimo_attn_api.cu")
-    host = _function(api, "int launch_bwd(") + "\n".join(_function(api, f"int {e}(") for e in ENTRY_POINTS)
+    host = "\n".join([_function(api, "int launch_bwd("), _function(api, "int launch_decode(")] +
+                     [_function(api, f"int {e}(") for e in ENTRY_POINTS])
     for pat, new in HOST_FORMS:
         host, n = re.subn(pat, new, host)
         assert n >= 1, f"host form not found: {pat}"
     host, n = _launches(host)
-    assert n == 6, f"expected 6 launches, found {n}"
+    assert n == 9, f"expected 9 launches, found {n}"
     rope = _read("rope_smem.cuh")
     rope = rope[rope.index("constexpr double kTwoPi"):rope.index("// Rotates chunk pair")]
     sm100 = _read("sm100.cuh")
     a = sm100.index("enum : unsigned int {")
     errs = sm100[a:sm100.index("};", a) + 2]
     validate = api[api.index("bool aligned16(const void* p)"):api.index("void fill_params(")]
+    validate += api[api.index("// Query rows per KV head (q_len x Hq/Hkv)"):api.index("int launch_decode(")]
+    lines = [ln for ln in api.splitlines() if ln.startswith(("constexpr uint64_t kDefaultWaitLimitNs",
+                                                             "std::atomic<int> g_decode_choice", "size_t align256("))]
+    assert len(lines) == 3, lines
+    tc = _read("attn_decode_tc.cuh")
+    tc_consts = [re.search(rf"constexpr (\w+) {n} = [^;]+;", tc).group(0) for n in ("kThreads", "kChunk")]
+    tc_stub = ("namespace dtc {\n" + "\n".join(tc_consts) + "\nconstexpr uint32_t kSmemBytes = 0;\n}\n"
+               "void attn_decode_tc_kernel(const dec::DecParams&) { ++hemu::g_errors; }\n")
     wrappers = []
     for e in ENTRY_POINTS:
         sig = _function(api, f"int {e}(")
@@ -84,9 +113,11 @@ def generate() -> str:
         '#include "fiber_runtime.h"',
         f'#include "{os.path.join(ROOT, "include", "mimo_attn.h")}"',
         f'#include "{os.path.join(CS, "params.cuh")}"',
-        "namespace mimo {", errs, rope, "}",
-        _kernel("attn_bwd_simple.cuh"), _kernel("neighbors.cuh"),
-        "namespace mimo {", "namespace {", f"constexpr int kSms = {SMS};", "bool g_launch_ok = true;", validate,
+        "#include <atomic>",
+        "namespace mimo {", errs, rope, "inline float ex2_approx(float x) { return exp2f(x); }", "}",
+        _kernel("attn_bwd_simple.cuh"), _kernel("neighbors.cuh"), _kernel("attn_decode.cuh"),
+        "namespace mimo {", tc_stub, "namespace {", f"constexpr int kSms = {SMS};", "bool g_launch_ok = true;",
+        *lines, validate,
         "cudaError_t host_malloc(void** p, size_t n) { *p = hemu::guarded_alloc(n); return cudaSuccess; }",
         host, "}  // namespace", "}  // namespace mimo",
         'extern "C" {', *wrappers,

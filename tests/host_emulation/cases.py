@@ -21,7 +21,13 @@ sys.path.insert(0, os.path.dirname(TESTS))
 sys.path.insert(0, TESTS)
 import oracle  # noqa: E402
 from oracle import neighbors as NB  # noqa: E402
-from global_attention_moe_b200 import synth  # noqa: E402
+from global_attention_moe_b200 import synth, workloads as W  # noqa: E402
+from decode_helpers import decode_reference  # noqa: E402
+
+# forward tolerances (BF16 out): max-abs, rel-L2, LSE max-abs
+TOL_MAX_ABS, TOL_REL_L2, TOL_LSE = 2e-2, 5e-3, 1e-3
+DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR = 0, 1, 2
+ERR_UNSUPPORTED = 2
 
 TOL_BWD = 1e-4
 LAYER_SWA, LAYER_GLOBAL = 0, 1
@@ -31,6 +37,11 @@ vp = C.c_void_p
 class Dims(C.Structure):
     _fields_ = [(n, C.c_int32) for n in ("num_seqs", "total_tokens", "max_seqlen", "num_q_heads", "num_kv_heads",
                                          "head_dim_qk", "head_dim_v")]
+
+
+class DecodeDims(C.Structure):
+    _fields_ = [(n, C.c_int32) for n in ("num_seqs", "total_q", "total_kv", "cache_rows", "max_q_len", "max_kv_len",
+                                         "num_q_heads", "num_kv_heads", "head_dim_qk", "head_dim_v")]
 
 
 class Host:
@@ -45,6 +56,9 @@ class Host:
         L.mimo_fp8_dequant_blockwise.argtypes = [vp, vp, C.c_int64, C.c_int64, C.c_int, C.c_int, vp, vp]
         L.mimo_qkv_split.argtypes = [vp, C.c_int64, C.c_int, C.c_int, vp, vp, vp, vp]
         L.mimo_moe_route.argtypes = [vp, vp, C.c_int64, C.c_int, C.c_int, C.c_int, vp, vp, vp]
+        L.mimo_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, C.POINTER(DecodeDims), C.c_int, C.c_int,
+                                       C.c_double, C.c_int, C.c_float, vp, vp, vp]
+        L.mimo_attn_set_decode_kernel.argtypes = [C.c_int]
         self.live = []
 
     def put(self, a):
@@ -157,6 +171,33 @@ def route(H, E, k, T, normalize=True, ties=False, seed=53):
     assert np.max(np.abs(w - rw)) <= 1e-6 * max(1.0, np.max(np.abs(rw)))
 
 
+def decode(H, kv, ql, hq, hkv, layer, window, base, has_sink, seed, choice=DECODE_AUTO, expect=0):
+    """The KV-cache path through mimo_attn_decode; AUTO sends more than 128 query rows per KV head to
+    the CUDA-core kernel in 128-row tiles (the tensor-core kernel is a stub here that flags an error)."""
+    x = W.make_decode_inputs(kv, ql, hq, hkv, has_sink, seed)
+    Tq = int(sum(ql))
+    d = DecodeDims(len(kv), Tq, int(sum(kv)), x.k_cache.shape[0], max(ql), max(kv), hq, hkv, 192, 128)
+    po, pl = H.empty((Tq, hq, 128), np.uint16), H.empty((hq, Tq), np.float32)
+    assert H.L.mimo_attn_set_decode_kernel(choice) == 0
+    st = H.L.mimo_attn_decode(H.put(x.q), H.put(x.k_cache), H.put(x.v_cache), H.put(x.kv_indices),
+                              H.put(x.kv_indptr), H.put(x.cu_q), H.put(x.sink), C.byref(d), layer, window, base, 64,
+                              0.707, po, pl, None)
+    H.L.mimo_attn_set_decode_kernel(DECODE_AUTO)
+    if expect:
+        H.done(0)
+        assert st == expect, f"status {st}, expected {expect}"
+        return
+    out = synth.bf16_bits_to_f32(H.get(po, (Tq, hq, 128), np.uint16)).astype(np.float64)
+    lse = H.get(pl, (hq, Tq), np.float32).astype(np.float64)
+    H.done(st)
+    ro, rl = decode_reference(x, window if layer == LAYER_SWA else -1, base)
+    diff = out - ro
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    assert np.max(np.abs(diff)) <= TOL_MAX_ABS, np.max(np.abs(diff))
+    assert np.linalg.norm(diff) / np.linalg.norm(ro) <= TOL_REL_L2
+    assert np.max(np.abs(lse - rl)) <= TOL_LSE, np.max(np.abs(lse - rl))
+
+
 CASES = {
     "bwd_swa_sink": lambda H: bwd(H, [300, 129, 17, 1], 8, 2, LAYER_SWA, 128, 1e4, True, 41),
     "bwd_window0": lambda H: bwd(H, [200, 70], 4, 2, LAYER_SWA, 0, 1e4, False, 42),
@@ -167,6 +208,18 @@ CASES = {
     "split": lambda H: (split(H, 64, 8, 33), split(H, 6, 2, 9), split(H, 8, 8, 3)),
     "route": lambda H: (route(H, 256, 8, 200), route(H, 64, 8, 33), route(H, 32, 1, 7),
                         route(H, 256, 8, 64, normalize=False), route(H, 96, 32, 40, ties=True)),
+    # 40 new tokens x 4 heads = 160 rows (two tiles) beside one-tile sequences; keys clipped per tile
+    "decode_tiles_swa": lambda H: decode(H, [300, 90, 20], [40, 20, 20], 8, 2, LAYER_SWA, 128, 1e4, True, 61),
+    # a 300-token chunk (ten tiles) after a 300-token prefix: later tiles start several splits in
+    "decode_tiles_swa_long": lambda H: decode(H, [600, 64], [300, 64], 8, 2, LAYER_SWA, 128, 1e4, True, 65),
+    # three and seven tiles, the second sequence a whole prompt as one chunk
+    "decode_tiles_global": lambda H: decode(H, [200, 50], [36, 50], 8, 1, LAYER_GLOBAL, -1, 1e7, False, 62),
+    # the CUDA-core kernel forced on one-tile sequences (decode and speculative chunks)
+    "decode_one_tile": lambda H: decode(H, [5, 129, 300], [1, 8, 3], 8, 2, LAYER_SWA, 128, 1e4, True, 63,
+                                        choice=DECODE_CUDA_CORES),
+    # the tensor-core kernel holds one tile: forcing it above 128 rows is refused
+    "decode_tensor_refuses_tiles": lambda H: decode(H, [300], [40], 8, 2, LAYER_SWA, 128, 1e4, True, 64,
+                                                    choice=DECODE_TENSOR, expect=ERR_UNSUPPORTED),
 }
 
 if __name__ == "__main__":

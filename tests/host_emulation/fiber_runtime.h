@@ -1,12 +1,14 @@
 // fiber_runtime.h -- host emulation of the CUDA features that the CUDA-core kernels (backward, FP8
-// dequant, fused-QKV split, MoE router) use, so that their unchanged source runs on the CPU in tests:
+// dequant, fused-QKV split, MoE router, KV-cache partial and combine) use, so that their unchanged
+// source runs on the CPU in tests:
 //   - one fiber (ucontext) per CUDA thread, a cooperative scheduler per block, blocks one after another;
 //   - __syncthreads / __syncwarp as barriers over the block's / warp's live fibers (exited threads do
 //     not count, as on the GPU); a barrier that can never complete is reported as a deadlock;
 //   - warp shuffles through an exchange array, with an error if a lane of the warp has exited;
 //   - atomics as plain read-modify-write (a single OS thread runs every fiber);
 //   - every buffer, and the block's dynamic shared memory, sits against a PROT_NONE guard page (at its
-//     end in mode 0, at its start in mode 1), so an out-of-range access faults on the host.
+//     end in mode 0, at its start in mode 1), so an out-of-range access faults on the host, and is
+//     filled with 0xFF bytes (NaN as FP32 or BF16), so a read of memory nobody wrote shows in the results.
 // Device math: __sincosf is taken as the host's sinf/cosf (the GPU's is an approximation with an
 // absolute error near 2^-21 on [-pi, pi]); exp2f, fmaf and the BF16/FP8 conversions are the host forms.
 // Test infrastructure only: nothing in the library includes or calls it.
@@ -62,7 +64,7 @@ inline void* guarded_alloc(size_t nbytes) {
   mprotect(m, g_page, PROT_NONE);
   mprotect(m + g_page + body, g_page, PROT_NONE);
   uint8_t* p = g_mode == 0 ? m + g_page + body - n16 : m + g_page;
-  std::memset(p, 0xA5, n16);
+  std::memset(p, 0xFF, n16);  // NaN in every float / BF16 lane: a read of unwritten memory shows
   g_allocs.push_back({p, {m, total}});
   return p;
 }
@@ -172,7 +174,7 @@ inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function
     for (unsigned by = 0; by < grid.y; ++by)
       for (unsigned bx = 0; bx < grid.x; ++bx) {
         g_bid_cur = make_uint3(bx, by, bz);
-        std::memset(g_smem, 0xCD, smem_bytes);
+        std::memset(g_smem, 0xFF, smem_bytes);
         g_block_gen = 0;
         g_block_arrived = 0;
         std::fill(g_warp_arrived.begin(), g_warp_arrived.end(), 0);

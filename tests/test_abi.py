@@ -133,7 +133,8 @@ def test_decode_kernel_choice_values(M):
 
 @pytest.mark.parametrize("case,expect", [
     (dict(hq=6, hkv=4), 1),                 # Hq % Hkv != 0
-    (dict(max_q_len=9, total_q=20, hq=64, hkv=4), 2),  # 9 x 16 rows per KV head > 128
+    (dict(max_q_len=70000, total_q=70000, max_kv_len=70000, total_kv=70000, cache_rows=70000, hq=64, hkv=4), 2),
+    # 70000 x 16 rows per KV head > 2^20
     (dict(max_q_len=20, max_kv_len=10), 1), # max_q_len > max_kv_len
     (dict(cache_rows=0), 1),                # keys but no cache
     (dict(dqk=128), 2),

@@ -1,9 +1,11 @@
-"""The CUDA-core kernels (backward, FP8 blockwise dequant, fused-QKV split, MoE router) and their C entry
-points, compiled unchanged for the CPU against a fiber runtime (tests/host_emulation), compared with
-the oracle.  Every buffer and the shared-memory block sit against guard pages, once at their end and
-once at their start, so any out-of-range index faults; barriers and warp shuffles are checked for
-deadlock and exited lanes.  This checks the kernels' index arithmetic, masks and block-level
-protocol on the CPU; the GPU parity tests check them on the device."""
+"""The CUDA-core kernels (backward, FP8 blockwise dequant, fused-QKV split, MoE router, the KV-cache
+partial kernel in 128-row tiles and the combine) and their C entry points, compiled unchanged for the
+CPU against a fiber runtime (tests/host_emulation), compared with the oracle.  Every buffer and the
+shared-memory block sit against guard pages, once at their end and once at their start, so any
+out-of-range index faults, and start filled with NaN, so a read of memory nobody wrote shows;
+barriers and warp shuffles are checked for deadlock and exited lanes.  This checks the kernels' index
+arithmetic, masks and block-level protocol on the CPU; the GPU parity tests check them on the
+device."""
 import os
 import subprocess
 import sys
@@ -44,6 +46,10 @@ PLANTED = [
      "    for (int e = tid; e < kChunk * (kRopeDims / 2); e += kThreads) {", "bwd_window0"),
     ("window mask one key short", "pos - kpos <= P.window", "pos - kpos < P.window", "bwd_window31_mqa"),
     ("router ties to the higher expert", "(ok == bk && oe < be)", "(ok == bk && oe > be)", "route"),
+    ("decode row tiles all start at row 0", "const int row0 = kMaxRows * qt;", "const int row0 = 0;",
+     "decode_tiles_swa"),
+    ("decode combine reads splits before the tile's keys", "const int s_lo = (lo_t - lo) / P.split_keys,",
+     "const int s_lo = 0,", "decode_tiles_swa_long"),
 ]
 
 
