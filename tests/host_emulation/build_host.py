@@ -102,7 +102,8 @@ def generate() -> str:
     tc = _read("attn_decode_tc.cuh")
     tc_consts = [re.search(rf"constexpr (\w+) {n} = [^;]+;", tc).group(0) for n in ("kThreads", "kChunk")]
     tc_stub = ("namespace dtc {\n" + "\n".join(tc_consts) + "\nconstexpr uint32_t kSmemBytes = 0;\n}\n"
-               "void attn_decode_tc_kernel(const dec::DecParams&) { ++hemu::g_errors; }\n")
+               "template <class... A> void attn_decode_tc_kernel(const A&...) { ++hemu::g_errors; }\n"
+               "template <class... A> bool encode_2d(A...) { return false; }  // tensor maps: device path only\n")
     wrappers = []
     for e in ENTRY_POINTS:
         sig = _function(api, f"int {e}(")
@@ -114,6 +115,7 @@ def generate() -> str:
         f'#include "{os.path.join(ROOT, "include", "mimo_attn.h")}"',
         f'#include "{os.path.join(CS, "params.cuh")}"',
         "#include <atomic>",
+        "#include <cuda.h>",
         "namespace mimo {", errs, rope, "inline float ex2_approx(float x) { return exp2f(x); }", "}",
         _kernel("attn_bwd_simple.cuh"), _kernel("neighbors.cuh"), _kernel("attn_decode.cuh"),
         "namespace mimo {", tc_stub, "namespace {", f"constexpr int kSms = {SMS};", "bool g_launch_ok = true;",

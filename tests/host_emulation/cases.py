@@ -172,8 +172,8 @@ def route(H, E, k, T, normalize=True, ties=False, seed=53):
 
 
 def decode(H, kv, ql, hq, hkv, layer, window, base, has_sink, seed, choice=DECODE_AUTO, expect=0):
-    """The KV-cache path through mimo_attn_decode; AUTO sends more than 128 query rows per KV head to
-    the CUDA-core kernel in 128-row tiles (the tensor-core kernel is a stub here that flags an error)."""
+    """The KV-cache path through mimo_attn_decode on the CUDA-core kernel (the tensor-core kernel is a
+    stub here that flags an error if launched)."""
     x = W.make_decode_inputs(kv, ql, hq, hkv, has_sink, seed)
     Tq = int(sum(ql))
     d = DecodeDims(len(kv), Tq, int(sum(kv)), x.k_cache.shape[0], max(ql), max(kv), hq, hkv, 192, 128)
@@ -209,10 +209,13 @@ CASES = {
     "route": lambda H: (route(H, 256, 8, 200), route(H, 64, 8, 33), route(H, 32, 1, 7),
                         route(H, 256, 8, 64, normalize=False), route(H, 96, 32, 40, ties=True)),
     # 40 new tokens x 4 heads = 160 rows (two tiles) beside one-tile sequences; keys clipped per tile
-    "decode_tiles_swa": lambda H: decode(H, [300, 90, 20], [40, 20, 20], 8, 2, LAYER_SWA, 128, 1e4, True, 61),
+    "decode_tiles_swa": lambda H: decode(H, [300, 90, 20], [40, 20, 20], 8, 2, LAYER_SWA, 128, 1e4, True, 61,
+                                         choice=DECODE_CUDA_CORES),
     # a 300-token chunk (ten tiles) after a 300-token prefix: later tiles start several splits in
-    "decode_tiles_swa_long": lambda H: decode(H, [600, 64], [300, 64], 8, 2, LAYER_SWA, 128, 1e4, True, 65),
-    # three and seven tiles, the second sequence a whole prompt as one chunk
+    "decode_tiles_swa_long": lambda H: decode(H, [600, 64], [300, 64], 8, 2, LAYER_SWA, 128, 1e4, True, 65,
+                                              choice=DECODE_CUDA_CORES),
+    # three and seven tiles, the second sequence a whole prompt as one chunk; the automatic choice,
+    # which takes the CUDA-core kernel above 128 rows per KV head
     "decode_tiles_global": lambda H: decode(H, [200, 50], [36, 50], 8, 1, LAYER_GLOBAL, -1, 1e7, False, 62),
     # the CUDA-core kernel forced on one-tile sequences (decode and speculative chunks)
     "decode_one_tile": lambda H: decode(H, [5, 129, 300], [1, 8, 3], 8, 2, LAYER_SWA, 128, 1e4, True, 63,
