@@ -107,36 +107,6 @@ def test_bad_index_and_lengths_reported():
     assert mimo_attn.check() == mimo_attn.OK
 
 
-def test_rows_per_kv_head_above_128(dkernel):
-    """9 and 12 new tokens x 16 heads = 144 and 192 rows per KV head: two row tiles on the CUDA-core
-    kernel; the tensor-core kernel holds one 128-row tile and refuses."""
-    from global_attention_moe_b200 import mimo_attn
-    x = W.make_decode_inputs([40, 300], [9, 12], 64, 4, False, seed=37)
-    if dkernel == "tensor":
-        with pytest.raises(mimo_attn.MimoAttnError) as e:
-            decode_gpu(x, W.LAYER_GLOBAL, -1, 1e7)
-        assert e.value.status == mimo_attn.ERR_UNSUPPORTED
-    else:
-        parity(x, W.LAYER_GLOBAL, -1, 1e7)
-
-
-@pytest.mark.parametrize("kind", ["swa", "global"])
-def test_chunked_prefill(kind, dkernel):
-    """Chunks of new tokens far above 128 rows per KV head against a cached prefix, and a whole short
-    prompt as one chunk: row tiles, each tile's keys clipped to its rows' positions, and the splits
-    merged per tile.  The automatic choice runs them (on the CUDA-core kernel)."""
-    from global_attention_moe_b200 import mimo_attn
-    if dkernel == "tensor":
-        pytest.skip("the tensor-core kernel holds one 128-row tile")
-    mimo_attn.set_decode_kernel(mimo_attn.DECODE_AUTO)
-    kv = [1200, 700, 300, 129]
-    ql = [300, 200, 300, 64]
-    if kind == "swa":
-        parity(W.make_decode_inputs(kv, ql, 64, 8, True, seed=38), W.LAYER_SWA, 128, 1e4)
-    else:
-        parity(W.make_decode_inputs(kv, ql, 64, 4, False, seed=39), W.LAYER_GLOBAL, -1, 1e7)
-
-
 def test_chunk_and_ring_boundaries():
     """Contexts at and around the 64-key step of the tensor-core kernel, and long enough per CTA
     (24 requests x 4 KV heads: few splits) that its 4-stage ring wraps several times."""

@@ -4,8 +4,8 @@ its own caching allocator, a serving loop that forbids allocation on its hot
 path).  Its results must match the default entry point's, call after call,
 while it keeps its scratch in a fixed array inside the library.
 
-This file is collected last on purpose: if it fails, a run that stops at the
-first failure has already run every other test.
+It is collected after the forward and KV-cache suites (tests/conftest.py
+orders the GPU modules by when they were established).
 """
 import numpy as np
 import pytest
