@@ -171,10 +171,13 @@ def route(H, E, k, T, normalize=True, ties=False, seed=53):
     assert np.max(np.abs(w - rw)) <= 1e-6 * max(1.0, np.max(np.abs(rw)))
 
 
-def decode(H, kv, ql, hq, hkv, layer, window, base, has_sink, seed, choice=DECODE_AUTO, expect=0):
+def decode(H, kv, ql, hq, hkv, layer, window, base, has_sink, seed, choice=DECODE_AUTO, expect=0, bad_index=False):
     """The KV-cache path through mimo_attn_decode on the CUDA-core kernel (the tensor-core kernel is a
     stub here that flags an error if launched)."""
     x = W.make_decode_inputs(kv, ql, hq, hkv, has_sink, seed)
+    if bad_index:  # cache rows past the end of the cache, and a negative one
+        x.kv_indices = x.kv_indices.copy()
+        x.kv_indices[[3, len(x.kv_indices) - 1]] = [x.k_cache.shape[0] + 1000, -7]
     Tq = int(sum(ql))
     d = DecodeDims(len(kv), Tq, int(sum(kv)), x.k_cache.shape[0], max(ql), max(kv), hq, hkv, 192, 128)
     po, pl = H.empty((Tq, hq, 128), np.uint16), H.empty((hq, Tq), np.float32)
@@ -186,6 +189,10 @@ def decode(H, kv, ql, hq, hkv, layer, window, base, has_sink, seed, choice=DECOD
     if expect:
         H.done(0)
         assert st == expect, f"status {st}, expected {expect}"
+        return
+    if bad_index:  # reported for mimo_attn_check; the guard pages show no row outside the cache was read
+        assert st == 0 and H.L.hemu_error_word() == 4, "bad index not reported as BAD_SEQLENS"
+        H.done(0)
         return
     out = synth.bf16_bits_to_f32(H.get(po, (Tq, hq, 128), np.uint16)).astype(np.float64)
     lse = H.get(pl, (hq, Tq), np.float32).astype(np.float64)
@@ -220,6 +227,9 @@ CASES = {
     # the CUDA-core kernel forced on one-tile sequences (decode and speculative chunks)
     "decode_one_tile": lambda H: decode(H, [5, 129, 300], [1, 8, 3], 8, 2, LAYER_SWA, 128, 1e4, True, 63,
                                         choice=DECODE_CUDA_CORES),
+    # cache indices outside the cache: reported, never dereferenced
+    "decode_bad_index": lambda H: decode(H, [50, 300], [2, 40], 8, 2, LAYER_SWA, 128, 1e4, True, 66,
+                                         choice=DECODE_CUDA_CORES, bad_index=True),
     # the tensor-core kernel holds one tile: forcing it above 128 rows is refused
     "decode_tensor_refuses_tiles": lambda H: decode(H, [300], [40], 8, 2, LAYER_SWA, 128, 1e4, True, 64,
                                                     choice=DECODE_TENSOR, expect=ERR_UNSUPPORTED),

@@ -6,9 +6,10 @@
 //     not count, as on the GPU); a barrier that can never complete is reported as a deadlock;
 //   - warp shuffles through an exchange array, with an error if a lane of the warp has exited;
 //   - atomics as plain read-modify-write (a single OS thread runs every fiber);
-//   - every buffer, and the block's dynamic shared memory, sits against a PROT_NONE guard page (at its
-//     end in mode 0, at its start in mode 1), so an out-of-range access faults on the host, and is
-//     filled with 0xFF bytes (NaN as FP32 or BF16), so a read of memory nobody wrote shows in the results.
+//   - every buffer, and the block's dynamic shared memory, sits between two 16 MB PROT_NONE guard
+//     regions, flush against the one at its end in mode 0 and the one at its start in mode 1, so an
+//     out-of-range access faults on the host; it starts filled with 0xFF bytes (NaN as FP32 or
+//     BF16), so a read of memory nobody wrote shows in the results.
 // Device math: __sincosf is taken as the host's sinf/cosf (the GPU's is an approximation with an
 // absolute error near 2^-21 on [-pi, pi]); exp2f, fmaf and the BF16/FP8 conversions are the host forms.
 // Test infrastructure only: nothing in the library includes or calls it.
@@ -48,6 +49,7 @@ namespace hemu {
 
 inline int g_mode = 0;  // 0: buffers end at a guard page; 1: buffers start right after one
 inline long g_page = sysconf(_SC_PAGESIZE);
+inline constexpr size_t kGuard = size_t(16) << 20;  // PROT_NONE address space on each side of a buffer
 
 struct Alloc {
   void* map;
@@ -58,12 +60,12 @@ inline std::vector<std::pair<void*, Alloc>> g_allocs;
 inline void* guarded_alloc(size_t nbytes) {
   const size_t n16 = (nbytes + 15) & ~size_t(15);
   const size_t body = (n16 + g_page - 1) / g_page * g_page;
-  const size_t total = body + 2 * g_page;
+  const size_t total = body + 2 * kGuard;
   uint8_t* m = static_cast<uint8_t*>(mmap(nullptr, total, PROT_READ | PROT_WRITE, MAP_PRIVATE | MAP_ANONYMOUS, -1, 0));
   if (m == MAP_FAILED) return nullptr;
-  mprotect(m, g_page, PROT_NONE);
-  mprotect(m + g_page + body, g_page, PROT_NONE);
-  uint8_t* p = g_mode == 0 ? m + g_page + body - n16 : m + g_page;
+  mprotect(m, kGuard, PROT_NONE);
+  mprotect(m + kGuard + body, kGuard, PROT_NONE);
+  uint8_t* p = g_mode == 0 ? m + kGuard + body - n16 : m + kGuard;
   std::memset(p, 0xFF, n16);  // NaN in every float / BF16 lane: a read of unwritten memory shows
   g_allocs.push_back({p, {m, total}});
   return p;
@@ -144,12 +146,12 @@ inline void set_smem(size_t bytes) {
   if (g_smem_map) munmap(g_smem_map, g_smem_map_bytes);
   const size_t n16 = (bytes + 15) & ~size_t(15);
   const size_t body = (n16 + g_page - 1) / g_page * g_page + g_page;
-  g_smem_map_bytes = body + 2 * g_page;
+  g_smem_map_bytes = body + 2 * kGuard;
   g_smem_map = static_cast<uint8_t*>(
       mmap(nullptr, g_smem_map_bytes, PROT_READ | PROT_WRITE, MAP_PRIVATE | MAP_ANONYMOUS, -1, 0));
-  mprotect(g_smem_map, g_page, PROT_NONE);
-  mprotect(g_smem_map + g_page + body, g_page, PROT_NONE);
-  g_smem = g_mode == 0 ? g_smem_map + g_page + body - n16 : g_smem_map + g_page;
+  mprotect(g_smem_map, kGuard, PROT_NONE);
+  mprotect(g_smem_map + kGuard + body, kGuard, PROT_NONE);
+  g_smem = g_mode == 0 ? g_smem_map + kGuard + body - n16 : g_smem_map + kGuard;
 }
 
 // Runs fn (the kernel call) for every thread of every block.  Returns false on a barrier deadlock or a

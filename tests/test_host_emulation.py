@@ -50,6 +50,8 @@ PLANTED = [
      "decode_tiles_swa"),
     ("decode combine reads splits before the tile's keys", "const int s_lo = (lo_t - lo) / P.split_keys,",
      "const int s_lo = 0,", "decode_tiles_swa_long"),
+    ("decode dereferences a cache index outside the cache",
+     "bad_index = true;\n        row = 0;", "bad_index = true;", "decode_bad_index"),
 ]
 
 
