@@ -12,6 +12,10 @@ section):
   head order); Megatron-Bridge API doc "mimo_v2_flash_bridge",
   ``_dequant_fp8_blockwise`` (out = fp8 value times scale_inv) and
   ``MiMoV2FlashQKVMapping`` (192-dim Q/K, 128-dim V).
+* Output projection (linear_proj): miles PR #3648 "add MiMo-V2.6-Flash-RL
+  support", commit message on MiMoV2SelfAttention (the layer's linear_qkv and
+  linear_proj are built for the 128-dim V heads: linear_proj takes the
+  Hq x 128 attention output of a token).
 * MoE router: miles docs section 1 (256 routed experts, top-8 sigmoid routing
   with a fixed score-correction bias); miles PR #3648 review (no group-limited
   routing in this checkpoint); SGLang cookbook "MiMo-V2.6", section 2
@@ -27,6 +31,9 @@ Readings where the pages are silent (each listed in the design notes):
 * kv-head-interleaved layout: along the fused output dimension, KV group g
   holds its Hq/Hkv query heads (192 each), then its K head (192), then its V
   head (128), groups in order.
+* linear_proj: y = x W^T with W stored as a Linear weight [out, in], no bias
+  (the pages name no bias anywhere in the layer); the output width (the
+  model's hidden size) is not on the pages, a parameter here.
 * Router: scores are sigmoid(logit); the correction bias enters the choice of
   experts only (top-8 of score + bias); the weights are the chosen experts'
   scores, normalised to sum to one (``normalize``) -- both parts of this
@@ -123,3 +130,24 @@ def route(logits: np.ndarray, bias: np.ndarray, top_k: int = 8, normalize: bool 
         sel = s64[t, order]
         w[t] = sel / sel.sum() if normalize else sel
     return ids, w, key
+
+
+# ---------------------------------------------------------------- output projection
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """BF16 bit patterns (uint16) to their exact FP64 values (the top half of an FP32)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def linear_proj(x: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """The attention's output projection y = x W^T, exactly in FP64.
+
+    x: BF16 bits [T, K], the attention output of each token with its Hq heads of 128 dims side by
+    side (K = Hq x 128); w: BF16 bits [N, K], a Linear weight (out_features x in_features).
+    Returns FP64 [T, N]; no bias."""
+    xf = bf16_bits_to_f64(x)
+    wf = bf16_bits_to_f64(w)
+    assert xf.ndim == 2 and wf.ndim == 2 and xf.shape[1] == wf.shape[1]
+    return xf @ wf.T

@@ -1,10 +1,10 @@
 """Pins for the oracle of the steps beside the attention kernel (FP8 blockwise
-dequant, fused-QKV split, MoE router), against what the pages and mathematics
+dequant, fused-QKV split, output projection, MoE router), against what the pages and mathematics
 fix: a library decoder of the FP8 format, closed forms, an independent
 construction of the fused layout, brute force over expert subsets, invariants.
 
 Each ``pin_*`` takes a handle ``N`` with ``e4m3_to_f64``,
-``dequant_fp8_blockwise``, ``split_qkv`` and ``route``, and raises
+``dequant_fp8_blockwise``, ``split_qkv``, ``linear_proj`` and ``route``, and raises
 AssertionError on a disagreement.  The same pins run against the real module
 and against deliberately broken copies of it.
 """
@@ -167,6 +167,54 @@ def pin_route_invariants(N):
     assert ids[0].tolist() == list(range(K))
 
 
+# ---------------------------------------------------------------- output projection
+
+
+def _bf16_exact(v):
+    """BF16 bits of FP32 values that are exactly representable (at most 8 significant bits)."""
+    f = np.asarray(v, dtype=np.float32)
+    bits = (f.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    assert np.array_equal((bits.astype(np.uint32) << np.uint32(16)).view(np.float32), f)
+    return bits
+
+
+def pin_linear_proj_brute_force(N):
+    """Against a pure-Python sum over the input features (math.fsum, exactly rounded), with the BF16
+    values decoded bit by bit, on a tiny ragged shape."""
+    rng = np.random.default_rng(21)
+    T, Kf, Nf = 3, 24, 5
+    # full 8-bit BF16 significands over a spread of exponents: the sums need far more than 24 bits
+    x = (rng.standard_normal((T, Kf)).astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    w = (rng.standard_normal((Nf, Kf)).astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+    def dec(b):
+        sign = -1.0 if b >> 15 else 1.0
+        e, m = (b >> 7) & 0xFF, b & 0x7F
+        return sign * (m / 128.0) * 2.0 ** -126 if e == 0 else sign * (1 + m / 128.0) * 2.0 ** (e - 127)
+
+    y = N.linear_proj(x, w)
+    assert y.shape == (T, Nf)
+    for t in range(T):
+        for n in range(Nf):
+            want = math.fsum(dec(int(x[t, k])) * dec(int(w[n, k])) for k in range(Kf))
+            assert abs(y[t, n] - want) <= 1e-12 * max(1.0, abs(want)), (t, n)
+
+
+def pin_linear_proj_selector_weights(N):
+    """A weight with a single 1 per output row picks that input feature: output n equals input
+    feature perm[n] exactly (catches a transposed or shifted operand)."""
+    rng = np.random.default_rng(22)
+    T, Kf, Nf = 4, DV * 2, 7
+    x = _bf16_exact(np.round(rng.standard_normal((T, Kf)) * 8) / 8)
+    perm = rng.permutation(Kf)[:Nf]
+    wf = np.zeros((Nf, Kf), np.float32)
+    wf[np.arange(Nf), perm] = 1.0
+    y = N.linear_proj(x, _bf16_exact(wf))
+    xv = (x.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    assert np.array_equal(y, xv[:, perm])
+
+
 ALL_PINS = [pin_e4m3_all_codes_match_torch, pin_e4m3_closed_forms, pin_dequant_blocks_by_kron,
             pin_dequant_identity_scale, pin_split_inverts_the_fused_layout, pin_route_zero_bias_is_logit_topk,
-            pin_route_brute_force_subsets, pin_route_weights_closed_form, pin_route_invariants]
+            pin_route_brute_force_subsets, pin_route_weights_closed_form, pin_route_invariants,
+            pin_linear_proj_brute_force, pin_linear_proj_selector_weights]

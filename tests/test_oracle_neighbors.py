@@ -33,6 +33,11 @@ MUTATIONS = [
     ("route_no_normalise", "w[t] = sel / sel.sum() if normalize else sel", "w[t] = sel"),
     ("route_softmax_scores", "s64 = sigmoid_f64(logits)", "s64 = np.exp(logits.astype(np.float64)) / np.exp(logits.astype(np.float64)).sum(1, keepdims=True)"),
     ("route_ties_to_higher_index", "key=lambda e: (-float(key[t, e]), e)", "key=lambda e: (-float(key[t, e]), -e)"),
+    ("proj_weight_not_transposed", "return xf @ wf.T", "return xf @ wf.reshape(wf.shape[1], wf.shape[0])"),
+    ("proj_drops_last_feature", "return xf @ wf.T", "return xf[:, :-1] @ wf[:, :-1].T"),
+    ("proj_rounds_to_fp32", "return xf @ wf.T", "return (xf @ wf.T).astype(np.float32).astype(np.float64)"),
+    ("proj_bf16_decoded_as_fp16", "b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)\n    return b.view(np.float32).astype(np.float64)",
+     "return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)"),
 ]
 
 
