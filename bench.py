@@ -62,8 +62,9 @@ def parse():
                     help="time the KV-cache path (64 requests x 8 new tokens) instead of the forward")
     ap.add_argument("--decode-requests", type=int, default=64,
                     help="requests in the KV-cache batch (fewer: a smaller case for profiling)")
-    ap.add_argument("--step", choices=("bwd", "dequant", "split", "route"), default=None,
-                    help="time a step beside the forward instead (backward, FP8 dequant, QKV split, MoE routing)")
+    ap.add_argument("--step", choices=("bwd", "dequant", "split", "proj", "route"), default=None,
+                    help="time a step beside the forward instead (backward, FP8 dequant, QKV split, output "
+                         "projection, MoE routing)")
     ap.add_argument("--decode-contiguous", action="store_true",
                     help="each request's cache rows in order instead of a random permutation")
     return ap.parse_args()
@@ -577,7 +578,7 @@ def run_decode(args):
     return 0
 
 
-STEP_KINDS = ("bwd", "dequant", "split", "route")
+STEP_KINDS = ("bwd", "dequant", "split", "proj", "route")
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core FP32 FMA peak at the maximum SM clock
 
 
@@ -625,6 +626,15 @@ def run_step(args):
         call = lambda: mimo_attn.qkv_split(fused, hq, hkv)
         flops, nbytes = 0, fused.numel() * 2 * 2
         units, unit, config, bound = T, "tokens/s", {"workload": f"qkv_split_T{T}_hq{hq}_hkv{hkv}"}, "hbm"
+    elif kind == "proj":
+        # the sliding layer's output projection: 64 heads x 128 dims -> hidden 4096 (synthetic), T = 4096
+        T, K_, N_ = 4096, 64 * 128, 4096
+        bf = lambda a: torch.from_numpy((a.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+                                        .view(np.int16)).cuda().view(torch.bfloat16)
+        xt, wt = bf(rng.standard_normal((T, K_))), bf(rng.standard_normal((N_, K_)) / np.sqrt(K_))
+        call = lambda: mimo_attn.linear_proj(xt, wt)
+        flops, nbytes = 2 * T * K_ * N_, 2 * (T * K_ + N_ * K_ + T * N_)
+        units, unit, config, bound = T, "tokens/s", {"workload": f"linear_proj_T{T}_in{K_}_out{N_}"}, "tensor"
     else:
         T, E = 262144, 256  # 268 MB of logits: larger than L2
         lg = torch.from_numpy((rng.standard_normal((T, E)) * 2).astype(np.float32)).cuda()
@@ -649,6 +659,8 @@ def run_step(args):
     assert mimo_attn.check() == mimo_attn.OK
     if bound == "hbm":
         ach, peak, runit = nbytes / (ms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    elif bound == "tensor":
+        ach, peak, runit = flops / (ms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
     else:
         ach, peak, runit = flops / (ms / 1e3) / 1e12, FP32_ALU_TFLOPS, "TFLOP/s"
         peak_src = "derived: 148 SMs x 128 FP32 lanes x 2 FLOP per FMA x 1965 MHz"
@@ -660,6 +672,8 @@ def run_step(args):
         "roofline": {"bound": bound, "achieved": ach, "peak": peak, "unit": runit, "frac": ach / peak, "traffic": None,
                      "peak_source": peak_src if bound == "alu" else f"{peak_src} (burst)", "algorithmic_bytes": nbytes, "algorithmic_flops": flops},
         "e2e": None, "clocks": clk.summary(),
+        # this library's kernels per step (the projection's GEMM runs in cuBLAS)
+        "gpu_launches": steps * {"bwd": 3, "dequant": 1, "split": 1, "route": 1, "proj": 0}[kind],
     }
     print(json.dumps(line), flush=True)
     return 0

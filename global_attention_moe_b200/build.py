@@ -40,7 +40,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden",
            "-Xcompiler", "-O2", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include"),
-           "-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES] + ["-lrt"]
+           "-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES] + ["-lrt", "-ldl"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)

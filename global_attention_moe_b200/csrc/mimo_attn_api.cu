@@ -1,9 +1,11 @@
 // mimo_attn_api.cu -- host side of the C ABI declared in include/mimo_attn.h:
 // argument validation (before any CUDA call), TMA tensor-map encoding, kernel
 // launch, the device error word and the host-buffer end-to-end entry point.
+#include <cublas_v2.h>  // types only: cuBLAS itself is loaded at the first output projection
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <dlfcn.h>
 
 #include <algorithm>
 #include <atomic>
@@ -219,6 +221,48 @@ DeviceInfo* device_info(int dev) {
     }
   }
   return &d;
+}
+
+// cuBLAS for the output projection (a plain BF16 GEMM), loaded with dlopen at its first call so that
+// nothing else in the library depends on it; one handle per device, used under the lock.
+struct CublasApi {
+  bool tried = false, ok = false;
+  decltype(&cublasCreate_v2) create = nullptr;
+  decltype(&cublasSetStream_v2) set_stream = nullptr;
+  // the C symbol (the header adds a C++ overload taking the compute type as a cudaDataType)
+  cublasStatus_t (*gemm_ex)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int, const void*,
+                            const void*, cudaDataType, int, const void*, cudaDataType, int, const void*, void*,
+                            cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t) = nullptr;
+  cublasHandle_t handles[64] = {};
+};
+
+// y[T, N] = x[T, K] . w[N, K]^T, BF16 in and out, FP32 accumulation (row-major operands; in cuBLAS's
+// column-major terms y^T = w . x^T with w read transposed).
+int gemm_bf16_nt(const void* x, const void* w, int T, int K, int N, void* y, cudaStream_t stream) {
+  static CublasApi a;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MIMO_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!a.tried) {
+    a.tried = true;
+    if (void* lib = dlopen("libcublas.so.12", RTLD_NOW | RTLD_LOCAL)) {
+      a.create = reinterpret_cast<decltype(a.create)>(dlsym(lib, "cublasCreate_v2"));
+      a.set_stream = reinterpret_cast<decltype(a.set_stream)>(dlsym(lib, "cublasSetStream_v2"));
+      a.gemm_ex = reinterpret_cast<decltype(a.gemm_ex)>(dlsym(lib, "cublasGemmEx"));
+      a.ok = a.create && a.set_stream && a.gemm_ex;
+    }
+  }
+  if (!a.ok) return MIMO_ERR_CUDA;
+  if (!a.handles[dev] && a.create(&a.handles[dev]) != CUBLAS_STATUS_SUCCESS) {
+    a.handles[dev] = nullptr;
+    return MIMO_ERR_CUDA;
+  }
+  if (a.set_stream(a.handles[dev], stream) != CUBLAS_STATUS_SUCCESS) return MIMO_ERR_CUDA;
+  const float alpha = 1.f, beta = 0.f;
+  const cublasStatus_t st = a.gemm_ex(a.handles[dev], CUBLAS_OP_T, CUBLAS_OP_N, N, T, K, &alpha, w, CUDA_R_16BF, K, x,
+                                      CUDA_R_16BF, K, &beta, y, CUDA_R_16BF, N, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+  return st == CUBLAS_STATUS_SUCCESS ? MIMO_OK : MIMO_ERR_CUDA;
 }
 
 int launch(const void* q, const void* k, const void* v, const FwdParams& P, cudaStream_t stream) {
@@ -761,6 +805,16 @@ int mimo_qkv_split(const void* fused, int64_t tokens, int num_q_heads, int num_k
       static_cast<const uint16_t*>(fused), static_cast<uint16_t*>(q), static_cast<uint16_t*>(k),
       static_cast<uint16_t*>(v), tokens, num_q_heads, num_kv_heads);
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
+int mimo_linear_proj(const void* x, const void* w, int64_t tokens, int64_t in_features, int64_t out_features,
+                     void* y, void* stream) {
+  if (tokens < 0 || in_features < 1 || out_features < 1) return MIMO_ERR_INVALID_ARG;
+  if (in_features % 8 != 0 || out_features % 8 != 0) return MIMO_ERR_UNSUPPORTED;  // 16-byte rows
+  if (tokens > INT32_MAX || in_features > INT32_MAX || out_features > INT32_MAX) return MIMO_ERR_UNSUPPORTED;
+  if (tokens == 0) return MIMO_OK;
+  if (!x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y)) return MIMO_ERR_INVALID_ARG;
+  return gemm_bf16_nt(x, w, (int)tokens, (int)in_features, (int)out_features, y, static_cast<cudaStream_t>(stream));
 }
 
 int mimo_moe_route(const float* logits, const float* bias, int64_t tokens, int num_experts, int top_k, int normalize,

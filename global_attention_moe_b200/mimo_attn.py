@@ -22,7 +22,8 @@ SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host
            "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_fwd_noalloc",
            "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_profile_start",
            "mimo_attn_profile_stop", "mimo_attn_decode", "mimo_attn_set_decode_kernel", "mimo_attn_version",
-           "mimo_attn_bwd", "mimo_fp8_dequant_blockwise", "mimo_qkv_split", "mimo_moe_route")
+           "mimo_attn_bwd", "mimo_fp8_dequant_blockwise", "mimo_qkv_split", "mimo_moe_route",
+           "mimo_linear_proj")
 KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED, KERNEL_WINDOW = 0, 1, 2, 3
 DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR = 0, 1, 2
 
@@ -83,6 +84,8 @@ def _load():
     lib.mimo_fp8_dequant_blockwise.argtypes = [P, P, L, L, I, I, P, P]
     lib.mimo_qkv_split.restype = I
     lib.mimo_qkv_split.argtypes = [P, L, I, I, P, P, P, P]
+    lib.mimo_linear_proj.restype = I
+    lib.mimo_linear_proj.argtypes = [P, P, L, L, L, P, P]
     lib.mimo_moe_route.restype = I
     lib.mimo_moe_route.argtypes = [P, P, L, I, I, I, P, P, P]
     lib.mimo_attn_set_decode_kernel.restype = I
@@ -166,6 +169,23 @@ def qkv_split(fused, num_q_heads, num_kv_heads, stream=None):
     if st != OK:
         raise MimoAttnError(st, "mimo_qkv_split")
     return q, k, v
+
+
+def linear_proj(x, w, out=None, stream=None):
+    """Output projection y = x . w^T: bf16 x [T, K] or the attention output [T, Hq, 128] (CUDA), bf16 w
+    [N, K] (a Linear weight) -> bf16 y [T, N] (cuBLAS, FP32 accumulation)."""
+    import torch
+    T = x.shape[0]
+    x2 = x.reshape(T, -1)
+    N, K = w.shape
+    if x2.shape[1] != K:
+        raise ValueError(f"x has {x2.shape[1]} features per token, w expects {K}")
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    st = LIB.mimo_linear_proj(x2.data_ptr(), w.data_ptr(), T, K, N, out.data_ptr(), _stream_handle(stream))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_linear_proj")
+    return out
 
 
 def moe_route(logits, bias, top_k=8, normalize=True, stream=None):

@@ -329,6 +329,21 @@ MIMO_API int mimo_qkv_split(const void* fused, int64_t tokens, int num_q_heads, 
                             void* k, void* v, void* stream);
 
 /*
+ * Output projection linear_proj of the attention (miles PR #3648, commit
+ * message on MiMoV2SelfAttention: the projection is built for the 128-dim V
+ * heads): y = x . w^T with x bf16 [tokens, in_features] (the attention output
+ * [T, Hq, 128] viewed as [T, Hq * 128]), w bf16 [out_features, in_features]
+ * (a Linear weight, no bias), y bf16 [tokens, out_features]; FP32
+ * accumulation, one rounding of each output to BF16.  A plain GEMM: it runs
+ * on cuBLAS, loaded at the first call (MIMO_ERR_CUDA if it cannot be loaded).
+ * Features must be multiples of 8 and at most 2^31 - 1 (else
+ * MIMO_ERR_UNSUPPORTED).  Device pointers, 16-byte aligned.  Does not
+ * synchronise.
+ */
+MIMO_API int mimo_linear_proj(const void* x, const void* w, int64_t tokens, int64_t in_features,
+                              int64_t out_features, void* y, void* stream);
+
+/*
  * MoE routing (miles docs section 1: 256 routed experts, top-8 sigmoid routing
  * with a fixed score-correction bias; router logits in FP32 per the SGLang
  * cookbook section 2).  logits fp32 [T, E], bias fp32 [E] (E a multiple of 32,

@@ -154,3 +154,20 @@ def test_decode_validation_rejects(M, case, expect):
     st = M.decode_raw(args["q"], FAKE, FAKE, FAKE, FAKE, FAKE, args["sink"], dims, args["layer"], args["window"],
                       1e4, args["rope_dims"], 0.707, FAKE, FAKE, None)
     assert st == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    (dict(tokens=-1), 1),                      # negative token count
+    (dict(k=0), 1),                            # no input features
+    (dict(n=-8), 1),
+    (dict(k=12), 2),                           # rows not a multiple of 16 bytes
+    (dict(n=20), 2),
+    (dict(k=1 << 31), 2),                      # beyond the GEMM's 32-bit sizes
+    (dict(x=FAKE + 8), 1),                     # misaligned
+    (dict(y=None), 1),                         # missing output
+    (dict(tokens=0, x=None, w=None, y=None), 0),  # nothing to do: no pointer is needed
+])
+def test_linear_proj_validation(M, args, expect):
+    a = dict(x=FAKE, w=FAKE, tokens=4, k=1024, n=512, y=FAKE)
+    a.update(args)
+    assert M.LIB.mimo_linear_proj(a["x"], a["w"], a["tokens"], a["k"], a["n"], a["y"], None) == expect

@@ -1,6 +1,7 @@
-"""GPU parity of the steps beside the attention kernel (FP8 blockwise dequant, fused-QKV split, MoE
-router) against the numpy oracle: bit-exact for the dequant and the split; the router's choice equal
-where the FP32 keys are not tied, weights to FP32 rounding."""
+"""GPU parity of the steps beside the attention kernel (FP8 blockwise dequant, fused-QKV split, output
+projection, MoE router) against the numpy oracle: bit-exact for the dequant and the split; the
+projection within the BF16 rounding of its outputs; the router's choice equal where the FP32 keys
+are not tied, weights to FP32 rounding."""
 import numpy as np
 import pytest
 import torch
@@ -69,3 +70,26 @@ def test_route(E, k, T):
     assert same.mean() > 0.999
     assert np.max(np.abs(w[same] - rw[same])) <= 1e-6
     assert np.allclose(w.sum(1), 1.0, atol=1e-6)
+
+
+@pytest.mark.parametrize("T,hq,N", [(300, 8, 512), (1, 64, 4096), (130, 64, 264)])
+def test_linear_proj(T, hq, N):
+    """y = x . W^T (cuBLAS, FP32 accumulation, one BF16 rounding per output) against the FP64 oracle.
+    Tolerance from the arithmetic: the BF16 rounding of each output is at most 2^-9 relative (RMS
+    about 2^-9 / sqrt(3) = 1.1e-3 over many outputs); FP32 accumulation over K <= 8192 terms adds
+    about sqrt(K) 2^-24 = 5e-6.  So rel-L2 <= 2e-3, and each output within 2^-8 |y| plus 1e-3 of
+    the outputs' RMS."""
+    from global_attention_moe_b200 import mimo_attn as M
+    rng = np.random.default_rng(54)
+    K = hq * 128
+    bf16 = lambda a: (a.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    x = bf16(rng.standard_normal((T, hq, 128)))
+    w = bf16(rng.standard_normal((N, K)) / np.sqrt(K))
+    dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    y = M.linear_proj(dev(x), dev(w))
+    assert M.check() == M.OK
+    assert tuple(y.shape) == (T, N)
+    got = NB.bf16_bits_to_f64(y.view(torch.int16).cpu().numpy().view(np.uint16))
+    ref = NB.linear_proj(x.reshape(T, K), w)
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 2e-3
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-3 * np.sqrt(np.mean(ref ** 2)))
