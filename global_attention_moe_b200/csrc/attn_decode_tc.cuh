@@ -88,8 +88,9 @@ static_assert(kStageBytes % 1024 == 0 && kStageOff % 1024 == 0 && kVOff % 1024 =
 struct Work {
   int q_beg, rows, p0;       // first query row, q_len * group, position of query 0
   int kv_beg, k_beg, k_end;  // index-list offset, key range [k_beg, k_end) of this split
-  int n;                     // chunks (0: the split lies past the sequence's keys)
+  int n;                     // chunks (0: no key of the split is visible to the tile's rows)
   int g, split;              // KV head, split
+  int row0;                  // first query row of the tile (rows row0 .. row0 + rows - 1 of the sequence's)
 };
 
 struct Ctrl {
@@ -109,26 +110,36 @@ static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
 // inconsistent (reported; the combine kernel skips the same rows).  The checks
 // are those of the CUDA-core kernel.
 __device__ __forceinline__ bool make_work(const dec::DecParams& P, long long u, Work& w) {
-  const long long per_split = static_cast<long long>(P.hkv) * P.num_seqs;
+  const long long per_tile = static_cast<long long>(P.hkv) * P.num_seqs;
+  const long long per_split = per_tile * P.qtiles;
   w.split = static_cast<int>(u / per_split);
-  const long long r = u % per_split;
+  const long long rt = u % per_split;
+  const int qt = static_cast<int>(rt / per_tile);
+  const long long r = rt % per_tile;
   w.g = static_cast<int>(r % P.hkv);
   const int b = static_cast<int>(r / P.hkv);
   w.q_beg = __ldg(P.cu_q + b);
   const int q_len = __ldg(P.cu_q + b + 1) - w.q_beg;
   w.kv_beg = __ldg(P.kv_indptr + b);
   const int kv_len = __ldg(P.kv_indptr + b + 1) - w.kv_beg;
-  w.rows = q_len * P.group;
+  const int all_rows = q_len * P.group;
   const int lo = dec::key_lo(kv_len, q_len, P.window);
-  if (q_len < 0 || kv_len < 0 || q_len > kv_len || w.rows > 128 || w.q_beg < 0 || w.q_beg + q_len > P.total_q ||
-      w.kv_beg < 0 || w.kv_beg + kv_len > P.total_kv || kv_len - lo > P.splits * P.split_keys) {
-    if (w.split == 0 && w.g == 0) atomicOr(&g_mimo_error, kErrSeqlens);
+  if (q_len < 0 || kv_len < 0 || q_len > kv_len || all_rows > 128 * P.qtiles || w.q_beg < 0 ||
+      w.q_beg + q_len > P.total_q || w.kv_beg < 0 || w.kv_beg + kv_len > P.total_kv ||
+      kv_len - lo > P.splits * P.split_keys) {
+    if (w.split == 0 && w.g == 0 && qt == 0) atomicOr(&g_mimo_error, kErrSeqlens);
     return false;
   }
-  if (w.rows == 0) return false;
+  w.row0 = 128 * qt;
+  w.rows = min(128, all_rows - w.row0);
+  if (w.rows <= 0) return false;
   w.p0 = kv_len - q_len;
-  w.k_beg = lo + w.split * P.split_keys;
-  w.k_end = min(kv_len, w.k_beg + P.split_keys);
+  // the split's keys, clipped to those the tile's rows may see
+  const int pos_first = w.p0 + w.row0 / P.group, pos_last = w.p0 + (w.row0 + w.rows - 1) / P.group;
+  const int lo_t = P.window >= 0 ? max(0, pos_first - P.window) : 0;
+  const int s_beg = lo + w.split * P.split_keys;
+  w.k_beg = max(s_beg, lo_t);
+  w.k_end = min(min(kv_len, s_beg + P.split_keys), pos_last + 1);
   w.n = w.k_end > w.k_beg ? (w.k_end - w.k_beg + kChunk - 1) / kChunk : 0;
   return true;
 }
@@ -171,7 +182,7 @@ constexpr uint32_t kItemReaders = 128 + 128 + 1 + 128;  // softmax, fetcher, MMA
 // inconsistent sequences), and publishes the rest; ends with an n < 0 entry.
 __device__ __forceinline__ void role_producer(Ctrl* C, const dec::DecParams& P) {
   const uint64_t lim = P.wait_limit_ns;
-  const long long total = static_cast<long long>(P.splits) * P.hkv * P.num_seqs;
+  const long long total = static_cast<long long>(P.splits) * P.qtiles * P.hkv * P.num_seqs;
 #pragma unroll 1
   for (uint32_t k = 0;; ++k) {
     const int slot = static_cast<int>(k % kRing);
@@ -286,7 +297,7 @@ __device__ __forceinline__ void role_lander(uint8_t* smem, Ctrl* C, const dec::D
     for (int pass = 0; pass < 8; ++pass) {  // zeros past q_len x group
       const int r = 16 * pass + rsub;
       const bool in = r < w.rows;
-      const int i = in ? r / group : 0, hh = in ? r % group : 0;
+      const int i = in ? (w.row0 + r) / group : 0, hh = in ? (w.row0 + r) % group : 0;
       const uint16_t* src =
           in ? P.q + (static_cast<size_t>(w.q_beg + i) * P.hq + w.g * group + hh) * kHeadDimQK : P.q;
       const uint32_t sw = static_cast<uint32_t>(r * 128 + ((l8 ^ (r & 7)) << 4));
@@ -297,7 +308,7 @@ __device__ __forceinline__ void role_lander(uint8_t* smem, Ctrl* C, const dec::D
     cp_async_commit();
     cp_async_wait<0>();
     named_bar_sync(kQBar, 128);
-    const int pos = qt < w.rows ? w.p0 + qt / group : 0;  // one row per thread
+    const int pos = qt < w.rows ? w.p0 + (w.row0 + qt) / group : 0;  // one row per thread
 #pragma unroll
     for (int c = 0; c < 4; ++c) amax = fmaxf(amax, rope_rotate_chunk_pair(smem + kQOff, qt, c, pos, C->theta));
     fence_proxy_async_smem();
@@ -376,7 +387,7 @@ __device__ __forceinline__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, 
 
 // Writes an item's partial for row r: (m, l) and the unnormalised O row.
 __device__ __forceinline__ float4* partial_row(const dec::DecParams& P, const Work& w, int r, size_t& slot) {
-  const int i = r / P.group, hh = r % P.group;
+  const int i = (w.row0 + r) / P.group, hh = (w.row0 + r) % P.group;
   slot = (static_cast<size_t>(w.q_beg + i) * P.hq + w.g * P.group + hh) * P.splits + w.split;
   return reinterpret_cast<float4*>(P.part_o + slot * kHeadDimV);
 }
@@ -395,7 +406,7 @@ __device__ __forceinline__ void role_softmax(Ctrl* C, uint32_t tmem, const dec::
     const bool have = items.next(C, w, failed, lim);
     if (!__all_sync(0xffffffffu, !failed) || !have) break;
     const bool valid = r < w.rows;
-    const int pos = valid ? w.p0 + r / P.group : -1;  // rows past the queries see no key
+    const int pos = valid ? w.p0 + (w.row0 + r) / P.group : -1;  // rows past the queries see no key
     const int last = min(w.k_end - 1, pos);           // last key this row may see
     const int first = P.window >= 0 ? pos - P.window : w.k_beg;
     float m = -INFINITY, l = 0.f;

@@ -477,19 +477,18 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
   P.v_scale = v_scale;
   P.wait_limit_ns = kDefaultWaitLimitNs;
   for (int i = 0; i < kRopeDims / 2; ++i) P.theta[i] = std::pow(rope_base, -2.0 * i / kRopeDims);
-  // Query rows per KV head above 128 (chunked prefill) run on the CUDA-core kernel in 128-row tiles;
-  // the tensor-core kernel holds one tile (its M = 128 accumulator).
+  // The query rows of a KV head are cut into 128-row tiles (one M = 128 accumulator of the tensor-core
+  // kernel): chunked prefill runs on either kernel with the tile as one more dimension of its work.
   const long long all_rows = (long long)d->max_q_len * P.group;
   const int choice = g_decode_choice.load();
-  if (choice == MIMO_DECODE_TENSOR && all_rows > dec::kMaxRows) return MIMO_ERR_UNSUPPORTED;
-  const bool tensor = choice == MIMO_DECODE_TENSOR || (choice == MIMO_DECODE_AUTO && all_rows <= dec::kMaxRows);
-  P.qtiles = tensor ? 1 : (int)std::max<long long>(1, (all_rows + dec::kMaxRows - 1) / dec::kMaxRows);
+  const bool tensor = choice != MIMO_DECODE_CUDA_CORES;
+  P.qtiles = (int)std::max<long long>(1, (all_rows + dec::kMaxRows - 1) / dec::kMaxRows);
   // Keys one sequence's queries can see, at most; split them so that the work covers the SMs a few
   // times over (tensor-core kernel: persistent, one CTA per SM walking about six (sequence, KV head,
   // split) items; CUDA-core kernel: one CTA per (split, row tile) item, about two per SM).
   const long long span = (P.window >= 0) ? std::min<long long>(d->max_kv_len, (long long)P.window + d->max_q_len)
                                          : (long long)d->max_kv_len;
-  const long long base_ctas = (long long)d->num_seqs * P.hkv * P.qtiles;
+  const long long base_ctas = (long long)d->num_seqs * P.hkv * P.qtiles;  // both kernels tile the rows
   const long long chunk = tensor ? dtc::kChunk : dec::kChunk;
   const long long target = (tensor ? 6LL : 2LL) * info->sms;
   long long splits = std::max<long long>(1, (target + base_ctas - 1) / base_ctas);
@@ -513,7 +512,7 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     st = MIMO_ERR_CUDA;
   if (st == MIMO_OK) {
     if (tensor) {  // persistent: at most one CTA per SM, items from the shared counter
-      const long long items = splits * P.hkv * (long long)d->num_seqs;
+      const long long items = splits * P.qtiles * P.hkv * (long long)d->num_seqs;
       attn_decode_tc_kernel<<<(unsigned)std::min<long long>(items, info->sms), dtc::kThreads, dtc::kSmemBytes,
                               stream>>>(P);
     } else {

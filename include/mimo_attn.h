@@ -249,8 +249,8 @@ MIMO_API int mimo_attn_profile_stop(int* launches, double* total_ms);
  * kv_len_b - q_len_b + i and attends the keys mimo_attn_fwd would give it, so
  * out and lse equal the forward's rows for those positions.  Chunked
  * prefill: the max_q_len * Hq/Hkv query rows of a KV head may exceed 128, up
- * to 2^20 (else MIMO_ERR_UNSUPPORTED); above 128 the CUDA-core kernel runs
- * them in 128-row tiles (see mimo_attn_set_decode_kernel); every q_len_b,
+ * to 2^20 (else MIMO_ERR_UNSUPPORTED); both kernels run them in 128-row
+ * tiles; every q_len_b,
  * kv_len_b must be at most max_q_len, max_kv_len.  Inconsistent cu_q /
  * kv_indptr, q_len_b > kv_len_b and cache rows outside [0, cache_rows) are
  * recorded as MIMO_ERR_BAD_SEQLENS for mimo_attn_check (such rows are left
@@ -270,16 +270,14 @@ MIMO_API int mimo_attn_decode(const void* q, const void* k_cache, const void* v_
 
 /*
  * Selects the kernel mimo_attn_decode launches (process-wide; default AUTO):
- *   MIMO_DECODE_AUTO        the tensor-core kernel while max_q_len * Hq/Hkv
- *                           <= 128, else the CUDA-core kernel
- *   MIMO_DECODE_CUDA_CORES  FP32 on the CUDA cores, 32 keys per step, the
- *                           query rows of a KV head in 128-row tiles (the
- *                           cross-check path, and chunked prefill)
- *   MIMO_DECODE_TENSOR      tcgen05: the query rows of one KV head as the
- *                           M = 128 operand, K/V gathered by index into
- *                           shared memory 64 keys per step, S and O in TMEM;
- *                           holds one tile: mimo_attn_decode returns
- *                           MIMO_ERR_UNSUPPORTED above 128 rows
+ *   MIMO_DECODE_AUTO        the tensor-core kernel
+ *   MIMO_DECODE_CUDA_CORES  FP32 on the CUDA cores, 32 keys per step (the
+ *                           cross-check path)
+ *   MIMO_DECODE_TENSOR      tcgen05: a 128-row tile of the query rows of one
+ *                           KV head as the M = 128 operand, K/V gathered by
+ *                           index into shared memory 64 keys per step, S and
+ *                           O in TMEM
+ * Both cut the query rows of a KV head into 128-row tiles (chunked prefill).
  * Both compute the same operation; they differ in rounding order (the
  * tensor-core kernel rounds P to BF16 and the rotated dims of Q and K to FP16,
  * as the forward does).  Returns MIMO_ERR_INVALID_ARG for any other value.

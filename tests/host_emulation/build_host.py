@@ -139,7 +139,7 @@ def build(out_dir: str, source: str | None = None) -> str:
     with open(src, "w") as f:
         f.write(source if source is not None else generate())
     so = os.path.join(out_dir, "libhost_kernels.so")
-    cmd = ["g++", "-std=c++20", "-O1", "-fPIC", "-shared", "-w", "-I/usr/local/cuda/include", "-I" + HERE, src,
+    cmd = ["g++", "-std=c++20", "-O1", "-fno-strict-aliasing", "-fPIC", "-shared", "-w", "-I/usr/local/cuda/include", "-I" + HERE, src,
            "-o", so]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode:

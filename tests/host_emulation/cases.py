@@ -221,18 +221,15 @@ CASES = {
     # a 300-token chunk (ten tiles) after a 300-token prefix: later tiles start several splits in
     "decode_tiles_swa_long": lambda H: decode(H, [600, 64], [300, 64], 8, 2, LAYER_SWA, 128, 1e4, True, 65,
                                               choice=DECODE_CUDA_CORES),
-    # three and seven tiles, the second sequence a whole prompt as one chunk; the automatic choice,
-    # which takes the CUDA-core kernel above 128 rows per KV head
-    "decode_tiles_global": lambda H: decode(H, [200, 50], [36, 50], 8, 1, LAYER_GLOBAL, -1, 1e7, False, 62),
+    # three and seven tiles, the second sequence a whole prompt as one chunk
+    "decode_tiles_global": lambda H: decode(H, [200, 50], [36, 50], 8, 1, LAYER_GLOBAL, -1, 1e7, False, 62,
+                                            choice=DECODE_CUDA_CORES),
     # the CUDA-core kernel forced on one-tile sequences (decode and speculative chunks)
     "decode_one_tile": lambda H: decode(H, [5, 129, 300], [1, 8, 3], 8, 2, LAYER_SWA, 128, 1e4, True, 63,
                                         choice=DECODE_CUDA_CORES),
     # cache indices outside the cache: reported, never dereferenced
     "decode_bad_index": lambda H: decode(H, [50, 300], [2, 40], 8, 2, LAYER_SWA, 128, 1e4, True, 66,
                                          choice=DECODE_CUDA_CORES, bad_index=True),
-    # the tensor-core kernel holds one tile: forcing it above 128 rows is refused
-    "decode_tensor_refuses_tiles": lambda H: decode(H, [300], [40], 8, 2, LAYER_SWA, 128, 1e4, True, 64,
-                                                    choice=DECODE_TENSOR, expect=ERR_UNSUPPORTED),
 }
 
 if __name__ == "__main__":

@@ -1,0 +1,379 @@
+// device_model/sm100.cuh -- host model of the library's sm100.cuh wrappers (mbarriers, TMA, tcgen05,
+// TMEM), so that the tensor-core kernels run unchanged on the CPU in tests (see build_library.py);
+// the library never includes it.  Modelled from the PTX ISA's description of each instruction:
+//   mbarrier: expected arrivals, pending arrivals, signed transaction bytes, phase; a phase completes
+//             when both reach zero; try_wait.parity P succeeds once the phase of parity P is over.
+//   TMA 2-D tile load/store: {64, box_rows} boxes of 16-bit elements, 128-byte swizzle by address
+//             (16-byte chunk c of the 128-byte row at smem address a goes to chunk c ^ ((a >> 7) & 7)),
+//             zero fill outside the tensor, completion as transaction bytes.
+//   tcgen05:  TMEM 128 lanes x 512 columns of 32 bits per block; MMAs are queued by the issuing thread
+//             and executed when it commits (then the commit arrives), so a read of an operand or of
+//             the accumulator before the commit is visible; SS and TS forms, kind::f16, M = 128; the
+//             16-term dot product of one instruction in FP64, added once to the FP32 accumulator.
+//   tcgen05.ld/st 32x32b: warp w reaches lanes 32 (w % 4) .. +31 only (checked).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include <chrono>
+#include <cstdio>
+#include <unordered_map>
+#include <vector>
+
+namespace mimo {
+
+enum : unsigned int {
+  kErrTimeout = 1u,
+  kErrRange = 2u,
+  kErrSeqlens = 4u,
+};
+
+inline uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(static_cast<const uint8_t*>(p) - hemu::g_smem);
+}
+inline uint8_t* smem_at(uint32_t a) { return hemu::g_smem + a; }
+
+inline uint64_t globaltimer_ns() {
+  return static_cast<uint64_t>(
+      std::chrono::duration_cast<std::chrono::nanoseconds>(std::chrono::steady_clock::now().time_since_epoch())
+          .count());
+}
+
+// ---------------------------------------------------------------- mbarrier
+struct MbarState {
+  uint32_t expected = 0, pending = 0;
+  int64_t tx = 0;
+  uint32_t phase = 0;
+  bool init = false;
+};
+inline std::unordered_map<uint32_t, MbarState> g_mbars;
+
+inline MbarState& mbar_state(const void* bar) {
+  MbarState& m = g_mbars[smem_u32(bar)];
+  if (!m.init) {
+    std::fprintf(stderr, "tcsim: mbarrier at smem %u used before init\n", smem_u32(bar));
+    ++hemu::g_errors;
+    m.init = true;
+    m.expected = m.pending = 1;
+  }
+  return m;
+}
+
+inline void mbar_check_phase(MbarState& m) {
+  if (m.pending == 0 && m.tx == 0) {
+    ++m.phase;
+    m.pending = m.expected;
+  }
+}
+
+inline void mbar_init(uint64_t* bar, uint32_t count) {
+  MbarState& m = g_mbars[smem_u32(bar)];
+  m = MbarState{};
+  m.init = true;
+  m.expected = m.pending = count;
+}
+inline void fence_barrier_init() {}
+
+inline void mbar_arrive_at(uint64_t* bar) {
+  MbarState& m = mbar_state(bar);
+  if (m.pending == 0) {
+    std::fprintf(stderr, "tcsim: arrival on a completed phase (smem %u)\n", smem_u32(bar));
+    ++hemu::g_errors;
+    return;
+  }
+  --m.pending;
+  mbar_check_phase(m);
+}
+inline void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  MbarState& m = mbar_state(bar);
+  m.tx -= bytes;
+  mbar_check_phase(m);
+}
+inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  MbarState& m = mbar_state(bar);
+  m.tx += bytes;
+  mbar_arrive_at(bar);
+}
+inline void mbar_arrive(uint64_t* bar) { mbar_arrive_at(bar); }
+
+inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  if ((mbar_state(bar).phase & 1u) != (parity & 1u)) return true;
+  hemu::yield();
+  return (mbar_state(bar).phase & 1u) != (parity & 1u);
+}
+inline bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t) { return mbar_try_wait(bar, parity); }
+
+constexpr uint32_t kWaitSliceNs = 1000000;
+
+inline bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSliceNs)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// ---------------------------------------------------------------- TMA
+struct HostTmap {
+  const uint8_t* base;
+  uint64_t inner, rows, stride;  // elements, rows, bytes per row
+  uint32_t box_inner, box_rows, elem;
+};
+static_assert(sizeof(HostTmap) <= sizeof(CUtensorMap), "tensor map model too large");
+
+inline void prefetch_tensormap(const CUtensorMap*) {}
+
+inline void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y) {
+  const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
+  uint8_t* d = static_cast<uint8_t*>(dst);
+  const uint32_t rb = t->box_inner * t->elem;
+  if (rb != 128 || (x * t->elem) % 16 != 0) {
+    std::fprintf(stderr, "tcsim: TMA box of %u bytes per row / x %d not 16-byte aligned\n", rb, x);
+    ++hemu::g_errors;
+  }
+  for (uint32_t r = 0; r < t->box_rows; ++r) {
+    uint8_t row[128];
+    const int64_t gy = static_cast<int64_t>(y) + r;
+    for (uint32_t i = 0; i < t->box_inner; ++i) {
+      const int64_t gx = static_cast<int64_t>(x) + i;
+      if (gy < 0 || gy >= static_cast<int64_t>(t->rows) || gx < 0 || gx >= static_cast<int64_t>(t->inner))
+        std::memset(row + i * t->elem, 0, t->elem);
+      else
+        std::memcpy(row + i * t->elem, t->base + gy * t->stride + gx * t->elem, t->elem);
+    }
+    const uint32_t a = smem_u32(d + r * rb);
+    for (uint32_t c = 0; c < 8; ++c) std::memcpy(d + r * rb + ((c ^ ((a >> 7) & 7u)) << 4), row + c * 16, 16);
+  }
+  mbar_complete_tx(bar, t->box_rows * rb);
+}
+
+inline void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y, uint64_t) {
+  tma_load_2d(dst, map, bar, x, y);
+}
+inline uint64_t policy_evict_first() { return 0; }
+inline uint64_t policy_evict_last() { return 0; }
+
+inline void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+  const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
+  const uint8_t* s = static_cast<const uint8_t*>(src);
+  const uint32_t rb = t->box_inner * t->elem;
+  for (uint32_t r = 0; r < t->box_rows; ++r) {
+    uint8_t row[128];
+    const uint32_t a = smem_u32(s + r * rb);
+    for (uint32_t c = 0; c < 8; ++c) std::memcpy(row + c * 16, s + r * rb + ((c ^ ((a >> 7) & 7u)) << 4), 16);
+    const int64_t gy = static_cast<int64_t>(y) + r;
+    if (gy < 0 || gy >= static_cast<int64_t>(t->rows)) continue;
+    for (uint32_t i = 0; i < t->box_inner; ++i) {
+      const int64_t gx = static_cast<int64_t>(x) + i;
+      if (gx >= 0 && gx < static_cast<int64_t>(t->inner))
+        std::memcpy(const_cast<uint8_t*>(t->base) + gy * t->stride + gx * t->elem, row + i * t->elem, t->elem);
+    }
+  }
+}
+inline void tma_store_commit() {}
+template <int N>
+inline void tma_store_wait_read() {}
+template <int N>
+inline void tma_store_wait() {}
+inline void fence_proxy_async_smem() {}
+
+// ---------------------------------------------------------------- TMEM and MMA
+inline uint32_t g_tmem[128][512];
+inline uint32_t g_tmem_next = 0;
+
+struct MmaOp {
+  bool ts;
+  uint32_t d, a_tmem;
+  uint64_t a, b;
+  uint32_t idesc, acc;
+};
+inline std::vector<MmaOp> g_mma_queue;
+
+inline void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  if (hemu::lin_tid() % 32 != 0) return;  // one allocation per warp
+  if (g_tmem_next + ncols > 512) {
+    std::fprintf(stderr, "tcsim: TMEM allocation beyond 512 columns\n");
+    ++hemu::g_errors;
+  }
+  *dst_smem = g_tmem_next;
+  g_tmem_next += ncols;
+}
+inline void tmem_relinquish() {}
+inline void tmem_dealloc(uint32_t, uint32_t) {}
+inline void tc_fence_before_sync() {}
+inline void tc_fence_after_sync() {}
+
+inline float f16_bits(uint16_t b, bool bf16) {
+  if (bf16) {
+    uint32_t u = static_cast<uint32_t>(b) << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    return f;
+  }
+  __half_raw r;
+  r.x = b;
+  return __half2float(__half(r));
+}
+
+// Element (mn, k) of a 128-byte-swizzled operand described by desc (K-major: mn rows of 128 bytes in
+// 8-row groups SBO apart; MN-major: k rows of 128 bytes holding 64 mn values, 8-row groups SBO apart,
+// 64-value column blocks LBO apart).
+inline float sdesc_elem(uint64_t desc, bool mn_major, uint32_t mn, uint32_t k, bool bf16) {
+  const uint32_t start = static_cast<uint32_t>(desc & 0x3FFFu) << 4;
+  const uint32_t lbo = static_cast<uint32_t>((desc >> 16) & 0x3FFFu) << 4;
+  const uint32_t sbo = static_cast<uint32_t>((desc >> 32) & 0x3FFFu) << 4;
+  if (((desc >> 61) & 7u) != 2u || ((desc >> 46) & 1u) != 1u) {
+    std::fprintf(stderr, "tcsim: descriptor without 128-byte swizzle or version bit\n");
+    ++hemu::g_errors;
+  }
+  uint32_t a = mn_major ? start + (mn / 64) * lbo + (k / 8) * sbo + (k % 8) * 128 + (mn % 64) * 2
+                        : start + (mn / 8) * sbo + (mn % 8) * 128 + k * 2;
+  a ^= ((a >> 7) & 7u) << 4;
+  uint16_t b;
+  std::memcpy(&b, smem_at(a), 2);
+  return f16_bits(b, bf16);
+}
+
+inline void mma_execute(const MmaOp& op) {
+  const uint32_t id = op.idesc;
+  const bool a_bf16 = ((id >> 7) & 7u) == 1u, b_bf16 = ((id >> 10) & 7u) == 1u;
+  const bool a_mn = (id >> 15) & 1u, b_mn = (id >> 16) & 1u;
+  const uint32_t N = ((id >> 17) & 0x3Fu) << 3, M = ((id >> 24) & 0x1Fu) << 4;
+  if (((id >> 4) & 3u) != 1u || a_bf16 != b_bf16 || M != 128 || a_mn) {
+    std::fprintf(stderr, "tcsim: unsupported instruction descriptor %08x\n", id);
+    ++hemu::g_errors;
+    return;
+  }
+  const uint32_t dl = op.d >> 16, dc = op.d & 0xFFFFu;
+  const uint32_t al = op.a_tmem >> 16, ac = op.a_tmem & 0xFFFFu;
+  static float A[128][16], B[256][16];
+  for (uint32_t m = 0; m < M; ++m)
+    for (uint32_t k = 0; k < 16; ++k) {
+      if (op.ts) {
+        const uint32_t w = g_tmem[al + m][ac + k / 2];
+        A[m][k] = f16_bits(static_cast<uint16_t>(k % 2 ? w >> 16 : w & 0xFFFFu), a_bf16);
+      } else {
+        A[m][k] = sdesc_elem(op.a, false, m, k, a_bf16);
+      }
+    }
+  for (uint32_t n = 0; n < N; ++n)
+    for (uint32_t k = 0; k < 16; ++k) B[n][k] = sdesc_elem(op.b, b_mn, n, k, b_bf16);
+  for (uint32_t m = 0; m < M; ++m)
+    for (uint32_t n = 0; n < N; ++n) {
+      double s = 0.0;
+      for (uint32_t k = 0; k < 16; ++k) s += static_cast<double>(A[m][k]) * B[n][k];
+      float acc = 0.f;
+      if (op.acc) std::memcpy(&acc, &g_tmem[dl + m][dc + n], 4);
+      acc = static_cast<float>(acc + s);
+      std::memcpy(&g_tmem[dl + m][dc + n], &acc, 4);
+    }
+}
+
+inline void tc_commit(uint64_t* bar) {
+  for (const MmaOp& op : g_mma_queue) mma_execute(op);
+  g_mma_queue.clear();
+  mbar_arrive_at(bar);
+}
+
+__host__ __device__ constexpr uint32_t make_idesc_f32acc(uint32_t ab_bf16, uint32_t b_mn_major, uint32_t M,
+                                                         uint32_t N) {
+  return (1u << 4) | (ab_bf16 << 7) | (ab_bf16 << 10) | (b_mn_major << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+inline uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+constexpr uint32_t kDescHiSw128Sbo1K = (1024u >> 4) | (1u << 14) | (2u << 29);
+__host__ __device__ constexpr uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+
+inline void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  g_mma_queue.push_back({false, d_tmem, 0, a_desc, b_desc, idesc, accumulate});
+}
+inline void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  g_mma_queue.push_back({true, d_tmem, a_tmem, 0, b_desc, idesc, accumulate});
+}
+inline void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc, uint32_t accumulate) {
+  const uint64_t hi = static_cast<uint64_t>(kDescHiSw128Sbo1K) << 32;
+  mma_ss(d_tmem, hi | a_lo, hi | b_lo, idesc, accumulate);
+}
+inline void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc, uint32_t accumulate) {
+  mma_ts(d_tmem, a_tmem, (static_cast<uint64_t>(kDescHiSw128Sbo1K) << 32) | b_lo, idesc, accumulate);
+}
+
+inline uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col) { return base + (lane << 16) + col; }
+
+inline void tmem_lane_check(uint32_t taddr) {
+  const uint32_t w = hemu::lin_tid() / 32;
+  if ((taddr >> 16) != 32 * (w % 4)) {
+    std::fprintf(stderr, "tcsim: warp %u addresses TMEM lanes from %u\n", w, taddr >> 16);
+    ++hemu::g_errors;
+  }
+}
+inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_lane_check(taddr);
+  const uint32_t lane = (taddr >> 16) + hemu::lin_tid() % 32, col = taddr & 0xFFFFu;
+  for (int j = 0; j < 32; ++j) r[j] = g_tmem[lane][col + j];
+}
+inline void tmem_ld_wait(uint32_t (&)[32]) {}
+inline void reg_fence(uint32_t (&)[32]) {}
+inline void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  tmem_lane_check(taddr);
+  const uint32_t lane = (taddr >> 16) + hemu::lin_tid() % 32, col = taddr & 0xFFFFu;
+  for (int j = 0; j < 32; ++j) g_tmem[lane][col + j] = r[j];
+}
+inline void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  tmem_lane_check(taddr);
+  const uint32_t lane = (taddr >> 16) + hemu::lin_tid() % 32, col = taddr & 0xFFFFu;
+  for (int j = 0; j < 16; ++j) g_tmem[lane][col + j] = r[j];
+}
+inline void tmem_st_wait() {}
+
+// ---------------------------------------------------------------- warp-group helpers
+inline void named_bar_sync(uint32_t id, uint32_t nthreads) { hemu::named_bar(static_cast<int>(id), nthreads, true); }
+inline bool named_bar_and(uint32_t id, uint32_t nthreads, bool pred) {
+  return hemu::named_bar(static_cast<int>(id), nthreads, pred);
+}
+template <uint32_t N>
+inline void setmaxnreg_inc() {}
+template <uint32_t N>
+inline void setmaxnreg_dec() {}
+
+inline void st_global_v8(void* dst, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4, uint32_t a5,
+                         uint32_t a6, uint32_t a7) {
+  const uint32_t v[8] = {a0, a1, a2, a3, a4, a5, a6, a7};
+  std::memcpy(dst, v, 32);
+}
+
+// ---------------------------------------------------------------- math helpers
+inline float ex2_approx(float x) { return exp2f(x); }
+inline uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  uint32_t u;
+  std::memcpy(&u, &v, 4);
+  return u;
+}
+
+// per-block state
+inline bool g_tc_reset_registered = [] {
+  hemu::g_block_reset.push_back([] {
+    g_mbars.clear();
+    g_tmem_next = 0;
+    g_mma_queue.clear();
+    std::memset(g_tmem, 0xFF, sizeof(g_tmem));
+  });
+  return true;
+}();
+
+}  // namespace mimo

@@ -1,10 +1,12 @@
-// fiber_runtime.h -- host emulation of the CUDA features that the CUDA-core kernels (backward, FP8
-// dequant, fused-QKV split, MoE router, KV-cache partial and combine) use, so that their unchanged
-// source runs on the CPU in tests:
+// fiber_runtime.h -- host emulation of the CUDA thread model, so that the library's kernels run on
+// the CPU in tests from their unchanged source (the CUDA-core kernels directly; the tensor-core kernels
+// with the device model of their tcgen05 / TMA / mbarrier wrappers in device_model/):
 //   - one fiber (ucontext) per CUDA thread, a cooperative scheduler per block, blocks one after another;
 //   - __syncthreads / __syncwarp as barriers over the block's / warp's live fibers (exited threads do
 //     not count, as on the GPU); a barrier that can never complete is reported as a deadlock;
-//   - warp shuffles through an exchange array, with an error if a lane of the warp has exited;
+//   - warp shuffles and votes through an exchange array, with an error if a lane has exited;
+//   - named barriers 1..15 with thread counts (bar.sync, bar.red.and) and __syncthreads_or;
+//   - a yield for spin-waits (a waiting fiber lets the others run);
 //   - atomics as plain read-modify-write (a single OS thread runs every fiber);
 //   - every buffer, and the block's dynamic shared memory, sits between two 16 MB PROT_NONE guard
 //     regions, flush against the one at its end in mode 0 and the one at its start in mode 1, so an
@@ -83,9 +85,19 @@ inline void guarded_free(void* p) {
 struct Fiber {
   ucontext_t ctx;
   bool done;
-  int wait;  // 0 runnable, 1 block barrier, 2 warp barrier
+  int wait;  // 0 runnable, 1 block barrier, 2 warp barrier, 3 named barrier
+  int bar_id;
   uint64_t gen;
+  bool result;  // reduction result handed back by a barrier
 };
+
+// named barriers 1..15 (bar.sync / bar.red.and): thread counts, arrivals, generations, AND reduction
+inline int g_nb_count[16], g_nb_arrived[16];
+inline uint64_t g_nb_gen[16];
+inline bool g_nb_and[16];
+inline bool g_block_or;
+inline std::vector<std::function<void()>> g_block_reset;  // per-block state of device models
+inline bool g_smem_start_aligned = false;
 
 inline uint3 g_tid_cur, g_bid_cur;
 inline dim3 g_grid_dim, g_block_dim;
@@ -111,6 +123,37 @@ inline void syncthreads() {
   f.gen = g_block_gen;
   ++g_block_arrived;
   swapcontext(&f.ctx, &g_sched);
+}
+
+inline bool syncthreads_or(bool pred) {
+  g_block_or = g_block_or || pred;
+  syncthreads();
+  return g_fibers[g_cur].result;
+}
+
+// Lets the other fibers run (a spin-wait step).
+inline void yield() {
+  Fiber& f = g_fibers[g_cur];
+  f.wait = 0;
+  swapcontext(&f.ctx, &g_sched);
+}
+
+inline bool named_bar(int id, int nthreads, bool pred) {
+  Fiber& f = g_fibers[g_cur];
+  if (g_nb_arrived[id] == 0) {
+    g_nb_count[id] = nthreads;
+    g_nb_and[id] = true;
+  } else if (g_nb_count[id] != nthreads) {
+    std::fprintf(stderr, "emu: named barrier %d used with %d and %d threads\n", id, g_nb_count[id], nthreads);
+    ++g_errors;
+  }
+  g_nb_and[id] = g_nb_and[id] && pred;
+  ++g_nb_arrived[id];
+  f.wait = 3;
+  f.bar_id = id;
+  f.gen = g_nb_gen[id];
+  swapcontext(&f.ctx, &g_sched);
+  return g_fibers[g_cur].result;
 }
 
 inline void syncwarp() {
@@ -151,7 +194,7 @@ inline void set_smem(size_t bytes) {
       mmap(nullptr, g_smem_map_bytes, PROT_READ | PROT_WRITE, MAP_PRIVATE | MAP_ANONYMOUS, -1, 0));
   mprotect(g_smem_map, kGuard, PROT_NONE);
   mprotect(g_smem_map + kGuard + body, kGuard, PROT_NONE);
-  g_smem = g_mode == 0 ? g_smem_map + kGuard + body - n16 : g_smem_map + kGuard;
+  g_smem = (g_mode == 0 && !g_smem_start_aligned) ? g_smem_map + kGuard + body - n16 : g_smem_map + kGuard;
 }
 
 // Runs fn (the kernel call) for every thread of every block.  Returns false on a barrier deadlock or a
@@ -179,6 +222,9 @@ inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function
         std::memset(g_smem, 0xFF, smem_bytes);
         g_block_gen = 0;
         g_block_arrived = 0;
+        g_block_or = false;
+        for (int i = 0; i < 16; ++i) g_nb_count[i] = g_nb_arrived[i] = 0, g_nb_gen[i] = 0;
+        for (auto& h : g_block_reset) h();
         std::fill(g_warp_arrived.begin(), g_warp_arrived.end(), 0);
         for (int i = 0; i < nt; ++i) {
           Fiber& f = g_fibers[i];
@@ -200,6 +246,7 @@ inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function
             if (f.done) continue;
             if (f.wait == 1 && f.gen == g_block_gen) continue;
             if (f.wait == 2 && f.gen == g_warp_gen[i / 32]) continue;
+            if (f.wait == 3 && f.gen == g_nb_gen[f.bar_id]) continue;
             f.wait = 0;
             g_cur = i;
             g_tid_cur = make_uint3(i % block.x, (i / block.x) % block.y, i / (block.x * block.y));
@@ -213,10 +260,23 @@ inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function
             }
           if (alive == 0) break;
           if (g_block_arrived > 0 && g_block_arrived == alive) {
+            for (int i = 0; i < nt; ++i)
+              if (!g_fibers[i].done && g_fibers[i].wait == 1) g_fibers[i].result = g_block_or;
             ++g_block_gen;
             g_block_arrived = 0;
+            g_block_or = false;
             progress = true;
           }
+          for (int id = 0; id < 16; ++id)
+            if (g_nb_arrived[id] > 0 && g_nb_arrived[id] == g_nb_count[id]) {
+              for (int i = 0; i < nt; ++i)
+                if (!g_fibers[i].done && g_fibers[i].wait == 3 && g_fibers[i].bar_id == id &&
+                    g_fibers[i].gen == g_nb_gen[id])
+                  g_fibers[i].result = g_nb_and[id];
+              ++g_nb_gen[id];
+              g_nb_arrived[id] = 0;
+              progress = true;
+            }
           for (int w = 0; w < nw; ++w)
             if (g_warp_arrived[w] > 0 && g_warp_arrived[w] == alive_w[w]) {
               if (alive_w[w] != std::min(32, nt - 32 * w)) {
@@ -253,6 +313,36 @@ template <class T>
 inline T __shfl_xor_sync(unsigned, T v, int o) { return hemu::shfl_idx(v, (hemu::lin_tid() % 32) ^ o); }
 template <class T>
 inline T __shfl_sync(unsigned, T v, int src) { return hemu::shfl_idx(v, src); }
+template <class T>
+inline T atomicAdd(T* p, T v) {
+  const T o = *p;
+  *p = o + v;
+  return o;
+}
+inline bool __all_sync(unsigned, int pred) {
+  const int l = hemu::lin_tid() % 32, w = hemu::lin_tid() / 32;
+  hemu::g_xch[w][l] = pred != 0;
+  hemu::syncwarp();
+  bool r = true;
+  for (int i = 0; i < 32; ++i) r = r && hemu::g_xch[w][i] != 0;
+  hemu::syncwarp();
+  return r;
+}
+inline bool __any_sync(unsigned, int pred) {
+  const int l = hemu::lin_tid() % 32, w = hemu::lin_tid() / 32;
+  hemu::g_xch[w][l] = pred != 0;
+  hemu::syncwarp();
+  bool r = false;
+  for (int i = 0; i < 32; ++i) r = r || hemu::g_xch[w][i] != 0;
+  hemu::syncwarp();
+  return r;
+}
+inline int __syncthreads_or(int pred) { return hemu::syncthreads_or(pred != 0); }
+inline uint32_t __float_as_uint(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return u;
+}
 inline float atomicAdd(float* p, float v) {
   const float o = *p;
   *p = o + v;

@@ -1,0 +1,132 @@
+"""Cases for the host build of the whole library (tensor-core kernels through the device model),
+checked against the oracle with the forward tolerances.  Run as a child process:
+
+    python library_cases.py <libmimo_attn_host.so> <case> [<case> ...]
+"""
+import ctypes as C
+import os
+import sys
+
+import numpy as np
+
+TESTS = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, os.path.dirname(TESTS))
+sys.path.insert(0, TESTS)
+import oracle  # noqa: E402
+from global_attention_moe_b200 import synth, workloads as W  # noqa: E402
+from decode_helpers import decode_reference  # noqa: E402
+
+TOL_MAX_ABS, TOL_REL_L2, TOL_LSE = 2e-2, 5e-3, 1e-3
+KERNEL = {"auto": 0, "simple": 1, "pipelined": 2, "window": 3}
+DECODE = {"auto": 0, "cuda_cores": 1, "tensor": 2}
+vp = C.c_void_p
+
+
+class Dims(C.Structure):
+    _fields_ = [(n, C.c_int32) for n in ("num_seqs", "total_tokens", "max_seqlen", "num_q_heads", "num_kv_heads",
+                                         "head_dim_qk", "head_dim_v")]
+
+
+class DecodeDims(C.Structure):
+    _fields_ = [(n, C.c_int32) for n in ("num_seqs", "total_q", "total_kv", "cache_rows", "max_q_len", "max_kv_len",
+                                         "num_q_heads", "num_kv_heads", "head_dim_qk", "head_dim_v")]
+
+
+class Lib:
+    def __init__(self, path):
+        L = self.L = C.CDLL(path)
+        L.hemu_alloc.restype = vp
+        L.hemu_alloc.argtypes = [C.c_size_t]
+        L.hemu_free.argtypes = [vp]
+        L.mimo_attn_fwd.argtypes = [vp, vp, vp, vp, vp, C.POINTER(Dims), C.c_int, C.c_int, C.c_double, C.c_int,
+                                    C.c_float, vp, vp, vp]
+        L.mimo_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, C.POINTER(DecodeDims), C.c_int, C.c_int,
+                                       C.c_double, C.c_int, C.c_float, vp, vp, vp]
+        L.mimo_attn_check.argtypes = [vp]
+        self.live = []
+
+    def put(self, a):
+        if a is None:
+            return None
+        a = np.ascontiguousarray(a)
+        p = self.L.hemu_alloc(max(a.nbytes, 1))
+        C.memmove(p, a.ctypes.data, a.nbytes)
+        self.live.append(p)
+        return p
+
+    def empty(self, nbytes):
+        p = self.L.hemu_alloc(max(nbytes, 1))
+        self.live.append(p)
+        return p
+
+    def get(self, p, shape, dtype):
+        a = np.empty(shape, dtype=dtype)
+        C.memmove(a.ctypes.data, p, a.nbytes)
+        return a
+
+    def finish(self, status):
+        while self.live:
+            self.L.hemu_free(self.live.pop())
+        assert status == 0, f"status {status}"
+        assert self.L.hemu_errors() == 0, "device-model or barrier error"
+        st = self.L.mimo_attn_check(None)
+        assert st == 0, f"kernel error status {st}"
+
+
+def check(out_bits, lse, ro, rl):
+    out = synth.bf16_bits_to_f32(out_bits).astype(np.float64)
+    d = out - ro
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    assert np.max(np.abs(d)) <= TOL_MAX_ABS, np.max(np.abs(d))
+    assert np.linalg.norm(d) / np.linalg.norm(ro) <= TOL_REL_L2
+    assert np.max(np.abs(lse - rl)) <= TOL_LSE, np.max(np.abs(lse - rl))
+
+
+def fwd(H, w, kernel):
+    x = W.make_inputs(w)
+    T, hq = w.total_tokens, w.num_q_heads
+    d = Dims(w.num_seqs, T, w.max_seqlen, hq, w.num_kv_heads, 192, 128)
+    assert H.L.mimo_attn_set_kernel(KERNEL[kernel]) == 0
+    po, pl = H.empty(T * hq * 128 * 2), H.empty(hq * T * 4)
+    st = H.L.mimo_attn_fwd(H.put(x.q), H.put(x.k), H.put(x.v), H.put(x.sink), H.put(x.cu_seqlens), C.byref(d),
+                           w.layer_kind, w.window, w.rope_base, 64, 0.707, po, pl, None)
+    out, lse = H.get(po, (T, hq, 128), np.uint16), H.get(pl, (hq, T), np.float32).astype(np.float64)
+    H.L.mimo_attn_set_kernel(0)
+    H.finish(st)
+    check(out, lse, *oracle.attn_fwd(x.q, x.k, x.v, x.sink, x.cu_seqlens, w.window, w.rope_base))
+
+
+def decode(H, kv, ql, hq, hkv, layer, window, base, has_sink, seed, kernel="tensor"):
+    x = W.make_decode_inputs(kv, ql, hq, hkv, has_sink, seed)
+    Tq = int(sum(ql))
+    d = DecodeDims(len(kv), Tq, int(sum(kv)), x.k_cache.shape[0], max(ql), max(kv), hq, hkv, 192, 128)
+    assert H.L.mimo_attn_set_decode_kernel(DECODE[kernel]) == 0
+    po, pl = H.empty(Tq * hq * 128 * 2), H.empty(hq * Tq * 4)
+    st = H.L.mimo_attn_decode(H.put(x.q), H.put(x.k_cache), H.put(x.v_cache), H.put(x.kv_indices),
+                              H.put(x.kv_indptr), H.put(x.cu_q), H.put(x.sink), C.byref(d), layer, window, base, 64,
+                              0.707, po, pl, None)
+    out, lse = H.get(po, (Tq, hq, 128), np.uint16), H.get(pl, (hq, Tq), np.float32).astype(np.float64)
+    H.L.mimo_attn_set_decode_kernel(0)
+    H.finish(st)
+    check(out, lse, *decode_reference(x, window if layer == W.LAYER_SWA else -1, base))
+
+
+CASES = {
+    # the three forward kernels on the small sliding-window config (T = 512, 4 query heads, 1 KV head)
+    "fwd_tiny_simple": lambda H: fwd(H, W.tiny_swa(), "simple"),
+    "fwd_tiny_pipelined": lambda H: fwd(H, W.tiny_swa(), "pipelined"),
+    "fwd_tiny_window": lambda H: fwd(H, W.tiny_swa(), "window"),
+    # ragged sequences across the 128-row tile and window edges; the global layer
+    "fwd_ragged_swa": lambda H: fwd(H, W.custom("ragged", W.LAYER_SWA, [1, 129, 257, 0, 5], 4, 2, 128, 1e4, True), "auto"),
+    "fwd_global": lambda H: fwd(H, W.custom("glob", W.LAYER_GLOBAL, [300, 77], 4, 2, -1, 1e7, False), "auto"),
+    # the tensor-core KV-cache kernel: decode and speculative chunks, then 128-row tiles
+    "decode_tensor": lambda H: decode(H, [5, 129, 300, 64], [1, 8, 3, 8], 8, 2, W.LAYER_SWA, 128, 1e4, True, 71),
+    "decode_tensor_tiles_swa": lambda H: decode(H, [600, 90], [300, 20], 8, 2, W.LAYER_SWA, 128, 1e4, True, 72),
+    "decode_tensor_tiles_global": lambda H: decode(H, [200, 50], [36, 50], 8, 1, W.LAYER_GLOBAL, -1, 1e7, False, 73),
+}
+
+if __name__ == "__main__":
+    H = Lib(sys.argv[1])
+    for name in sys.argv[2:]:
+        CASES[name](H)
+        print("ok", name, flush=True)

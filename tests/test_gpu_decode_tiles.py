@@ -1,6 +1,6 @@
-"""GPU parity of the KV-cache path above 128 query rows per KV head (chunked prefill): the CUDA-core
-kernel's 128-row tiles, each tile's keys clipped to its rows' positions, and the combine reading the
-splits that overlap the token's tile; the tensor-core kernel holds one tile and refuses more."""
+"""GPU parity of the KV-cache path above 128 query rows per KV head (chunked prefill) on both kernels:
+128-row tiles as one more dimension of the work, each tile's keys clipped to its rows' positions, and
+the combine reading the splits that overlap the token's tile."""
 import numpy as np
 import pytest
 import torch
@@ -35,16 +35,10 @@ def parity(x, layer, window, base):
 
 
 def test_rows_per_kv_head_above_128(dkernel):
-    """9 and 12 new tokens x 16 heads = 144 and 192 rows per KV head: two row tiles on the CUDA-core
-    kernel; the tensor-core kernel holds one 128-row tile and refuses."""
+    """9 and 12 new tokens x 16 heads = 144 and 192 rows per KV head: two row tiles."""
     from global_attention_moe_b200 import mimo_attn
     x = W.make_decode_inputs([40, 300], [9, 12], 64, 4, False, seed=37)
-    if dkernel == "tensor":
-        with pytest.raises(mimo_attn.MimoAttnError) as e:
-            decode_gpu(x, W.LAYER_GLOBAL, -1, 1e7)
-        assert e.value.status == mimo_attn.ERR_UNSUPPORTED
-    else:
-        parity(x, W.LAYER_GLOBAL, -1, 1e7)
+    parity(x, W.LAYER_GLOBAL, -1, 1e7)
 
 
 @pytest.mark.parametrize("kind", ["swa", "global"])
@@ -53,9 +47,6 @@ def test_chunked_prefill(kind, dkernel):
     prompt as one chunk: row tiles, each tile's keys clipped to its rows' positions, and the splits
     merged per tile.  The automatic choice runs them (on the CUDA-core kernel)."""
     from global_attention_moe_b200 import mimo_attn
-    if dkernel == "tensor":
-        pytest.skip("the tensor-core kernel holds one 128-row tile")
-    mimo_attn.set_decode_kernel(mimo_attn.DECODE_AUTO)
     kv = [1200, 700, 300, 129]
     ql = [300, 200, 300, 64]
     if kind == "swa":

@@ -1,0 +1,51 @@
+"""The whole library built for the CPU, tensor-core kernels included: their unchanged source runs on
+the fiber runtime with a device model of the tcgen05 / TMA / mbarrier wrappers
+(tests/host_emulation/device_model), and the results are compared with the oracle at the forward's
+tolerances.  The model reproduces the errors measured on a B200 for the tensor-core forward kernels
+on the small sliding-window config (max-abs 4.4e-3 simple, 7.3e-3 pipelined), i.e. the same
+rounding points.  Planted mistakes in the kernels' operand addressing and row tiling are caught."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+EMU = os.path.join(HERE, "host_emulation")
+sys.path.insert(0, EMU)
+import build_library  # noqa: E402
+from library_cases import CASES  # noqa: E402
+
+
+def run_cases(lib, names):
+    r = subprocess.run([sys.executable, os.path.join(EMU, "library_cases.py"), lib, *names], capture_output=True,
+                       text=True, timeout=900)
+    return r.returncode, (r.stdout + r.stderr)[-2000:]
+
+
+@pytest.fixture(scope="module")
+def host_library(tmp_path_factory):
+    return build_library.build(str(tmp_path_factory.mktemp("library_host")))
+
+
+def test_library_matches_oracle(host_library):
+    rc, log = run_cases(host_library, list(CASES))
+    assert rc == 0, log
+
+
+PLANTED = [
+    ("rotated-dims K operand not advanced per K-step", "attn_fwd_pipelined.cuh",
+     "mma_ss_lo(d_tmem, q0 + 2 * sub, k0 + 2 * sub, pipe::kIdescSF16",
+     "mma_ss_lo(d_tmem, q0 + 2 * sub, k0, pipe::kIdescSF16", "fwd_tiny_pipelined"),
+    ("V operand stepped by 8 keys instead of 16", "attn_fwd_pipelined.cuh",
+     "v_lo + kk * (2048 >> 4)", "v_lo + kk * (1024 >> 4)", "fwd_tiny_pipelined"),
+    ("KV-cache row tiles all start at row 0", "attn_decode_tc.cuh", "w.row0 = 128 * qt;", "w.row0 = 0;",
+     "decode_tensor_tiles_swa"),
+]
+
+
+@pytest.mark.parametrize("what,file,old,new,case", PLANTED, ids=[p[0] for p in PLANTED])
+def test_planted_kernel_mistake_is_caught(tmp_path, what, file, old, new, case):
+    lib = build_library.build(str(tmp_path), mutations=[(file, old, new)])
+    rc, _ = run_cases(lib, [case])
+    assert rc != 0, f"not caught: {what}"
