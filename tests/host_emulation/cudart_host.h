@@ -79,3 +79,8 @@ cudaError_t cudaGetSymbolAddress(void** p, const T& sym) {
 }
 template <class T>
 cudaError_t cudaFuncSetAttribute(T*, enum cudaFuncAttribute, int) { return cudaSuccess; }
+
+extern "C" cudaError_t cudaOccupancyMaxActiveClusters(int* n, const void*, const cudaLaunchConfig_t* cfg) {
+  *n = static_cast<int>(cfg->gridDim.x / 2);  // one two-CTA cluster per SM pair
+  return cudaSuccess;
+}

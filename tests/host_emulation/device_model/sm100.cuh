@@ -49,18 +49,19 @@ struct MbarState {
   uint32_t phase = 0;
   bool init = false;
 };
-inline std::unordered_map<uint32_t, MbarState> g_mbars;
+inline std::unordered_map<uint32_t, MbarState> g_mbars[hemu::kMaxCluster];  // per CTA, by smem offset
 
-inline MbarState& mbar_state(const void* bar) {
-  MbarState& m = g_mbars[smem_u32(bar)];
+inline MbarState& mbar_state_at(int cta, uint32_t off) {
+  MbarState& m = g_mbars[cta][off];
   if (!m.init) {
-    std::fprintf(stderr, "tcsim: mbarrier at smem %u used before init\n", smem_u32(bar));
+    std::fprintf(stderr, "tcsim: mbarrier at smem %u of CTA %d used before init\n", off, cta);
     ++hemu::g_errors;
     m.init = true;
     m.expected = m.pending = 1;
   }
   return m;
 }
+inline MbarState& mbar_state(const void* bar) { return mbar_state_at(hemu::g_cur_cta, smem_u32(bar)); }
 
 inline void mbar_check_phase(MbarState& m) {
   if (m.pending == 0 && m.tx == 0) {
@@ -70,28 +71,38 @@ inline void mbar_check_phase(MbarState& m) {
 }
 
 inline void mbar_init(uint64_t* bar, uint32_t count) {
-  MbarState& m = g_mbars[smem_u32(bar)];
+  MbarState& m = g_mbars[hemu::g_cur_cta][smem_u32(bar)];
   m = MbarState{};
   m.init = true;
   m.expected = m.pending = count;
 }
 inline void fence_barrier_init() {}
 
-inline void mbar_arrive_at(uint64_t* bar) {
-  MbarState& m = mbar_state(bar);
+inline void mbar_arrive_cta(int cta, uint32_t off) {
+  MbarState& m = mbar_state_at(cta, off);
   if (m.pending == 0) {
-    std::fprintf(stderr, "tcsim: arrival on a completed phase (smem %u)\n", smem_u32(bar));
+    std::fprintf(stderr, "tcsim: arrival on a completed phase (smem %u of CTA %d)\n", off, cta);
     ++hemu::g_errors;
     return;
   }
   --m.pending;
   mbar_check_phase(m);
 }
-inline void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
-  MbarState& m = mbar_state(bar);
+inline void mbar_arrive_at(uint64_t* bar) { mbar_arrive_cta(hemu::g_cur_cta, smem_u32(bar)); }
+inline void mbar_complete_tx_cta(int cta, uint32_t off, uint32_t bytes) {
+  MbarState& m = mbar_state_at(cta, off);
   m.tx -= bytes;
   mbar_check_phase(m);
 }
+inline void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  mbar_complete_tx_cta(hemu::g_cur_cta, smem_u32(bar), bytes);
+}
+
+// shared::cluster addresses: mapa results carry the target CTA as (rank + 1) << 24; a plain
+// shared::cta offset means the executing CTA.
+inline uint32_t cluster_addr(uint32_t off, uint32_t rank) { return ((rank + 1u) << 24) | off; }
+inline int cluster_cta(uint32_t a) { return (a >> 24) ? static_cast<int>((a >> 24) - 1u) : hemu::g_cur_cta; }
+inline uint32_t cluster_off(uint32_t a) { return a & 0xFFFFFFu; }
 inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   MbarState& m = mbar_state(bar);
   m.tx += bytes;
@@ -127,7 +138,19 @@ static_assert(sizeof(HostTmap) <= sizeof(CUtensorMap), "tensor map model too lar
 
 inline void prefetch_tensormap(const CUtensorMap*) {}
 
+inline void tma_box_to_smem(void* dst, const CUtensorMap* map, int32_t x, int32_t y);
 inline void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y) {
+  tma_box_to_smem(dst, map, x, y);
+  const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
+  mbar_complete_tx(bar, t->box_rows * t->box_inner * t->elem);
+}
+// Pair form: the box lands in this CTA's shared memory, its bytes count on the (leader's) barrier.
+inline void tma_load_2d_pair_model(void* dst, const CUtensorMap* map, uint32_t bar, int32_t x, int32_t y) {
+  tma_box_to_smem(dst, map, x, y);
+  const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
+  mbar_complete_tx_cta(cluster_cta(bar), cluster_off(bar), t->box_rows * t->box_inner * t->elem);
+}
+inline void tma_box_to_smem(void* dst, const CUtensorMap* map, int32_t x, int32_t y) {
   const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
   uint8_t* d = static_cast<uint8_t*>(dst);
   const uint32_t rb = t->box_inner * t->elem;
@@ -148,7 +171,6 @@ inline void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_
     const uint32_t a = smem_u32(d + r * rb);
     for (uint32_t c = 0; c < 8; ++c) std::memcpy(d + r * rb + ((c ^ ((a >> 7) & 7u)) << 4), row + c * 16, 16);
   }
-  mbar_complete_tx(bar, t->box_rows * rb);
 }
 
 inline void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y, uint64_t) {
@@ -182,11 +204,12 @@ inline void tma_store_wait() {}
 inline void fence_proxy_async_smem() {}
 
 // ---------------------------------------------------------------- TMEM and MMA
-inline uint32_t g_tmem[128][512];
-inline uint32_t g_tmem_next = 0;
+inline uint32_t g_tmem_all[hemu::kMaxCluster][128][512];  // per CTA
+inline uint32_t g_tmem_next[hemu::kMaxCluster] = {};
 
 struct MmaOp {
-  bool ts;
+  bool ts, pair;
+  int cta;  // issuing CTA
   uint32_t d, a_tmem;
   uint64_t a, b;
   uint32_t idesc, acc;
@@ -195,12 +218,13 @@ inline std::vector<MmaOp> g_mma_queue;
 
 inline void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   if (hemu::lin_tid() % 32 != 0) return;  // one allocation per warp
-  if (g_tmem_next + ncols > 512) {
+  uint32_t& next = g_tmem_next[hemu::g_cur_cta];
+  if (next + ncols > 512) {
     std::fprintf(stderr, "tcsim: TMEM allocation beyond 512 columns\n");
     ++hemu::g_errors;
   }
-  *dst_smem = g_tmem_next;
-  g_tmem_next += ncols;
+  *dst_smem = next;
+  next += ncols;
 }
 inline void tmem_relinquish() {}
 inline void tmem_dealloc(uint32_t, uint32_t) {}
@@ -222,7 +246,7 @@ inline float f16_bits(uint16_t b, bool bf16) {
 // Element (mn, k) of a 128-byte-swizzled operand described by desc (K-major: mn rows of 128 bytes in
 // 8-row groups SBO apart; MN-major: k rows of 128 bytes holding 64 mn values, 8-row groups SBO apart,
 // 64-value column blocks LBO apart).
-inline float sdesc_elem(uint64_t desc, bool mn_major, uint32_t mn, uint32_t k, bool bf16) {
+inline float sdesc_elem(const uint8_t* base, uint64_t desc, bool mn_major, uint32_t mn, uint32_t k, bool bf16) {
   const uint32_t start = static_cast<uint32_t>(desc & 0x3FFFu) << 4;
   const uint32_t lbo = static_cast<uint32_t>((desc >> 16) & 0x3FFFu) << 4;
   const uint32_t sbo = static_cast<uint32_t>((desc >> 32) & 0x3FFFu) << 4;
@@ -234,7 +258,7 @@ inline float sdesc_elem(uint64_t desc, bool mn_major, uint32_t mn, uint32_t k, b
                         : start + (mn / 8) * sbo + (mn % 8) * 128 + k * 2;
   a ^= ((a >> 7) & 7u) << 4;
   uint16_t b;
-  std::memcpy(&b, smem_at(a), 2);
+  std::memcpy(&b, base + a, 2);
   return f16_bits(b, bf16);
 }
 
@@ -243,40 +267,60 @@ inline void mma_execute(const MmaOp& op) {
   const bool a_bf16 = ((id >> 7) & 7u) == 1u, b_bf16 = ((id >> 10) & 7u) == 1u;
   const bool a_mn = (id >> 15) & 1u, b_mn = (id >> 16) & 1u;
   const uint32_t N = ((id >> 17) & 0x3Fu) << 3, M = ((id >> 24) & 0x1Fu) << 4;
-  if (((id >> 4) & 3u) != 1u || a_bf16 != b_bf16 || M != 128 || a_mn) {
+  // single CTA: M = 128 rows in the issuer's TMEM and smem; pair (cta_group::2): M = 256, rows
+  // 0..127 in CTA 0 and 128..255 in CTA 1 (A from each CTA's smem or TMEM, D into each CTA's TMEM),
+  // B's N rows split in halves, the first from CTA 0's smem and the second from CTA 1's, at the same
+  // descriptor address.
+  const uint32_t Mc = op.pair ? 256u : 128u;
+  if (((id >> 4) & 3u) != 1u || a_bf16 != b_bf16 || M != Mc || a_mn || (op.pair && N % 16 != 0)) {
     std::fprintf(stderr, "tcsim: unsupported instruction descriptor %08x\n", id);
     ++hemu::g_errors;
     return;
   }
+  const int c0 = op.pair ? 0 : op.cta;
   const uint32_t dl = op.d >> 16, dc = op.d & 0xFFFFu;
   const uint32_t al = op.a_tmem >> 16, ac = op.a_tmem & 0xFFFFu;
-  static float A[128][16], B[256][16];
-  for (uint32_t m = 0; m < M; ++m)
+  static float A[256][16], B[256][16];
+  for (uint32_t m = 0; m < M; ++m) {
+    const int cta = c0 + static_cast<int>(m / 128);
     for (uint32_t k = 0; k < 16; ++k) {
       if (op.ts) {
-        const uint32_t w = g_tmem[al + m][ac + k / 2];
+        const uint32_t w = g_tmem_all[cta][al + m % 128][ac + k / 2];
         A[m][k] = f16_bits(static_cast<uint16_t>(k % 2 ? w >> 16 : w & 0xFFFFu), a_bf16);
       } else {
-        A[m][k] = sdesc_elem(op.a, false, m, k, a_bf16);
+        A[m][k] = sdesc_elem(hemu::g_smem_cta[cta], op.a, false, m % 128, k, a_bf16);
       }
     }
-  for (uint32_t n = 0; n < N; ++n)
-    for (uint32_t k = 0; k < 16; ++k) B[n][k] = sdesc_elem(op.b, b_mn, n, k, b_bf16);
-  for (uint32_t m = 0; m < M; ++m)
+  }
+  for (uint32_t n = 0; n < N; ++n) {
+    const uint32_t half = op.pair ? N / 2 : N;
+    const int cta = c0 + static_cast<int>(n / half);
+    for (uint32_t k = 0; k < 16; ++k) B[n][k] = sdesc_elem(hemu::g_smem_cta[cta], op.b, b_mn, n % half, k, b_bf16);
+  }
+  for (uint32_t m = 0; m < M; ++m) {
+    uint32_t (&T)[128][512] = g_tmem_all[c0 + static_cast<int>(m / 128)];
     for (uint32_t n = 0; n < N; ++n) {
       double s = 0.0;
       for (uint32_t k = 0; k < 16; ++k) s += static_cast<double>(A[m][k]) * B[n][k];
       float acc = 0.f;
-      if (op.acc) std::memcpy(&acc, &g_tmem[dl + m][dc + n], 4);
+      if (op.acc) std::memcpy(&acc, &T[dl + m % 128][dc + n], 4);
       acc = static_cast<float>(acc + s);
-      std::memcpy(&g_tmem[dl + m][dc + n], &acc, 4);
+      std::memcpy(&T[dl + m % 128][dc + n], &acc, 4);
     }
+  }
 }
 
 inline void tc_commit(uint64_t* bar) {
   for (const MmaOp& op : g_mma_queue) mma_execute(op);
   g_mma_queue.clear();
   mbar_arrive_at(bar);
+}
+// Pair commit with multicast: arrives on the barrier at the same offset in every CTA of the mask.
+inline void tc_commit_multicast(uint64_t* bar, uint16_t mask) {
+  for (const MmaOp& op : g_mma_queue) mma_execute(op);
+  g_mma_queue.clear();
+  for (int c = 0; c < hemu::g_cluster; ++c)
+    if ((mask >> c) & 1u) mbar_arrive_cta(c, smem_u32(bar));
 }
 
 __host__ __device__ constexpr uint32_t make_idesc_f32acc(uint32_t ab_bf16, uint32_t b_mn_major, uint32_t M,
@@ -299,10 +343,24 @@ __host__ __device__ constexpr uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) {
 }
 
 inline void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
-  g_mma_queue.push_back({false, d_tmem, 0, a_desc, b_desc, idesc, accumulate});
+  g_mma_queue.push_back({false, false, hemu::g_cur_cta, d_tmem, 0, a_desc, b_desc, idesc, accumulate});
 }
 inline void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
-  g_mma_queue.push_back({true, d_tmem, a_tmem, 0, b_desc, idesc, accumulate});
+  g_mma_queue.push_back({true, false, hemu::g_cur_cta, d_tmem, a_tmem, 0, b_desc, idesc, accumulate});
+}
+inline void mma_ss_pair_model(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if (hemu::g_cur_cta % 2 != 0) {
+    std::fprintf(stderr, "tcsim: pair MMA issued by an odd CTA\n");
+    ++hemu::g_errors;
+  }
+  g_mma_queue.push_back({false, true, hemu::g_cur_cta, d, 0, a, b, idesc, acc});
+}
+inline void mma_ts_pair_model(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if (hemu::g_cur_cta % 2 != 0) {
+    std::fprintf(stderr, "tcsim: pair MMA issued by an odd CTA\n");
+    ++hemu::g_errors;
+  }
+  g_mma_queue.push_back({true, true, hemu::g_cur_cta, d, a_tmem, 0, b, idesc, acc});
 }
 inline void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc, uint32_t accumulate) {
   const uint64_t hi = static_cast<uint64_t>(kDescHiSw128Sbo1K) << 32;
@@ -324,19 +382,19 @@ inline void tmem_lane_check(uint32_t taddr) {
 inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   tmem_lane_check(taddr);
   const uint32_t lane = (taddr >> 16) + hemu::lin_tid() % 32, col = taddr & 0xFFFFu;
-  for (int j = 0; j < 32; ++j) r[j] = g_tmem[lane][col + j];
+  for (int j = 0; j < 32; ++j) r[j] = g_tmem_all[hemu::g_cur_cta][lane][col + j];
 }
 inline void tmem_ld_wait(uint32_t (&)[32]) {}
 inline void reg_fence(uint32_t (&)[32]) {}
 inline void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   tmem_lane_check(taddr);
   const uint32_t lane = (taddr >> 16) + hemu::lin_tid() % 32, col = taddr & 0xFFFFu;
-  for (int j = 0; j < 32; ++j) g_tmem[lane][col + j] = r[j];
+  for (int j = 0; j < 32; ++j) g_tmem_all[hemu::g_cur_cta][lane][col + j] = r[j];
 }
 inline void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   tmem_lane_check(taddr);
   const uint32_t lane = (taddr >> 16) + hemu::lin_tid() % 32, col = taddr & 0xFFFFu;
-  for (int j = 0; j < 16; ++j) g_tmem[lane][col + j] = r[j];
+  for (int j = 0; j < 16; ++j) g_tmem_all[hemu::g_cur_cta][lane][col + j] = r[j];
 }
 inline void tmem_st_wait() {}
 
@@ -367,11 +425,11 @@ inline uint32_t pack_bf16x2(float lo, float hi) {
 
 // per-block state
 inline bool g_tc_reset_registered = [] {
-  hemu::g_block_reset.push_back([] {
-    g_mbars.clear();
-    g_tmem_next = 0;
+  hemu::g_block_reset.push_back([](int c) {
+    g_mbars[c].clear();
+    g_tmem_next[c] = 0;
     g_mma_queue.clear();
-    std::memset(g_tmem, 0xFF, sizeof(g_tmem));
+    std::memset(g_tmem_all[c], 0xFF, sizeof(g_tmem_all[c]));
   });
   return true;
 }();

@@ -40,6 +40,7 @@
 #undef __host__
 #define __host__
 #define __launch_bounds__(...)
+#define __cluster_dims__(...)
 #define __grid_constant__
 #undef __shared__
 #define __shared__ static
@@ -85,18 +86,30 @@ inline void guarded_free(void* p) {
 struct Fiber {
   ucontext_t ctx;
   bool done;
-  int wait;  // 0 runnable, 1 block barrier, 2 warp barrier, 3 named barrier
+  int wait;  // 0 runnable, 1 block barrier, 2 warp barrier, 3 named barrier, 4 cluster barrier
   int bar_id;
+  int cta;   // CTA of the fiber within its cluster
   uint64_t gen;
   bool result;  // reduction result handed back by a barrier
 };
 
-// named barriers 1..15 (bar.sync / bar.red.and): thread counts, arrivals, generations, AND reduction
-inline int g_nb_count[16], g_nb_arrived[16];
-inline uint64_t g_nb_gen[16];
-inline bool g_nb_and[16];
-inline bool g_block_or;
-inline std::vector<std::function<void()>> g_block_reset;  // per-block state of device models
+constexpr int kMaxCluster = 8;
+// Per-CTA barrier state (the blocks of one cluster run together): block barrier (bar.sync 0, with the
+// OR reduction of __syncthreads_or) and named barriers 1..15 (thread counts, AND reduction).
+struct CtaState {
+  uint64_t block_gen = 0;
+  int block_arrived = 0;
+  bool block_or = false;
+  int nb_count[16] = {}, nb_arrived[16] = {};
+  uint64_t nb_gen[16] = {};
+  bool nb_and[16] = {};
+};
+inline CtaState g_cta[kMaxCluster];
+inline int g_cluster = 1;    // CTAs per cluster of the current launch
+inline int g_cur_cta = 0;    // CTA of the running fiber
+inline uint64_t g_cl_gen = 0;
+inline int g_cl_arrived = 0;
+inline std::vector<std::function<void(int)>> g_block_reset;  // per-CTA state of device models (CTA index)
 inline bool g_smem_start_aligned = false;
 
 inline uint3 g_tid_cur, g_bid_cur;
@@ -106,29 +119,40 @@ inline std::vector<uint8_t*> g_stacks;
 inline constexpr size_t kStack = 256 * 1024;
 inline ucontext_t g_sched;
 inline int g_cur = -1;
-inline uint64_t g_block_gen;
-inline int g_block_arrived;
 inline std::vector<uint64_t> g_warp_gen;
 inline std::vector<int> g_warp_arrived;
 inline std::function<void()> g_body;
-inline uint8_t* g_smem = nullptr;
-inline uint64_t g_xch[64][32];
+inline uint8_t* g_smem = nullptr;  // the running fiber's CTA's shared memory
+inline uint8_t* g_smem_cta[kMaxCluster] = {};
+inline uint64_t g_xch[64 * kMaxCluster][32];
 inline int g_errors = 0;
 
 inline int lin_tid() { return static_cast<int>(g_tid_cur.x + g_block_dim.x * (g_tid_cur.y + g_block_dim.y * g_tid_cur.z)); }
+inline int warp_slot() { return g_cur / 32; }  // warp index over the whole cluster
 
 inline void syncthreads() {
   Fiber& f = g_fibers[g_cur];
+  CtaState& c = g_cta[f.cta];
   f.wait = 1;
-  f.gen = g_block_gen;
-  ++g_block_arrived;
+  f.gen = c.block_gen;
+  ++c.block_arrived;
   swapcontext(&f.ctx, &g_sched);
 }
 
 inline bool syncthreads_or(bool pred) {
-  g_block_or = g_block_or || pred;
+  CtaState& c = g_cta[g_fibers[g_cur].cta];
+  c.block_or = c.block_or || pred;
   syncthreads();
   return g_fibers[g_cur].result;
+}
+
+// Every thread of every CTA of the cluster (barrier.cluster arrive + wait).
+inline void cluster_barrier() {
+  Fiber& f = g_fibers[g_cur];
+  f.wait = 4;
+  f.gen = g_cl_gen;
+  ++g_cl_arrived;
+  swapcontext(&f.ctx, &g_sched);
 }
 
 // Lets the other fibers run (a spin-wait step).
@@ -140,25 +164,26 @@ inline void yield() {
 
 inline bool named_bar(int id, int nthreads, bool pred) {
   Fiber& f = g_fibers[g_cur];
-  if (g_nb_arrived[id] == 0) {
-    g_nb_count[id] = nthreads;
-    g_nb_and[id] = true;
-  } else if (g_nb_count[id] != nthreads) {
-    std::fprintf(stderr, "emu: named barrier %d used with %d and %d threads\n", id, g_nb_count[id], nthreads);
+  CtaState& c = g_cta[f.cta];
+  if (c.nb_arrived[id] == 0) {
+    c.nb_count[id] = nthreads;
+    c.nb_and[id] = true;
+  } else if (c.nb_count[id] != nthreads) {
+    std::fprintf(stderr, "emu: named barrier %d used with %d and %d threads\n", id, c.nb_count[id], nthreads);
     ++g_errors;
   }
-  g_nb_and[id] = g_nb_and[id] && pred;
-  ++g_nb_arrived[id];
+  c.nb_and[id] = c.nb_and[id] && pred;
+  ++c.nb_arrived[id];
   f.wait = 3;
   f.bar_id = id;
-  f.gen = g_nb_gen[id];
+  f.gen = c.nb_gen[id];
   swapcontext(&f.ctx, &g_sched);
   return g_fibers[g_cur].result;
 }
 
 inline void syncwarp() {
   Fiber& f = g_fibers[g_cur];
-  const int w = lin_tid() / 32;
+  const int w = warp_slot();
   f.wait = 2;
   f.gen = g_warp_gen[w];
   ++g_warp_arrived[w];
@@ -168,7 +193,7 @@ inline void syncwarp() {
 template <class T>
 inline T shfl_idx(T v, int src) {
   static_assert(sizeof(T) <= 8, "shuffle width");
-  const int t = lin_tid(), w = t / 32, l = t % 32;
+  const int w = warp_slot(), l = lin_tid() % 32;
   std::memcpy(&g_xch[w][l], &v, sizeof(T));
   syncwarp();
   T r;
@@ -182,55 +207,60 @@ inline void trampoline() {
   g_fibers[g_cur].done = true;
 }
 
-inline uint8_t* g_smem_map = nullptr;
-inline size_t g_smem_map_bytes = 0;
+inline uint8_t* g_smem_map[kMaxCluster] = {};
+inline size_t g_smem_map_bytes[kMaxCluster] = {};
 
-inline void set_smem(size_t bytes) {
-  if (g_smem_map) munmap(g_smem_map, g_smem_map_bytes);
+inline void set_smem(int cta, size_t bytes) {
+  if (g_smem_map[cta]) munmap(g_smem_map[cta], g_smem_map_bytes[cta]);
   const size_t n16 = (bytes + 15) & ~size_t(15);
   const size_t body = (n16 + g_page - 1) / g_page * g_page + g_page;
-  g_smem_map_bytes = body + 2 * kGuard;
-  g_smem_map = static_cast<uint8_t*>(
-      mmap(nullptr, g_smem_map_bytes, PROT_READ | PROT_WRITE, MAP_PRIVATE | MAP_ANONYMOUS, -1, 0));
-  mprotect(g_smem_map, kGuard, PROT_NONE);
-  mprotect(g_smem_map + kGuard + body, kGuard, PROT_NONE);
-  g_smem = (g_mode == 0 && !g_smem_start_aligned) ? g_smem_map + kGuard + body - n16 : g_smem_map + kGuard;
+  g_smem_map_bytes[cta] = body + 2 * kGuard;
+  uint8_t* m = static_cast<uint8_t*>(
+      mmap(nullptr, g_smem_map_bytes[cta], PROT_READ | PROT_WRITE, MAP_PRIVATE | MAP_ANONYMOUS, -1, 0));
+  g_smem_map[cta] = m;
+  mprotect(m, kGuard, PROT_NONE);
+  mprotect(m + kGuard + body, kGuard, PROT_NONE);
+  g_smem_cta[cta] = (g_mode == 0 && !g_smem_start_aligned) ? m + kGuard + body - n16 : m + kGuard;
 }
 
-// Runs fn (the kernel call) for every thread of every block.  Returns false on a barrier deadlock or a
-// shuffle with exited lanes.
-inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function<void()>& fn) {
+// Runs fn (the kernel call) for every thread of every block; blocks in clusters of `cluster` CTAs
+// along x run together.  Returns false on a barrier deadlock or a warp-collective with exited lanes.
+inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function<void()>& fn, int cluster = 1) {
   g_grid_dim = grid;
   g_block_dim = block;
   const int nt = static_cast<int>(block.x * block.y * block.z);
   const int nw = (nt + 31) / 32;
-  if (nw > 64) return false;
+  if (nw > 64 || cluster < 1 || cluster > kMaxCluster || grid.x % cluster != 0 || (cluster > 1 && nt % 32 != 0))
+    return false;
   if (smem_bytes > 227 * 1024) {
     std::fprintf(stderr, "emu: dynamic shared memory %zu above the per-block limit\n", smem_bytes);
     return false;
   }
-  set_smem(smem_bytes > 0 ? smem_bytes : 16);
-  while (static_cast<int>(g_stacks.size()) < nt) g_stacks.push_back(static_cast<uint8_t*>(std::malloc(kStack)));
-  g_fibers.assign(nt, Fiber{});
-  g_warp_gen.assign(nw, 0);
-  g_warp_arrived.assign(nw, 0);
+  g_cluster = cluster;
+  for (int c = 0; c < cluster; ++c) set_smem(c, smem_bytes > 0 ? smem_bytes : 16);
+  const int nf = nt * cluster, nwf = nw * cluster;
+  while (static_cast<int>(g_stacks.size()) < nf) g_stacks.push_back(static_cast<uint8_t*>(std::malloc(kStack)));
+  g_fibers.assign(nf, Fiber{});
+  g_warp_gen.assign(nwf, 0);
+  g_warp_arrived.assign(nwf, 0);
   g_body = fn;
   for (unsigned bz = 0; bz < grid.z; ++bz)
     for (unsigned by = 0; by < grid.y; ++by)
-      for (unsigned bx = 0; bx < grid.x; ++bx) {
-        g_bid_cur = make_uint3(bx, by, bz);
-        std::memset(g_smem, 0xFF, smem_bytes);
-        g_block_gen = 0;
-        g_block_arrived = 0;
-        g_block_or = false;
-        for (int i = 0; i < 16; ++i) g_nb_count[i] = g_nb_arrived[i] = 0, g_nb_gen[i] = 0;
-        for (auto& h : g_block_reset) h();
+      for (unsigned bx0 = 0; bx0 < grid.x; bx0 += cluster) {
+        for (int c = 0; c < cluster; ++c) {
+          std::memset(g_smem_cta[c], 0xFF, smem_bytes);
+          g_cta[c] = CtaState{};
+          for (auto& h : g_block_reset) h(c);
+        }
+        g_cl_gen = 0;
+        g_cl_arrived = 0;
         std::fill(g_warp_arrived.begin(), g_warp_arrived.end(), 0);
-        for (int i = 0; i < nt; ++i) {
+        for (int i = 0; i < nf; ++i) {
           Fiber& f = g_fibers[i];
           f.done = false;
           f.wait = 0;
           f.gen = 0;
+          f.cta = i / nt;
           getcontext(&f.ctx);
           f.ctx.uc_stack.ss_sp = g_stacks[i];
           f.ctx.uc_stack.ss_size = kStack;
@@ -239,48 +269,63 @@ inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function
         }
         for (;;) {
           bool progress = false;
-          int alive = 0;
-          std::vector<int> alive_w(nw, 0);
-          for (int i = 0; i < nt; ++i) {
+          int alive_all = 0;
+          std::vector<int> alive_w(nwf, 0), alive_c(cluster, 0);
+          for (int i = 0; i < nf; ++i) {
             Fiber& f = g_fibers[i];
             if (f.done) continue;
-            if (f.wait == 1 && f.gen == g_block_gen) continue;
+            const CtaState& c = g_cta[f.cta];
+            if (f.wait == 1 && f.gen == c.block_gen) continue;
             if (f.wait == 2 && f.gen == g_warp_gen[i / 32]) continue;
-            if (f.wait == 3 && f.gen == g_nb_gen[f.bar_id]) continue;
+            if (f.wait == 3 && f.gen == c.nb_gen[f.bar_id]) continue;
+            if (f.wait == 4 && f.gen == g_cl_gen) continue;
             f.wait = 0;
             g_cur = i;
-            g_tid_cur = make_uint3(i % block.x, (i / block.x) % block.y, i / (block.x * block.y));
+            g_cur_cta = f.cta;
+            g_smem = g_smem_cta[f.cta];
+            const int t = i % nt;
+            g_tid_cur = make_uint3(t % block.x, (t / block.x) % block.y, t / (block.x * block.y));
+            g_bid_cur = make_uint3(bx0 + f.cta, by, bz);
             swapcontext(&g_sched, &f.ctx);
             progress = true;
           }
-          for (int i = 0; i < nt; ++i)
+          for (int i = 0; i < nf; ++i)
             if (!g_fibers[i].done) {
-              ++alive;
+              ++alive_all;
               ++alive_w[i / 32];
+              ++alive_c[i / nt];
             }
-          if (alive == 0) break;
-          if (g_block_arrived > 0 && g_block_arrived == alive) {
-            for (int i = 0; i < nt; ++i)
-              if (!g_fibers[i].done && g_fibers[i].wait == 1) g_fibers[i].result = g_block_or;
-            ++g_block_gen;
-            g_block_arrived = 0;
-            g_block_or = false;
-            progress = true;
-          }
-          for (int id = 0; id < 16; ++id)
-            if (g_nb_arrived[id] > 0 && g_nb_arrived[id] == g_nb_count[id]) {
-              for (int i = 0; i < nt; ++i)
-                if (!g_fibers[i].done && g_fibers[i].wait == 3 && g_fibers[i].bar_id == id &&
-                    g_fibers[i].gen == g_nb_gen[id])
-                  g_fibers[i].result = g_nb_and[id];
-              ++g_nb_gen[id];
-              g_nb_arrived[id] = 0;
+          if (alive_all == 0) break;
+          for (int cc = 0; cc < cluster; ++cc) {
+            CtaState& c = g_cta[cc];
+            if (c.block_arrived > 0 && c.block_arrived == alive_c[cc]) {
+              for (int i = cc * nt; i < (cc + 1) * nt; ++i)
+                if (!g_fibers[i].done && g_fibers[i].wait == 1) g_fibers[i].result = c.block_or;
+              ++c.block_gen;
+              c.block_arrived = 0;
+              c.block_or = false;
               progress = true;
             }
-          for (int w = 0; w < nw; ++w)
+            for (int id = 0; id < 16; ++id)
+              if (c.nb_arrived[id] > 0 && c.nb_arrived[id] == c.nb_count[id]) {
+                for (int i = cc * nt; i < (cc + 1) * nt; ++i)
+                  if (!g_fibers[i].done && g_fibers[i].wait == 3 && g_fibers[i].bar_id == id &&
+                      g_fibers[i].gen == c.nb_gen[id])
+                    g_fibers[i].result = c.nb_and[id];
+                ++c.nb_gen[id];
+                c.nb_arrived[id] = 0;
+                progress = true;
+              }
+          }
+          if (g_cl_arrived > 0 && g_cl_arrived == alive_all) {
+            ++g_cl_gen;
+            g_cl_arrived = 0;
+            progress = true;
+          }
+          for (int w = 0; w < nwf; ++w)
             if (g_warp_arrived[w] > 0 && g_warp_arrived[w] == alive_w[w]) {
-              if (alive_w[w] != std::min(32, nt - 32 * w)) {
-                std::fprintf(stderr, "emu: warp-collective with exited lanes (block %u,%u,%u warp %d)\n", bx, by, bz, w);
+              if (alive_w[w] != std::min(32, nt - 32 * (w % nw))) {
+                std::fprintf(stderr, "emu: warp-collective with exited lanes (block %u,%u,%u warp %d)\n", bx0, by, bz, w);
                 ++g_errors;
               }
               ++g_warp_gen[w];
@@ -288,8 +333,8 @@ inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function
               progress = true;
             }
           if (!progress) {
-            std::fprintf(stderr, "emu: barrier deadlock in block %u,%u,%u (alive %d, at block barrier %d)\n", bx, by,
-                         bz, alive, g_block_arrived);
+            std::fprintf(stderr, "emu: barrier deadlock in cluster at block %u,%u,%u (alive %d)\n", bx0, by, bz,
+                         alive_all);
             ++g_errors;
             return false;
           }
@@ -300,10 +345,12 @@ inline bool launch(dim3 grid, dim3 block, size_t smem_bytes, const std::function
 
 }  // namespace hemu
 
-#define threadIdx (hemu::g_tid_cur)
-#define blockIdx (hemu::g_bid_cur)
-#define gridDim (hemu::g_grid_dim)
-#define blockDim (hemu::g_block_dim)
+// the built-in index variables: references to the running fiber's values (variables, not macros, so
+// that members of the same names, such as cudaLaunchConfig_t::gridDim, stay untouched)
+inline const uint3& threadIdx = hemu::g_tid_cur;
+inline const uint3& blockIdx = hemu::g_bid_cur;
+inline const dim3& gridDim = hemu::g_grid_dim;
+inline const dim3& blockDim = hemu::g_block_dim;
 #define __syncthreads() hemu::syncthreads()
 #define __syncwarp(...) hemu::syncwarp()
 
@@ -320,7 +367,7 @@ inline T atomicAdd(T* p, T v) {
   return o;
 }
 inline bool __all_sync(unsigned, int pred) {
-  const int l = hemu::lin_tid() % 32, w = hemu::lin_tid() / 32;
+  const int l = hemu::lin_tid() % 32, w = hemu::warp_slot();
   hemu::g_xch[w][l] = pred != 0;
   hemu::syncwarp();
   bool r = true;
@@ -329,7 +376,7 @@ inline bool __all_sync(unsigned, int pred) {
   return r;
 }
 inline bool __any_sync(unsigned, int pred) {
-  const int l = hemu::lin_tid() % 32, w = hemu::lin_tid() / 32;
+  const int l = hemu::lin_tid() % 32, w = hemu::warp_slot();
   hemu::g_xch[w][l] = pred != 0;
   hemu::syncwarp();
   bool r = false;
