@@ -73,9 +73,12 @@ def adapt_pair_kernel(s):
 
 def build(out_dir: str, src_root: str = ROOT, mutations=()) -> str:
     """mutations: (file, old text, new text) applied to the copied sources (planted-mistake tests)."""
-    csrc = os.path.join(out_dir, "csrc")
-    shutil.rmtree(csrc, ignore_errors=True)
+    # the repository's layout, so that the API file finds its header by its relative path
+    csrc = os.path.join(out_dir, "global_attention_moe_b200", "csrc")
+    shutil.rmtree(os.path.join(out_dir, "global_attention_moe_b200"), ignore_errors=True)
+    shutil.rmtree(os.path.join(out_dir, "include"), ignore_errors=True)
     shutil.copytree(os.path.join(src_root, "global_attention_moe_b200", "csrc"), csrc)
+    shutil.copytree(os.path.join(src_root, "include"), os.path.join(out_dir, "include"))
     for h in ("sm100.cuh", "cp_async.cuh"):
         shutil.copy(os.path.join(HERE, "device_model", h), os.path.join(csrc, h))
     decls = {"extern __shared__ __align__(1024) uint8_t smem[];": "uint8_t* smem = hemu::g_smem;",
@@ -110,7 +113,7 @@ def build(out_dir: str, src_root: str = ROOT, mutations=()) -> str:
                 '#include "tensormap_host.h"\n' + EXPORTS)
     so = os.path.join(out_dir, "libmimo_attn_host.so")
     cmd = ["g++", "-std=c++20", "-O2", "-fno-strict-aliasing", "-fPIC", "-shared", "-w", "-Wl,-Bsymbolic",
-           "-I/usr/local/cuda/include", "-I" + HERE, "-I" + os.path.join(src_root, "include"), tu, "-o", so]
+           "-I/usr/local/cuda/include", "-I" + HERE, tu, "-o", so]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode:
         raise RuntimeError("host build of the library failed:\n" + r.stderr[-4000:])
