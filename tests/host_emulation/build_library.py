@@ -61,6 +61,12 @@ PAIR_STATEMENTS = [
 ]
 
 
+# The KV-cache kernel's gather4 fetcher keeps its TMA gather instruction in a helper of its own.
+GATHER4_HELPER = ("__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, "
+                  "int32_t r0,\n                                            int32_t r1, int32_t r2, int32_t r3)",
+                  "  tma_gather4_model(dst, map, bar, x, r0, r1, r2, r3);")
+
+
 def adapt_pair_kernel(s):
     for sig, body in PAIR_HELPERS:
         s = _replace_function(s, sig, body)
@@ -96,6 +102,8 @@ def build(out_dir: str, src_root: str = ROOT, mutations=()) -> str:
                 s = s.replace(old, new)
         if name == "attn_fwd_swa2.cuh":
             s = adapt_pair_kernel(s)
+        if name == "attn_decode_tc.cuh" and "void tma_gather4(" in s:
+            s = _replace_function(s, *GATHER4_HELPER)
         if name == "mimo_attn_api.cu":
             s, n = build_host._launches(s)
             assert n >= 16, n

@@ -173,6 +173,32 @@ inline void tma_box_to_smem(void* dst, const CUtensorMap* map, int32_t x, int32_
   }
 }
 
+// tile::gather4: rows r0..r3 of the 64-element box column x land as four consecutive 128-byte rows at
+// dst (swizzled by address; rows outside the tensor as zeros); their bytes complete on bar.
+inline void tma_gather4_model(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t r0, int32_t r1,
+                              int32_t r2, int32_t r3) {
+  const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
+  const int32_t rows[4] = {r0, r1, r2, r3};
+  uint8_t* d = static_cast<uint8_t*>(dst);
+  if (t->box_rows != 1 || t->box_inner * t->elem != 128 || (x * t->elem) % 16 != 0) {
+    std::fprintf(stderr, "tcsim: gather4 needs a {64, 1} box and a 16-byte-aligned x\n");
+    ++hemu::g_errors;
+  }
+  for (int i = 0; i < 4; ++i) {
+    uint8_t row[128];
+    for (uint32_t e = 0; e < t->box_inner; ++e) {
+      const int64_t gx = static_cast<int64_t>(x) + e;
+      if (rows[i] < 0 || rows[i] >= static_cast<int64_t>(t->rows) || gx >= static_cast<int64_t>(t->inner))
+        std::memset(row + e * t->elem, 0, t->elem);
+      else
+        std::memcpy(row + e * t->elem, t->base + rows[i] * t->stride + gx * t->elem, t->elem);
+    }
+    const uint32_t a = smem_u32(d + i * 128);
+    for (uint32_t c = 0; c < 8; ++c) std::memcpy(d + i * 128 + ((c ^ ((a >> 7) & 7u)) << 4), row + c * 16, 16);
+  }
+  mbar_complete_tx(bar, 4 * 128);
+}
+
 inline void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y, uint64_t) {
   tma_load_2d(dst, map, bar, x, y);
 }
