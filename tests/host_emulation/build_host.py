@@ -80,6 +80,12 @@ HOST_FORMS = [
 ]
 
 
+# forms that only some versions of the host code contain
+OPTIONAL_HOST_FORMS = [
+    (r"cudaMemsetAsync\((\w+), 0, ([^,]+), stream\)", r"(std::memset(\1, 0, \2), cudaSuccess)"),
+]
+
+
 def generate() -> str:
     api = _read("mimo_attn_api.cu")
     host = "\n".join([_function(api, "int launch_bwd("), _function(api, "int launch_decode(")] +
@@ -87,8 +93,10 @@ def generate() -> str:
     for pat, new in HOST_FORMS:
         host, n = re.subn(pat, new, host)
         assert n >= 1, f"host form not found: {pat}"
+    for pat, new in OPTIONAL_HOST_FORMS:
+        host = re.sub(pat, new, host)
     host, n = _launches(host)
-    assert n == 9, f"expected 9 launches, found {n}"
+    assert n >= 9, f"expected at least 9 launches, found {n}"
     rope = _read("rope_smem.cuh")
     rope = rope[rope.index("constexpr double kTwoPi"):rope.index("// Rotates chunk pair")]
     sm100 = _read("sm100.cuh")
@@ -97,13 +105,18 @@ def generate() -> str:
     validate = api[api.index("bool aligned16(const void* p)"):api.index("void fill_params(")]
     validate += api[api.index("// Query rows per KV head (q_len x Hq/Hkv)"):api.index("int launch_decode(")]
     lines = [ln for ln in api.splitlines() if ln.startswith(("constexpr uint64_t kDefaultWaitLimitNs",
-                                                             "std::atomic<int> g_decode_choice", "size_t align256("))]
-    assert len(lines) == 3, lines
+                                                             "std::atomic<int> g_decode_choice", "size_t align256(",
+                                                             "std::atomic<int> g_bwd_choice"))]
+    assert len(lines) >= 3, lines
     tc = _read("attn_decode_tc.cuh")
     tc_consts = [re.search(rf"constexpr (\w+) {n} = [^;]+;", tc).group(0) for n in ("kThreads", "kChunk")]
     tc_stub = ("namespace dtc {\n" + "\n".join(tc_consts) + "\nconstexpr uint32_t kSmemBytes = 0;\n}\n"
                "template <class... A> void attn_decode_tc_kernel(const A&...) { ++hemu::g_errors; }\n"
                "template <class... A> bool encode_2d(A...) { return false; }  // tensor maps: device path only\n")
+    if "attn_bwd_tc_kernel" in api:  # the tensor-core backward: device path only (the device model runs it)
+        tc_stub += ("namespace bwdtc {\nconstexpr int kThreads = 128;\nconstexpr uint32_t kSmemBytes = 0;\n}\n"
+                    "template <class... A> void attn_bwd_tc_kernel(const A&...) { ++hemu::g_errors; }\n"
+                    "template <class... A> void bwdtc_prep_kernel(const A&...) { ++hemu::g_errors; }\n")
     wrappers = []
     for e in ENTRY_POINTS:
         sig = _function(api, f"int {e}(")
