@@ -141,9 +141,18 @@ bool set_smem_attributes() {
          cudaFuncSetAttribute(dec::attn_decode_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               dec::kSmemBytes) == cudaSuccess &&
          cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              dtc::kSmemBytes) == cudaSuccess &&
-         cudaFuncSetAttribute(bwd::bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              bwd::kSmemBytes) == cudaSuccess;
+                              dtc::kSmemBytes) == cudaSuccess;
+}
+
+// The backward's shared-memory limit, raised on its first call on each device (so that a failure here
+// concerns the backward only).
+bool bwd_attributes_ready(int dev) {
+  static std::atomic<int> state[64];  // 0 unknown, 1 ready, -1 failed
+  if (dev < 0 || dev >= 64) return false;
+  if (state[dev].load() == 0)
+    state[dev].store(cudaFuncSetAttribute(bwd::bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          bwd::kSmemBytes) == cudaSuccess ? 1 : -1);
+  return state[dev].load() == 1;
 }
 
 std::atomic<int> g_decode_choice{MIMO_DECODE_AUTO};
@@ -539,6 +548,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const float* sink, c
   if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
   DeviceInfo* info = device_info(dev);
   if (!info || !info->kernels_ready || !info->pool) return MIMO_ERR_CUDA;
+  if (!bwd_attributes_ready(dev)) return MIMO_ERR_CUDA;
   bwd::BwdParams P;
   std::memset(&P, 0, sizeof P);
   P.q = static_cast<const uint16_t*>(q);

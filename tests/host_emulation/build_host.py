@@ -83,6 +83,7 @@ HOST_FORMS = [
 # forms that only some versions of the host code contain
 OPTIONAL_HOST_FORMS = [
     (r"cudaMemsetAsync\((\w+), 0, ([^,]+), stream\)", r"(std::memset(\1, 0, \2), cudaSuccess)"),
+    (r"  if \(!bwd_attributes_ready\(dev\)\) return MIMO_ERR_CUDA;\n", ""),
 ]
 
 
