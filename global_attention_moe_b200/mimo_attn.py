@@ -176,7 +176,10 @@ def linear_proj(x, w, out=None, stream=None):
     [N, K] (a Linear weight) -> bf16 y [T, N] (cuBLAS, FP32 accumulation)."""
     import torch
     T = x.shape[0]
-    x2 = x.reshape(T, -1)
+    feats = 1
+    for d in x.shape[1:]:
+        feats *= int(d)
+    x2 = x.reshape(T, feats)  # explicit: reshape(T, -1) is ambiguous for zero tokens
     N, K = w.shape
     if x2.shape[1] != K:
         raise ValueError(f"x has {x2.shape[1]} features per token, w expects {K}")

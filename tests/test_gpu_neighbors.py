@@ -93,3 +93,28 @@ def test_linear_proj(T, hq, N):
     ref = NB.linear_proj(x.reshape(T, K), w)
     assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 2e-3
     assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-3 * np.sqrt(np.mean(ref ** 2)))
+
+
+def test_route_exact_ties_take_lower_experts():
+    """Rows of equal logits with a zero bias tie on every key: the choice is experts 0..k-1, in order,
+    and the normalised weights are all 1/k."""
+    from global_attention_moe_b200 import mimo_attn as M
+    logits = np.full((5, 256), 0.25, dtype=np.float32)
+    ids, w = M.moe_route(torch.from_numpy(logits).cuda(), torch.zeros(256).cuda(), 8)
+    assert M.check() == M.OK
+    assert np.array_equal(ids.cpu().numpy(), np.tile(np.arange(8, dtype=np.int32), (5, 1)))
+    assert np.allclose(w.cpu().numpy(), 1.0 / 8, rtol=0, atol=1e-7)
+
+
+def test_empty_inputs():
+    """Zero tokens / rows: nothing to launch, empty results."""
+    from global_attention_moe_b200 import mimo_attn as M
+    ids, w = M.moe_route(torch.zeros((0, 256)).cuda(), torch.zeros(256).cuda(), 8)
+    assert tuple(ids.shape) == (0, 8) and tuple(w.shape) == (0, 8)
+    q, k, v = M.qkv_split(torch.zeros((0, 8 * (8 * 192 + 320)), dtype=torch.bfloat16).cuda(), 64, 8)
+    assert tuple(q.shape) == (0, 64, 192) and tuple(k.shape) == (0, 8, 192) and tuple(v.shape) == (0, 8, 128)
+    out = M.fp8_dequant_blockwise(torch.zeros((0, 512), dtype=torch.uint8).cuda(), torch.ones((0, 4)).cuda())
+    assert tuple(out.shape) == (0, 512)
+    y = M.linear_proj(torch.zeros((0, 8, 128), dtype=torch.bfloat16).cuda(), torch.zeros((64, 1024), dtype=torch.bfloat16).cuda())
+    assert tuple(y.shape) == (0, 64)
+    assert M.check() == M.OK
