@@ -123,6 +123,15 @@ CASES = {
     "decode_tensor": lambda H: decode(H, [5, 129, 300, 64], [1, 8, 3, 8], 8, 2, W.LAYER_SWA, 128, 1e4, True, 71),
     "decode_tensor_tiles_swa": lambda H: decode(H, [600, 90], [300, 20], 8, 2, W.LAYER_SWA, 128, 1e4, True, 72),
     "decode_tensor_tiles_global": lambda H: decode(H, [200, 50], [36, 50], 8, 1, W.LAYER_GLOBAL, -1, 1e7, False, 73),
+    # tile edges on both kernels: exactly 128 rows; 129 rows (a one-row tile); 6 query heads per KV head
+    # (a token's heads straddle two tiles); window 0 over a whole prompt
+    "decode_tile_edges": lambda H: [decode(H, kv, ql, hq, hkv, layer, win, base, sink, seed, kernel=k)
+                                    for k in ("tensor", "cuda_cores")
+                                    for kv, ql, hq, hkv, layer, win, base, sink, seed in (
+                                        ([300, 40], [16, 16], 8, 1, W.LAYER_SWA, 128, 1e4, True, 81),
+                                        ([300, 129], [43, 43], 6, 2, W.LAYER_SWA, 128, 1e4, True, 82),
+                                        ([500, 200], [30, 25], 6, 1, W.LAYER_GLOBAL, -1, 1e7, False, 83),
+                                        ([260, 700], [260, 100], 12, 2, W.LAYER_SWA, 0, 1e4, False, 84))],
 }
 
 if __name__ == "__main__":
