@@ -7,8 +7,9 @@
 //             (16-byte chunk c of the 128-byte row at smem address a goes to chunk c ^ ((a >> 7) & 7)),
 //             zero fill outside the tensor, completion as transaction bytes.
 //   tcgen05:  TMEM 128 lanes x 512 columns of 32 bits per block; MMAs are queued by the issuing thread
-//             and executed when it commits (then the commit arrives), so a read of an operand or of
-//             the accumulator before the commit is visible; SS (A K- or MN-major) and TS forms,
+//             and run only when a thread first polls a barrier that their commit arrives on (the
+//             latest moment the hardware could finish them), so an operand overwritten, or an
+//             accumulator read, before that wait shows; SS (A K- or MN-major) and TS forms,
 //             kind::f16, M = 128; the
 //             16-term dot product of one instruction in FP64, added once to the FP32 accumulator.
 //   tcgen05.ld/st 32x32b: warp w reaches lanes 32 (w % 4) .. +31 only (checked).
@@ -111,7 +112,9 @@ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
 }
 inline void mbar_arrive(uint64_t* bar) { mbar_arrive_at(bar); }
 
+inline void mma_flush_for(int cta, uint32_t off);
 inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  mma_flush_for(hemu::g_cur_cta, smem_u32(bar));
   if ((mbar_state(bar).phase & 1u) != (parity & 1u)) return true;
   hemu::yield();
   return (mbar_state(bar).phase & 1u) != (parity & 1u);
@@ -337,17 +340,41 @@ inline void mma_execute(const MmaOp& op) {
   }
 }
 
+// A commit does not run its MMAs: they run, in issue order, when a thread first polls a barrier that
+// one of the commits arrives on (the latest moment the hardware could finish them), or when the
+// cluster's CTAs have all exited.  So an operand overwritten, or an accumulator read, before the
+// commit's barrier has been waited on shows in the results.
+struct PendingCommit {
+  std::vector<MmaOp> ops;
+  std::vector<std::pair<int, uint32_t>> targets;  // (CTA, barrier offset) arrivals
+};
+inline std::vector<PendingCommit> g_pending;
+
+inline void mma_flush_upto(size_t n) {  // runs the first n pending commits
+  for (size_t i = 0; i < n; ++i) {
+    for (const MmaOp& op : g_pending[i].ops) mma_execute(op);
+    for (const auto& t : g_pending[i].targets) mbar_arrive_cta(t.first, t.second);
+  }
+  g_pending.erase(g_pending.begin(), g_pending.begin() + static_cast<long>(n));
+}
+inline void mma_flush_for(int cta, uint32_t off) {
+  size_t last = 0;
+  for (size_t i = 0; i < g_pending.size(); ++i)
+    for (const auto& t : g_pending[i].targets)
+      if (t.first == cta && t.second == off) last = i + 1;
+  if (last) mma_flush_upto(last);
+}
 inline void tc_commit(uint64_t* bar) {
-  for (const MmaOp& op : g_mma_queue) mma_execute(op);
+  g_pending.push_back({std::move(g_mma_queue), {{hemu::g_cur_cta, smem_u32(bar)}}});
   g_mma_queue.clear();
-  mbar_arrive_at(bar);
 }
 // Pair commit with multicast: arrives on the barrier at the same offset in every CTA of the mask.
 inline void tc_commit_multicast(uint64_t* bar, uint16_t mask) {
-  for (const MmaOp& op : g_mma_queue) mma_execute(op);
+  PendingCommit pc{std::move(g_mma_queue), {}};
   g_mma_queue.clear();
   for (int c = 0; c < hemu::g_cluster; ++c)
-    if ((mask >> c) & 1u) mbar_arrive_cta(c, smem_u32(bar));
+    if ((mask >> c) & 1u) pc.targets.push_back({c, smem_u32(bar)});
+  g_pending.push_back(std::move(pc));
 }
 
 __host__ __device__ constexpr uint32_t make_idesc_f32acc(uint32_t ab_bf16, uint32_t b_mn_major, uint32_t M,
@@ -456,6 +483,7 @@ inline bool g_tc_reset_registered = [] {
     g_mbars[c].clear();
     g_tmem_next[c] = 0;
     g_mma_queue.clear();
+    g_pending.clear();
     std::memset(g_tmem_all[c], 0xFF, sizeof(g_tmem_all[c]));
   });
   return true;

@@ -3,7 +3,8 @@ the fiber runtime with a device model of the tcgen05 / TMA / mbarrier wrappers
 (tests/host_emulation/device_model), and the results are compared with the oracle at the forward's
 tolerances.  The model reproduces the errors measured on a B200 for the tensor-core forward kernels
 on the small sliding-window config (max-abs 4.4e-3 simple, 7.3e-3 pipelined), i.e. the same
-rounding points.  Planted mistakes in the kernels' operand addressing and row tiling are caught."""
+rounding points.  Planted mistakes in the kernels' operand addressing, row tiling and MMA completion
+waits are caught (the device model runs an MMA only when its commit's barrier is first waited on)."""
 import os
 import subprocess
 import sys
@@ -41,6 +42,11 @@ PLANTED = [
      "v_lo + kk * (2048 >> 4)", "v_lo + kk * (1024 >> 4)", "fwd_tiny_pipelined"),
     ("KV-cache row tiles all start at row 0", "attn_decode_tc.cuh", "w.row0 = 128 * qt;", "w.row0 = 0;",
      "decode_tensor_tiles_swa"),
+    ("scores read from TMEM without waiting for their MMAs", "attn_fwd_simple.cuh",
+     "      fail = !mbar_wait(&bars[2], mma_phase, P.wait_limit_ns);\n      mma_phase ^= 1;\n"
+     "      if (__syncthreads_or(fail)) { fail = true; break; }\n      tc_fence_after_sync();\n\n      uint32_t s[4][32];",
+     "      mma_phase ^= 1;\n      if (__syncthreads_or(fail)) { fail = true; break; }\n      tc_fence_after_sync();\n\n"
+     "      uint32_t s[4][32];", "fwd_tiny_simple"),
 ]
 
 
