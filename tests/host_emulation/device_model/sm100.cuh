@@ -12,7 +12,8 @@
 //             accumulator read, before that wait shows; SS (A K- or MN-major) and TS forms,
 //             kind::f16, M = 128; the
 //             16-term dot product of one instruction in FP64, added once to the FP32 accumulator.
-//   tcgen05.ld/st 32x32b: warp w reaches lanes 32 (w % 4) .. +31 only (checked).
+//   tcgen05.ld/st 32x32b: warp-collective (a warp barrier); warp w reaches lanes 32 (w % 4) .. +31
+//             only (checked).
 #pragma once
 
 #include <cuda.h>
@@ -426,7 +427,10 @@ inline void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t 
 
 inline uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col) { return base + (lane << 16) + col; }
 
+// tcgen05.ld / st are .sync.aligned: all 32 lanes of the warp execute each one together (a warp
+// barrier here, which reports lanes that have exited).
 inline void tmem_lane_check(uint32_t taddr) {
+  hemu::syncwarp();
   const uint32_t w = hemu::lin_tid() / 32;
   if ((taddr >> 16) != 32 * (w % 4)) {
     std::fprintf(stderr, "tcsim: warp %u addresses TMEM lanes from %u\n", w, taddr >> 16);

@@ -111,6 +111,24 @@ def decode(H, kv, ql, hq, hkv, layer, window, base, has_sink, seed, kernel="tens
     check(out, lse, *decode_reference(x, window if layer == W.LAYER_SWA else -1, base))
 
 
+def fwd_timeout(H, kernel):
+    """With a wait limit of zero the waits on other roles give up: the kernel must record a timeout and
+    leave without a deadlock or a warp-collective instruction with exited lanes."""
+    w = W.tiny_swa()
+    x = W.make_inputs(w)
+    T, hq = w.total_tokens, w.num_q_heads
+    d = Dims(w.num_seqs, T, w.max_seqlen, hq, w.num_kv_heads, 192, 128)
+    assert H.L.mimo_attn_set_kernel(KERNEL[kernel]) == 0
+    po, pl = H.empty(T * hq * 128 * 2), H.empty(hq * T * 4)
+    st = H.L.mimo_attn_fwd(H.put(x.q), H.put(x.k), H.put(x.v), H.put(x.sink), H.put(x.cu_seqlens), C.byref(d),
+                           w.layer_kind, w.window, w.rope_base, 64, 0.707, po, pl, None)
+    H.L.mimo_attn_set_kernel(0)
+    while H.live:
+        H.L.hemu_free(H.live.pop())
+    assert st == 0 and H.L.hemu_errors() == 0, "deadlock or warp-collective with exited lanes"
+    assert H.L.mimo_attn_check(None) == 4, "timeout not reported"  # MIMO_ERR_TIMEOUT
+
+
 CASES = {
     # the three forward kernels on the small sliding-window config (T = 512, 4 query heads, 1 KV head)
     "fwd_tiny_simple": lambda H: fwd(H, W.tiny_swa(), "simple"),
@@ -132,7 +150,11 @@ CASES = {
                                         ([300, 129], [43, 43], 6, 2, W.LAYER_SWA, 128, 1e4, True, 82),
                                         ([500, 200], [30, 25], 6, 1, W.LAYER_GLOBAL, -1, 1e7, False, 83),
                                         ([260, 700], [260, 100], 12, 2, W.LAYER_SWA, 0, 1e4, False, 84))],
+    # only for a build whose wait limit is zero
+    "fwd_timeout_pipelined": lambda H: fwd_timeout(H, "pipelined"),
+    "fwd_timeout_window": lambda H: fwd_timeout(H, "window"),
 }
+TIMEOUT_CASES = ("fwd_timeout_pipelined", "fwd_timeout_window")
 
 if __name__ == "__main__":
     H = Lib(sys.argv[1])

@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 EMU = os.path.join(HERE, "host_emulation")
 sys.path.insert(0, EMU)
 import build_library  # noqa: E402
-from library_cases import CASES  # noqa: E402
+from library_cases import CASES, TIMEOUT_CASES  # noqa: E402
 
 
 def run_cases(lib, names):
@@ -30,7 +30,17 @@ def host_library(tmp_path_factory):
 
 
 def test_library_matches_oracle(host_library):
-    rc, log = run_cases(host_library, list(CASES))
+    rc, log = run_cases(host_library, [c for c in CASES if c not in TIMEOUT_CASES])
+    assert rc == 0, log
+
+
+def test_timed_out_waits_end_cleanly(tmp_path):
+    """A build whose bounded waits have a zero limit: the forward kernels' roles give up on each other,
+    record a timeout and leave without a deadlock or a warp-collective instruction with exited lanes."""
+    lib = build_library.build(str(tmp_path), mutations=[(
+        "mimo_attn_api.cu", "constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;",
+        "constexpr uint64_t kDefaultWaitLimitNs = 0ull;")])
+    rc, log = run_cases(lib, list(TIMEOUT_CASES))
     assert rc == 0, log
 
 
