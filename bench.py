@@ -62,7 +62,7 @@ def parse():
                     help="time the KV-cache path (64 requests x 8 new tokens) instead of the forward")
     ap.add_argument("--decode-requests", type=int, default=64,
                     help="requests in the KV-cache batch (fewer: a smaller case for profiling)")
-    ap.add_argument("--step", choices=("bwd", "dequant", "split", "proj", "route"), default=None,
+    ap.add_argument("--step", choices=("bwd", "bwd_tc", "dequant", "split", "proj", "route"), default=None,
                     help="time a step beside the forward instead (backward, FP8 dequant, QKV split, output "
                          "projection, MoE routing)")
     ap.add_argument("--decode-contiguous", action="store_true",
@@ -578,7 +578,7 @@ def run_decode(args):
     return 0
 
 
-STEP_KINDS = ("bwd", "dequant", "split", "proj", "route")
+STEP_KINDS = ("bwd", "bwd_tc", "dequant", "split", "proj", "route")
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core FP32 FMA peak at the maximum SM clock
 
 
@@ -594,6 +594,9 @@ def run_step(args):
     rng = np.random.default_rng(0)
     peaks, peak_src = load_peaks()
     kind = args.step
+    if kind == "bwd_tc":
+        mimo_attn.set_bwd_kernel(mimo_attn.BWD_TENSOR)
+        kind = "bwd"
     if kind == "bwd":
         w = W.WORKLOADS["swa4096"]()
         x = W.make_inputs(w)

@@ -23,6 +23,7 @@
 #include "attn_decode.cuh"
 #include "attn_decode_tc.cuh"
 #include "attn_bwd_simple.cuh"
+#include "attn_bwd_tc.cuh"
 #include "neighbors.cuh"
 #include "rope_k_prepass.cuh"
 #include "params.cuh"
@@ -151,11 +152,16 @@ bool bwd_attributes_ready(int dev) {
   if (dev < 0 || dev >= 64) return false;
   if (state[dev].load() == 0)
     state[dev].store(cudaFuncSetAttribute(bwd::bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          bwd::kSmemBytes) == cudaSuccess ? 1 : -1);
+                                          bwd::kSmemBytes) == cudaSuccess &&
+                             cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  bwdtc::kSmemBytes) == cudaSuccess
+                         ? 1
+                         : -1);
   return state[dev].load() == 1;
 }
 
 std::atomic<int> g_decode_choice{MIMO_DECODE_AUTO};
+std::atomic<int> g_bwd_choice{0};  // 0 auto (CUDA cores), 1 CUDA cores, 2 tensor cores
 
 // Persistent grid of the two-head kernels: one CTA per SM, at most one per unit.
 int persistent_grid(const FwdParams& P, int sms) {
@@ -580,6 +586,29 @@ int launch_bwd(const void* q, const void* k, const void* v, const float* sink, c
   if (cudaMallocFromPoolAsync(&scratch, n_d * sizeof(float), info->pool, stream) != cudaSuccess) return MIMO_ERR_CUDA;
   P.D = static_cast<float*>(scratch);
   int st = MIMO_OK;
+  if (g_bwd_choice.load() == 2) {  // tensor cores: dq / dk / dv / dsink accumulate with atomics
+    const size_t T = (size_t)d->total_tokens;
+    CUtensorMap tq, tk, tv, to;
+    if (cudaMemsetAsync(dq, 0, T * P.hq * kHeadDimQK * 4, stream) != cudaSuccess ||
+        cudaMemsetAsync(dk, 0, T * P.hkv * kHeadDimQK * 4, stream) != cudaSuccess ||
+        cudaMemsetAsync(dv, 0, T * P.hkv * kHeadDimV * 4, stream) != cudaSuccess ||
+        (dsink && cudaMemsetAsync(dsink, 0, P.hq * 4, stream) != cudaSuccess) ||
+        !encode_2d(&tq, q, (uint64_t)P.hq * kHeadDimQK, T) || !encode_2d(&tk, k, (uint64_t)P.hkv * kHeadDimQK, T) ||
+        !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, T) || !encode_2d(&to, dout, (uint64_t)P.hq * kHeadDimV, T)) {
+      st = MIMO_ERR_CUDA;
+    } else {
+      bwdtc_prep_kernel<<<info->sms * 8, 256, 0, stream>>>(P);
+      if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+      if (st == MIMO_OK && d->max_seqlen > 0) {
+        dim3 grid((unsigned)((d->max_seqlen + 127) / 128), (unsigned)d->num_seqs, (unsigned)d->num_q_heads);
+        attn_bwd_tc_kernel<<<grid, bwdtc::kThreads, bwdtc::kSmemBytes, stream>>>(tq, tk, tv, to, P,
+                                                                                 kDefaultWaitLimitNs);
+        if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
+      }
+    }
+    if (cudaFreeAsync(scratch, stream) != cudaSuccess) st = MIMO_ERR_CUDA;
+    return st;
+  }
   bwd::bwd_prep_kernel<<<info->sms * 8, bwd::kThreads, 0, stream>>>(P);
   if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
   if (st == MIMO_OK && d->max_seqlen > 0) {
@@ -858,6 +887,12 @@ int mimo_attn_fwd_noalloc(const void* q, const void* k, const void* v, const flo
 }
 
 size_t mimo_attn_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+int mimo_attn_set_bwd_kernel(int choice) {
+  if (choice < 0 || choice > 2) return MIMO_ERR_INVALID_ARG;
+  g_bwd_choice.store(choice);
+  return MIMO_OK;
+}
 
 int mimo_attn_set_decode_kernel(int choice) {
   if (choice != MIMO_DECODE_AUTO && choice != MIMO_DECODE_CUDA_CORES && choice != MIMO_DECODE_TENSOR)

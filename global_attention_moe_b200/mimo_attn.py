@@ -23,7 +23,7 @@ SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host
            "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_profile_start",
            "mimo_attn_profile_stop", "mimo_attn_decode", "mimo_attn_set_decode_kernel", "mimo_attn_version",
            "mimo_attn_bwd", "mimo_fp8_dequant_blockwise", "mimo_qkv_split", "mimo_moe_route",
-           "mimo_linear_proj")
+           "mimo_linear_proj", "mimo_attn_set_bwd_kernel")
 KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED, KERNEL_WINDOW = 0, 1, 2, 3
 DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR = 0, 1, 2
 
@@ -84,6 +84,8 @@ def _load():
     lib.mimo_fp8_dequant_blockwise.argtypes = [P, P, L, L, I, I, P, P]
     lib.mimo_qkv_split.restype = I
     lib.mimo_qkv_split.argtypes = [P, L, I, I, P, P, P, P]
+    lib.mimo_attn_set_bwd_kernel.restype = I
+    lib.mimo_attn_set_bwd_kernel.argtypes = [I]
     lib.mimo_linear_proj.restype = I
     lib.mimo_linear_proj.argtypes = [P, P, L, L, L, P, P]
     lib.mimo_moe_route.restype = I
@@ -169,6 +171,15 @@ def qkv_split(fused, num_q_heads, num_kv_heads, stream=None):
     if st != OK:
         raise MimoAttnError(st, "mimo_qkv_split")
     return q, k, v
+
+
+BWD_AUTO, BWD_CUDA_CORES, BWD_TENSOR = 0, 1, 2
+
+
+def set_bwd_kernel(choice: int) -> None:
+    st = LIB.mimo_attn_set_bwd_kernel(int(choice))
+    if st != OK:
+        raise MimoAttnError(st, "mimo_attn_set_bwd_kernel")
 
 
 def linear_proj(x, w, out=None, stream=None):

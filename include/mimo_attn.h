@@ -285,6 +285,10 @@ MIMO_API int mimo_attn_decode(const void* q, const void* k_cache, const void* v_
 typedef enum { MIMO_DECODE_AUTO = 0, MIMO_DECODE_CUDA_CORES = 1, MIMO_DECODE_TENSOR = 2 } mimo_decode_choice;
 MIMO_API int mimo_attn_set_decode_kernel(int choice);
 
+/* Kernel of mimo_attn_bwd: 0 automatic (FP32 CUDA cores), 1 FP32 CUDA cores, 2 tensor cores (BF16
+ * operands: the rotated Q / K dims, P and dS each rounded once to BF16).  Process-wide. */
+MIMO_API int mimo_attn_set_bwd_kernel(int choice);
+
 /*
  * Backward of mimo_attn_fwd (miles PR #3648 trains this layer; the LSE with the
  * sink included is the convention it needs).  Inputs as mimo_attn_fwd, plus the

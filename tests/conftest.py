@@ -20,7 +20,7 @@ def pytest_configure(config):
 # keep the older suites from running (and being reported).  Modules not listed (CPU tests) come
 # first, in their own order.
 _GPU_MODULE_ORDER = ("test_gpu_parity.py", "test_gpu_decode.py", "test_zz_no_alloc.py", "test_gpu_decode_tiles.py",
-                     "test_gpu_neighbors.py", "test_gpu_bwd.py")
+                     "test_gpu_neighbors.py", "test_gpu_bwd.py", "test_gpu_bwd_tc.py")
 
 
 def pytest_collection_modifyitems(session, config, items):

@@ -43,6 +43,8 @@ class Lib:
         L.mimo_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, C.POINTER(DecodeDims), C.c_int, C.c_int,
                                        C.c_double, C.c_int, C.c_float, vp, vp, vp]
         L.mimo_attn_check.argtypes = [vp]
+        L.mimo_attn_bwd.argtypes = [vp, vp, vp, vp, vp, C.POINTER(Dims), C.c_int, C.c_int, C.c_double, C.c_int,
+                                    C.c_float, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         self.live = []
 
     def put(self, a):
@@ -111,6 +113,47 @@ def decode(H, kv, ql, hq, hkv, layer, window, base, has_sink, seed, kernel="tens
     check(out, lse, *decode_reference(x, window if layer == W.LAYER_SWA else -1, base))
 
 
+def f64_to_bf16_bits(x):
+    """Round-to-nearest-even of FP64 values to BF16 (one rounding; finite values in FP32 range)."""
+    b = np.asarray(x, dtype=np.float64).view(np.uint64)
+    lsb = (b >> np.uint64(45)) & np.uint64(1)
+    r = (b + np.uint64((1 << 44) - 1) + lsb) & ~np.uint64((1 << 45) - 1)
+    return (r.view(np.float64).astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def bwd(H, lens, hq, hkv, layer, window, base, has_sink, seed, kernel, tol):
+    """The backward against the oracle's, with dLSE shifted by -dO . (out_stored - out) (the kernels form
+    D from the stored BF16 out; the gradients are linear in dLSE)."""
+    rng = np.random.default_rng(seed)
+    T = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    q = synth.f32_to_bf16_bits(rng.standard_normal((T, hq, 192)).astype(np.float32))
+    k = synth.f32_to_bf16_bits(rng.standard_normal((T, hkv, 192)).astype(np.float32))
+    v = synth.f32_to_bf16_bits(rng.standard_normal((T, hkv, 128)).astype(np.float32))
+    sink = rng.standard_normal(hq).astype(np.float32) if has_sink else None
+    go = synth.f32_to_bf16_bits(rng.standard_normal((T, hq, 128)).astype(np.float32))
+    gl = (rng.standard_normal((hq, T)) * 0.3).astype(np.float32)
+    w = window if layer == W.LAYER_SWA else -1
+    out, lse = oracle.attn_fwd(q, k, v, sink, cu, w, base)
+    out_b = f64_to_bf16_bits(out)
+    d = Dims(len(lens), T, max(lens), hq, hkv, 192, 128)
+    shapes = ((T, hq, 192), (T, hkv, 192), (T, hkv, 128), (hq,))
+    ptrs = [H.empty(int(np.prod(s)) * 4) for s in shapes[:3]] + [H.empty(hq * 4) if has_sink else None]
+    assert H.L.mimo_attn_set_bwd_kernel({"cuda_cores": 1, "tensor": 2}[kernel]) == 0
+    st = H.L.mimo_attn_bwd(H.put(q), H.put(k), H.put(v), H.put(sink), H.put(cu), C.byref(d), layer, window, base, 64,
+                           0.707, H.put(out_b), H.put(lse.astype(np.float32)), H.put(go), H.put(gl), *ptrs, None)
+    got = [None if p is None else H.get(p, s, np.float32) for p, s in zip(ptrs, shapes)]
+    H.L.mimo_attn_set_bwd_kernel(0)
+    H.finish(st)
+    go64 = synth.bf16_bits_to_f32(go).astype(np.float64)
+    shift = np.einsum("thd,thd->ht", go64, synth.bf16_bits_to_f32(out_b).astype(np.float64) - out)
+    ref = oracle.attn_bwd(q, k, v, sink, cu, w, base, 64, 0.707, go64, gl.astype(np.float64) - shift)
+    for name, a, r in zip(("dq", "dk", "dv", "dsink"), got, ref):
+        if r is not None:
+            rel = np.linalg.norm(a.astype(np.float64) - r) / np.linalg.norm(r)
+            assert rel <= tol, f"{kernel} {name}: rel-L2 {rel:.2e}"
+
+
 def fwd_timeout(H, kernel):
     """With a wait limit of zero the waits on other roles give up: the kernel must record a timeout and
     leave without a deadlock or a warp-collective instruction with exited lanes."""
@@ -150,6 +193,11 @@ CASES = {
                                         ([300, 129], [43, 43], 6, 2, W.LAYER_SWA, 128, 1e4, True, 82),
                                         ([500, 200], [30, 25], 6, 1, W.LAYER_GLOBAL, -1, 1e7, False, 83),
                                         ([260, 700], [260, 100], 12, 2, W.LAYER_SWA, 0, 1e4, False, 84))],
+    # the backward on the tensor cores (BF16 operands: 1e-2) and on the CUDA cores (FP32: 1e-4)
+    "bwd_tensor": lambda H: [bwd(H, *c, "tensor", 1e-2) for c in (
+        ([300, 129, 17, 1], 8, 2, W.LAYER_SWA, 128, 1e4, True, 41), ([200, 70], 4, 2, W.LAYER_SWA, 0, 1e4, False, 42),
+        ([333, 64, 5], 8, 2, W.LAYER_GLOBAL, -1, 1e7, False, 43))],
+    "bwd_cuda_cores": lambda H: bwd(H, [300, 129, 17, 1], 8, 2, W.LAYER_SWA, 128, 1e4, True, 41, "cuda_cores", 1e-4),
     # only for a build whose wait limit is zero
     "fwd_timeout_pipelined": lambda H: fwd_timeout(H, "pipelined"),
     "fwd_timeout_window": lambda H: fwd_timeout(H, "window"),

@@ -52,6 +52,9 @@ PLANTED = [
      "v_lo + kk * (2048 >> 4)", "v_lo + kk * (1024 >> 4)", "fwd_tiny_pipelined"),
     ("KV-cache row tiles all start at row 0", "attn_decode_tc.cuh", "w.row0 = 128 * qt;", "w.row0 = 0;",
      "decode_tensor_tiles_swa"),
+    ("backward dQ reads dS without its MN-major flag", "attn_bwd_tc.cuh",
+     "kIdescDQ = make_idesc_f32acc(1, 1, 128, 192) | (1u << 15);", "kIdescDQ = make_idesc_f32acc(1, 1, 128, 192);",
+     "bwd_tensor"),
     ("scores read from TMEM without waiting for their MMAs", "attn_fwd_simple.cuh",
      "      fail = !mbar_wait(&bars[2], mma_phase, P.wait_limit_ns);\n      mma_phase ^= 1;\n"
      "      if (__syncthreads_or(fail)) { fail = true; break; }\n      tc_fence_after_sync();\n\n      uint32_t s[4][32];",
