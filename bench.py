@@ -594,7 +594,8 @@ def run_step(args):
     rng = np.random.default_rng(0)
     peaks, peak_src = load_peaks()
     kind = args.step
-    if kind == "bwd_tc":
+    tensor_bwd = kind == "bwd_tc"
+    if tensor_bwd:
         mimo_attn.set_bwd_kernel(mimo_attn.BWD_TENSOR)
         kind = "bwd"
     if kind == "bwd":
@@ -610,8 +611,10 @@ def run_step(args):
         flops = W.attended_pairs(w.lengths, w.window, w.num_q_heads) * (2 * 192 * 3 + 2 * 128 * 2)  # S, dQ, dK; dP, dV
         nbytes = w.total_tokens * (w.num_q_heads * (192 * 2 + 128 * 2 * 2 + 4 + 192 * 4)
                                    + w.num_kv_heads * (192 * 2 + 128 * 2 + 192 * 4 + 128 * 4))
-        units, unit, config = w.total_tokens, "tokens/s", {"workload": "bwd_" + w.name, "grads": "fp32"}
-        bound = "alu"  # FP32 FMAs on the CUDA cores
+        units, unit = w.total_tokens, "tokens/s"
+        config = {"workload": ("bwd_tc_" if tensor_bwd else "bwd_") + w.name, "grads": "fp32",
+                  "kernel": "tcgen05, bf16 operands" if tensor_bwd else "fp32 cuda cores"}
+        bound = "tensor" if tensor_bwd else "alu"  # BF16 tcgen05 MMAs / FP32 FMAs on the CUDA cores
     elif kind == "dequant":
         # a fused qkv_proj weight of the sliding layer (hidden 4096, synthetic): 61 MB of codes, 122 MB out
         M_, N_ = 8 * (8 * 192 + 320), 4096
@@ -668,7 +671,8 @@ def run_step(args):
         ach, peak, runit = flops / (ms / 1e3) / 1e12, FP32_ALU_TFLOPS, "TFLOP/s"
         peak_src = "derived: 148 SMs x 128 FP32 lanes x 2 FLOP per FMA x 1965 MHz"
     line = {
-        "metric": f"{kind} throughput on 1 B200; % of roofline", "value": units / (ms / 1e3), "unit": unit,
+        "metric": f"{'bwd_tc' if tensor_bwd else kind} throughput on 1 B200; % of roofline", "value": units / (ms / 1e3),
+        "unit": unit,
         "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if kind != "route" else "f32", "data": "synthetic",
         "config": dict(config, l2="inputs larger than L2"),
@@ -676,7 +680,7 @@ def run_step(args):
                      "peak_source": peak_src if bound == "alu" else f"{peak_src} (burst)", "algorithmic_bytes": nbytes, "algorithmic_flops": flops},
         "e2e": None, "clocks": clk.summary(),
         # this library's kernels per step (the projection's GEMM runs in cuBLAS)
-        "gpu_launches": steps * {"bwd": 3, "dequant": 1, "split": 1, "route": 1, "proj": 0}[kind],
+        "gpu_launches": steps * ({"bwd": 3, "dequant": 1, "split": 1, "route": 1, "proj": 0}[kind] - tensor_bwd),
     }
     print(json.dumps(line), flush=True)
     return 0
