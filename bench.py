@@ -582,6 +582,38 @@ STEP_KINDS = ("bwd", "bwd_tc", "dequant", "split", "proj", "route")
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core FP32 FMA peak at the maximum SM clock
 
 
+# Shapes of the step lines (synthetic, layer-shaped) and their algorithmic FLOPs / bytes: every tensor
+# moved once, masked work and the exponentials not counted.
+STEP_SHAPES = {
+    "dequant": dict(M=8 * (8 * 192 + 320), N=4096, block=128),  # a fused qkv_proj weight, hidden 4096
+    "split": dict(T=16384, hq=64, hkv=8),
+    "proj": dict(T=4096, K=64 * 128, N=4096),  # 64 heads x 128 dims -> hidden 4096
+    "route": dict(T=262144, E=256, k=8),
+}
+
+
+def step_accounting(kind):
+    """(FLOPs, bytes, units) of one call of a step line; the backward on the swa4096 workload."""
+    if kind in ("bwd", "bwd_tc"):
+        w = W.WORKLOADS["swa4096"]()
+        flops = W.attended_pairs(w.lengths, w.window, w.num_q_heads) * (2 * 192 * 3 + 2 * 128 * 2)  # S dQ dK; dP dV
+        nbytes = w.total_tokens * (w.num_q_heads * (192 * 2 + 128 * 2 * 2 + 4 + 192 * 4)  # q, out, dout, lse, dq
+                                   + w.num_kv_heads * (192 * 2 + 128 * 2 + 192 * 4 + 128 * 4))  # k, v, dk, dv
+        return flops, nbytes, w.total_tokens
+    s = STEP_SHAPES[kind]
+    if kind == "dequant":
+        M, N, b = s["M"], s["N"], s["block"]
+        return 0, M * N * 3 + (-(-M // b)) * (-(-N // b)) * 4, M * N  # codes in, bf16 out, scales
+    if kind == "split":
+        width = s["hkv"] * (s["hq"] // s["hkv"] * 192 + 320)
+        return 0, s["T"] * width * 2 * 2, s["T"]  # every element read once and written once
+    if kind == "proj":
+        T, K, N = s["T"], s["K"], s["N"]
+        return 2 * T * K * N, 2 * (T * K + N * K + T * N), T
+    T, E, k = s["T"], s["E"], s["k"]
+    return 0, T * E * 4 + E * 4 + T * k * 8, T  # logits, bias, ids + weights
+
+
 def run_step(args):
     """One of the steps beside the forward (backward, FP8 dequant, fused-QKV split, MoE routing) on a
     layer-shaped synthetic input; one JSON line (single GPU)."""
@@ -608,46 +640,44 @@ def run_step(args):
         out, lse = mimo_attn.fwd(q, k, v, sk, cu, w.max_seqlen, w.layer_kind, w.window, w.rope_base)
         go = dev(synth.f32_to_bf16_bits(rng.standard_normal((w.total_tokens, w.num_q_heads, 128)).astype(np.float32)))
         call = lambda: mimo_attn.bwd(q, k, v, sk, cu, w.max_seqlen, w.layer_kind, w.window, w.rope_base, out, lse, go)
-        flops = W.attended_pairs(w.lengths, w.window, w.num_q_heads) * (2 * 192 * 3 + 2 * 128 * 2)  # S, dQ, dK; dP, dV
-        nbytes = w.total_tokens * (w.num_q_heads * (192 * 2 + 128 * 2 * 2 + 4 + 192 * 4)
-                                   + w.num_kv_heads * (192 * 2 + 128 * 2 + 192 * 4 + 128 * 4))
-        units, unit = w.total_tokens, "tokens/s"
+        flops, nbytes, units = step_accounting("bwd")
+        unit = "tokens/s"
         config = {"workload": ("bwd_tc_" if tensor_bwd else "bwd_") + w.name, "grads": "fp32",
                   "kernel": "tcgen05, bf16 operands" if tensor_bwd else "fp32 cuda cores"}
         bound = "tensor" if tensor_bwd else "alu"  # BF16 tcgen05 MMAs / FP32 FMAs on the CUDA cores
     elif kind == "dequant":
         # a fused qkv_proj weight of the sliding layer (hidden 4096, synthetic): 61 MB of codes, 122 MB out
-        M_, N_ = 8 * (8 * 192 + 320), 4096
+        M_, N_ = STEP_SHAPES["dequant"]["M"], STEP_SHAPES["dequant"]["N"]
         codes = rng.integers(0, 256, size=(M_, N_)).astype(np.uint8)
         codes[(codes & 0x7F) == 0x7F] = 0x3F
         scale = rng.uniform(0.5, 2.0, size=(-(-M_ // 128), -(-N_ // 128))).astype(np.float32)
         ct, st = torch.from_numpy(codes).cuda(), torch.from_numpy(scale).cuda()
         call = lambda: mimo_attn.fp8_dequant_blockwise(ct, st)
-        flops, nbytes = 0, M_ * N_ * 3 + scale.size * 4
-        units, unit, config, bound = M_ * N_, "elements/s", {"workload": f"fp8_dequant_{M_}x{N_}_block128"}, "hbm"
+        flops, nbytes, units = step_accounting("dequant")
+        unit, config, bound = "elements/s", {"workload": f"fp8_dequant_{M_}x{N_}_block128"}, "hbm"
     elif kind == "split":
-        T, hq, hkv = 16384, 64, 8  # 486 MB in, 486 MB out: larger than L2
+        T, hq, hkv = (STEP_SHAPES["split"][n] for n in ("T", "hq", "hkv"))  # 486 MB in and out: larger than L2
         fused = torch.from_numpy(rng.integers(0, 1 << 16, size=(T, hkv * (hq // hkv * 192 + 320))).astype(np.uint16)
                                  .view(np.int16)).cuda().view(torch.bfloat16)
         call = lambda: mimo_attn.qkv_split(fused, hq, hkv)
-        flops, nbytes = 0, fused.numel() * 2 * 2
-        units, unit, config, bound = T, "tokens/s", {"workload": f"qkv_split_T{T}_hq{hq}_hkv{hkv}"}, "hbm"
+        flops, nbytes, units = step_accounting("split")
+        unit, config, bound = "tokens/s", {"workload": f"qkv_split_T{T}_hq{hq}_hkv{hkv}"}, "hbm"
     elif kind == "proj":
         # the sliding layer's output projection: 64 heads x 128 dims -> hidden 4096 (synthetic), T = 4096
-        T, K_, N_ = 4096, 64 * 128, 4096
+        T, K_, N_ = (STEP_SHAPES["proj"][n] for n in ("T", "K", "N"))
         bf = lambda a: torch.from_numpy((a.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
                                         .view(np.int16)).cuda().view(torch.bfloat16)
         xt, wt = bf(rng.standard_normal((T, K_))), bf(rng.standard_normal((N_, K_)) / np.sqrt(K_))
         call = lambda: mimo_attn.linear_proj(xt, wt)
-        flops, nbytes = 2 * T * K_ * N_, 2 * (T * K_ + N_ * K_ + T * N_)
-        units, unit, config, bound = T, "tokens/s", {"workload": f"linear_proj_T{T}_in{K_}_out{N_}"}, "tensor"
+        flops, nbytes, units = step_accounting("proj")
+        unit, config, bound = "tokens/s", {"workload": f"linear_proj_T{T}_in{K_}_out{N_}"}, "tensor"
     else:
-        T, E = 262144, 256  # 268 MB of logits: larger than L2
+        T, E = STEP_SHAPES["route"]["T"], STEP_SHAPES["route"]["E"]  # 268 MB of logits: larger than L2
         lg = torch.from_numpy((rng.standard_normal((T, E)) * 2).astype(np.float32)).cuda()
         bias = torch.from_numpy((rng.standard_normal(E) * 0.1).astype(np.float32)).cuda()
         call = lambda: mimo_attn.moe_route(lg, bias, 8)
-        flops, nbytes = 0, T * E * 4 + E * 4 + T * 8 * 8
-        units, unit, config, bound = T, "tokens/s", {"workload": f"moe_route_T{T}_E{E}_top8"}, "hbm"
+        flops, nbytes, units = step_accounting("route")
+        unit, config, bound = "tokens/s", {"workload": f"moe_route_T{T}_E{E}_top8"}, "hbm"
     for _ in range(max(3, args.warmup)):
         call()
     torch.cuda.synchronize()

@@ -40,3 +40,20 @@ def test_decode_bytes_and_flops_by_hand():
     nbytes, flops = bench.decode_bytes_flops(x, -1)
     assert nbytes == 305 * (2 * (192 + 128) * 2 + 4) + 5 * 8 * (192 * 2 + 128 * 2 + 4)
     assert flops == 640 * ((4 + 5) + (298 + 299 + 300)) * 8
+
+
+def test_step_lines_by_hand():
+    """The step lines' algorithmic counts against hand counts of their shapes."""
+    # backward: 1664 FLOPs per attended pair (S, dQ, dK over 192 dims; dP, dV over 128)
+    flops, nbytes, units = bench.step_accounting("bwd")
+    assert flops == 1664 * 520128 * 64 and units == 4096
+    assert nbytes == 4096 * (64 * (384 + 512 + 4 + 768) + 8 * (384 + 256 + 768 + 512))
+    assert bench.step_accounting("bwd_tc") == (flops, nbytes, units)
+    # FP8 dequant of a 14848 x 4096 weight: 1 byte in, 2 out per element, 116 x 32 FP32 scales
+    assert bench.step_accounting("dequant") == (0, 14848 * 4096 * 3 + 116 * 32 * 4, 14848 * 4096)
+    # fused-QKV split: 8 groups x (8 x 192 + 192 + 128) = 14848 BF16 per token, read and written once
+    assert bench.step_accounting("split") == (0, 16384 * 14848 * 2 * 2, 16384)
+    # output projection 4096 x 8192 by 8192 x 4096
+    assert bench.step_accounting("proj") == (2 * 4096 * 8192 * 4096, 2 * (2 * 4096 * 8192 + 4096 * 4096), 4096)
+    # router: FP32 logits and bias in, int32 ids and FP32 weights of the top 8 out
+    assert bench.step_accounting("route") == (0, 262144 * 256 * 4 + 256 * 4 + 262144 * 8 * 8, 262144)
