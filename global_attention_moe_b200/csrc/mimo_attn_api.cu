@@ -211,7 +211,7 @@ std::pair<cudaEvent_t, cudaEvent_t>* profile_slot(int dev) {
 struct DeviceInfo {
   int sms = 0;
   bool kernels_ready = false;  // dynamic shared memory limits raised
-  cudaMemPool_t pool = nullptr;  // stream-ordered scratch, kept by the library (never released to the OS)
+  cudaMemPool_t pool = nullptr;  // stream-ordered scratch; returned to the device at the next synchronization
 };
 
 DeviceInfo* device_info(int dev) {
@@ -228,9 +228,15 @@ DeviceInfo* device_info(int dev) {
     props.allocType = cudaMemAllocationTypePinned;
     props.location.type = cudaMemLocationTypeDevice;
     props.location.id = dev;
+    // Release threshold 0: memory freed (stream-ordered) by a call is reused by later calls on the same
+    // stream without synchronizing, and goes back to the device at the next synchronization, so the
+    // library keeps no scratch between synchronized calls.
     if (cudaMemPoolCreate(&d.pool, &props) == cudaSuccess) {
-      uint64_t keep = UINT64_MAX;
-      cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+      uint64_t keep = 0;
+      if (cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+        cudaMemPoolDestroy(d.pool);
+        d.pool = nullptr;
+      }
     } else {
       d.pool = nullptr;
     }
@@ -384,13 +390,14 @@ NoAllocInfo* noalloc_info(int dev) {
 }
 
 int launch_noalloc(const void* q, const void* k, const void* v, const FwdParams& P, cudaStream_t stream) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
   Path path;
   if (const int sel = select_path(P, path); sel != MIMO_OK) return sel;
   const bool pipelined = path != Path::Simple;
   const size_t kr_rows = (size_t)P.total_tokens * P.hkv;
+  // The size check comes before any CUDA call, so that it holds on a machine without a GPU too.
   if (pipelined && kr_rows * kRopeDims * 2 > kNoAllocScratchBytes) return MIMO_ERR_SCRATCH_LIMIT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ERR_CUDA;
   NoAllocInfo* info = noalloc_info(dev);
   if (!info) return MIMO_ERR_CUDA;
   if (P.max_seqlen == 0) return MIMO_OK;

@@ -99,15 +99,22 @@ typedef struct {
  *   out        bf16 [T, Hq, 128]          (device) every row of every head is written
  *   lse        fp32 [Hq, T]               (device) natural-log normaliser, including
  *              the sink term
- * Rotated Q/K rope dims enter the tensor cores as FP16 (the pass-through dims
- * stay BF16), so |q|, |k| on the first 64 dims must stay below 2^15; a larger
- * rotated value is recorded as MIMO_ERR_RANGE for mimo_attn_check.
- * Scratch: when a two-head kernel runs (Hq/Hkv even: the window or the
- * pipelined kernel, see mimo_attn_set_kernel), the call rotates K's
- * rope dims once into T * Hkv * 128 bytes of transient device scratch taken
- * from a library-owned stream-ordered memory pool (cudaMallocFromPoolAsync on
- * `stream`, returned with cudaFreeAsync on the same stream; the pool keeps
- * its memory for reuse until the process exits).  Does not synchronise.
+ * Range: rotated Q/K rope dims enter the tensor cores as FP16 (the pass-through
+ * dims stay BF16).  A rotated value is x_i cos(a) - x_{i+32} sin(a) (or its
+ * partner), at most sqrt(2) max(|x_i|, |x_{i+32}|) in magnitude, so inputs
+ * whose first 64 dims stay within 65504 / sqrt(2) = 46318 in magnitude never
+ * overflow.  Larger inputs may, depending on the position; a rotated value
+ * above 65504 in magnitude (the largest finite FP16) is recorded as
+ * MIMO_ERR_RANGE for mimo_attn_check and that call's output is not valid.
+ * Scratch: when a two-head kernel that reads K's rope dims pre-rotated runs
+ * (the pipelined kernel, and the window kernel where it is chosen, see
+ * mimo_attn_set_kernel), the call rotates them once into T * Hkv * 128 bytes
+ * of transient device scratch from a library-owned stream-ordered pool
+ * (cudaMallocFromPoolAsync on `stream`, cudaFreeAsync on the same stream).
+ * The pool's release threshold is 0: later calls on the stream reuse the
+ * memory without synchronizing, and the next synchronization returns it to
+ * the device, so nothing persists between synchronized calls.  Does not
+ * synchronise.
  */
 MIMO_API int mimo_attn_fwd(const void* q, const void* k, const void* v, const float* sink,
                   const int32_t* cu_seqlens, const mimo_attn_dims* dims, int layer_kind,

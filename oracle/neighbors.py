@@ -22,7 +22,7 @@ section):
   Configuration tips, Parallelism and precision (router logits computed in
   FP32).
 
-Readings where the pages are silent (each listed in the design notes):
+Readings where the pages are silent:
 
 * FP8 element format: OCP E4M3 ("fn": no infinities, S.1111.111 is NaN).
   The block size of the scales is not given: 128 x 128 blocks here, a

@@ -19,8 +19,11 @@ def pytest_configure(config):
 # GPU modules in the order they were established: under -x, a failure in a newer module does not
 # keep the older suites from running (and being reported).  Modules not listed (CPU tests) come
 # first, in their own order.
-_GPU_MODULE_ORDER = ("test_gpu_parity.py", "test_gpu_decode.py", "test_zz_no_alloc.py", "test_gpu_decode_tiles.py",
-                     "test_gpu_neighbors.py", "test_gpu_bwd.py", "test_gpu_bwd_tc.py")
+# The no-alloc entry point's module comes last of all, so that a failure there cannot stop any other
+# suite under -x.
+_GPU_MODULE_ORDER = ("test_gpu_parity.py", "test_gpu_full_tensor.py", "test_gpu_decode.py",
+                     "test_gpu_decode_tiles.py", "test_gpu_neighbors.py", "test_gpu_bwd.py", "test_gpu_bwd_tc.py",
+                     "test_zz_no_alloc.py")
 
 
 def pytest_collection_modifyitems(session, config, items):

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(M):
 
 
 def test_status_strings_and_version(M):
-    for s in range(7):
+    for s in range(8):
         assert M.status_string(s) and M.status_string(s) != "unknown status"
     assert M.status_string(99) == "unknown status"
     assert M.version()[0] == 1
@@ -171,3 +171,16 @@ def test_linear_proj_validation(M, args, expect):
     a = dict(x=FAKE, w=FAKE, tokens=4, k=1024, n=512, y=FAKE)
     a.update(args)
     assert M.LIB.mimo_linear_proj(a["x"], a["w"], a["tokens"], a["k"], a["n"], a["y"], None) == expect
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch(M):
+    """The no-alloc entry point checks its fixed scratch size before any CUDA
+    call: one row past the limit is refused on a machine without a GPU too."""
+    limit_rows = M.noalloc_scratch_bytes() // 128  # T * Hkv rows of 64 FP16 dims
+    hkv = 8
+    T = limit_rows // hkv + 1
+    dims = M.make_dims(1, T, T, 16, hkv)
+    st = M.LIB.mimo_attn_fwd_noalloc(FAKE, FAKE, FAKE, None, FAKE, ctypes.byref(dims), 1, -1, 1e7, 64, 0.707,
+                                     FAKE, FAKE, None)
+    assert st == M.ERR_SCRATCH_LIMIT
+    assert "scratch" in M.status_string(st)

@@ -296,3 +296,44 @@ def test_many_short_sequences_cross_pair_and_sequence_boundaries():
     rng = np.random.default_rng(15)
     lengths = [int(v) for v in rng.integers(1, 301, size=40)]
     full_parity(W.custom("many", W.LAYER_SWA, lengths, 16, 2, 128, 1e4, True, seed=15))
+
+
+@pytest.mark.parametrize("which", ["q", "k"])
+@pytest.mark.parametrize("value,overflows", [(46080.0, False), (48128.0, True)])
+def test_fp16_range_limit_of_rotated_dims(which, value, overflows):
+    """A rope pair (x_0, x_32) = (a, -a) at position 1 rotates to a (cos 1 + sin 1) = 1.3818 a on
+    dim 0: a = 46080 gives 63673, inside FP16's largest finite value 65504, and a = 48128 gives
+    66503, past it.  The first call runs clean, the second records MIMO_ERR_RANGE."""
+    from global_attention_moe_b200 import mimo_attn
+    w = W.custom("range_limit", W.LAYER_SWA, [64], 4, 1, 128, 1e4, True, seed=17)
+    x = W.make_inputs(w)
+    a = W.synth.f32_to_bf16_bits(np.array([value, -value], dtype=np.float32))
+    t = getattr(x, which).copy()
+    t[1, 0, 0], t[1, 0, 32] = a[0], a[1]
+    setattr(x, which, t)
+    dq, dk, dv, ds, dcu = to_device(x)
+    out, lse = mimo_attn.fwd(dq, dk, dv, ds, dcu, 64, 0, 128, 1e4)
+    st = mimo_attn.check()
+    if overflows:
+        assert st == mimo_attn.ERR_RANGE
+    else:
+        assert st == mimo_attn.OK
+        assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+def test_pool_scratch_returned_after_synchronize():
+    """Scratch a call takes from the library's stream-ordered pool (here the pre-rotated K rope
+    dims of the global layer's kernel, T * Hkv * 128 bytes = 32 MiB) goes back to the device at
+    the next synchronization: free device memory after a synchronized call is what it was before."""
+    w = W.custom("pool", W.LAYER_GLOBAL, [8192] * 4, 16, 8, -1, 1e7, False, seed=18)
+    x = W.make_inputs(w)
+    dev = to_device(x)
+    out = torch.empty(w.total_tokens, 16, 128, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(16, w.total_tokens, dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(2):
+        run_gpu(w, x, dev_inputs=dev, out=out, lse=lse)  # synchronizes (mimo_attn_check)
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
+    assert free0 - free1 < 4 * 2 ** 20, (free0, free1)
