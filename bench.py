@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-parity", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="SWA-4096 only: skip the global layer's record that the line otherwise carries")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--ref-budget-s", type=float, default=90.0, help="reference arm: total CPU seconds to aim for")
     ap.add_argument("--decode", choices=W.DECODE_KINDS, default=None,
@@ -182,7 +184,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.0002)  # short timed regions still get several samples
 
     def __enter__(self):
         if self._ok:
@@ -203,11 +205,12 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle
-def cpu_oracle_rate(w: W.Workload, x: W.Inputs, target_s: float, max_rows_per_call: int | None = None):
+def cpu_oracle_rate(w: W.Workload, x: W.Inputs, target_s: float, max_rows_per_call: int | None = None,
+                    threads: int | None = None):
     """Time the oracle (as it stands) on samples of the workload's rows.
     Returns (tokens/s, cores, description)."""
     import oracle
-    cores = oracle.default_threads()
+    cores = threads or oracle.default_threads()
     rng = np.random.default_rng(0)
     order = rng.permutation(w.total_tokens)
     # calibrate on a small sample
@@ -233,7 +236,7 @@ def cpu_oracle_rate(w: W.Workload, x: W.Inputs, target_s: float, max_rows_per_ca
         if rows == w.total_tokens and elapsed >= 0.5 * target_s:
             break
     desc = (f"{calls} oracle call(s) of {rows} seeded-random token rows (all {w.num_q_heads} heads each) of "
-            f"{w.name}; {elapsed:.1f} s of CPU time")
+            f"{w.name} on {cores} host thread(s); {elapsed:.1f} s of CPU time")
     return done / elapsed, cores, desc
 
 
@@ -286,23 +289,31 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args):
+TC_FLOP_PER_CLK_SM = 8192  # dense BF16 tcgen05: one M128 N256 K16 MMA (1 MFLOP) per 128 cycles per SM
+SECONDARY = {"swa4096": "global"}  # the metric names both layer kinds: the SWA line carries the global one
+
+
+def launches_per_step(w) -> int:
+    """This library's kernels per forward: the attention kernel, plus the K RoPE pre-pass where the
+    chosen kernel reads K's rope dims pre-rotated."""
+    return 2 if dominant_kernel(w) in ("attn_fwd_pipelined_kernel", "attn_fwd_swa_kernel") else 1
+
+
+def percentiles(xs):
+    xs = sorted(xs)
+    pick = lambda f: xs[min(len(xs) - 1, max(0, int(round(f * (len(xs) - 1)))))]
+    return {"p10": pick(0.10), "p50": pick(0.50), "p90": pick(0.90), "n": len(xs)}
+
+
+def measure(args, w, rank, world, dev, with_cpu: bool):
+    """Times one workload on this rank: K steps over rotating input sets (one event pair around all,
+    one per step), the attention kernel alone (library events), a repeat on one input set, the
+    end-to-end host-buffer entry, a parity spot check and the CPU oracle.  Returns a dict of fields."""
     import torch
     import torch.distributed as dist
 
     from global_attention_moe_b200 import mimo_attn
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus and rank == 0:
-        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-
-    w = rank_workload(args.workload, rank)
     x = W.make_inputs(w)
     T = w.total_tokens
     stream = torch.cuda.current_stream()
@@ -340,41 +351,52 @@ def run_ours(args):
     if st != mimo_attn.OK:
         raise mimo_attn.MimoAttnError(st, "warm-up")
 
+    # K steps: one event pair around all of them (the value), one event per step boundary (spread)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index) as clk:
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         ev0.record(stream)
         for i in range(args.steps):
+            evs[i].record(stream)
             step(i)
+        evs[args.steps].record(stream)
         ev1.record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
     ms = ev0.elapsed_time(ev1)
+    per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
     st = mimo_attn.check()
     if st != mimo_attn.OK:
         raise mimo_attn.MimoAttnError(st, "timed region")
     ms = max_over_ranks(ms, dev)
     ms_per_step = ms / max(args.steps, 1)
-    value = aggregate_rate(world, T, args.steps, ms)
-    launches_per_step = 2 if (w.num_q_heads // w.num_kv_heads) % 2 == 0 else 1  # K RoPE pre-pass + attention
+    n_launch = launches_per_step(w)
 
-    # --- the dominant (attention) kernel alone, timed by library-recorded events in a second pass
-    kernel_ms = None
-    if launches_per_step == 2:
-        kn = max(1, min(args.steps, 500))
-        mimo_attn.profile_start()
-        for i in range(kn):
-            step(i)
-        torch.cuda.synchronize()
-        n_rec, tot = mimo_attn.profile_stop()
-        if n_rec:
-            kernel_ms = max_over_ranks(tot / n_rec, dev)
+    # the attention kernel alone, timed by library-recorded events on the launching stream
+    kn = max(1, min(args.steps, 500))
+    mimo_attn.profile_start()
+    for i in range(kn):
+        step(i)
+    torch.cuda.synchronize()
+    n_rec, tot = mimo_attn.profile_stop()
+    kernel_ms = max_over_ranks(tot / n_rec, dev) if n_rec else None
 
-    # --- end to end through the host-buffer C-ABI entry (pinned host memory, copies inside the region)
+    # the same K steps on one input set (its inputs partly L2-resident between steps): context only
+    torch.cuda.synchronize()
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
+    for _ in range(args.steps):
+        step(0)
+    w1.record(stream)
+    torch.cuda.synchronize()
+    warm_ms = max_over_ranks(w0.elapsed_time(w1), dev) / max(args.steps, 1)
+
+    # end to end through the host-buffer C-ABI entry (pinned host memory, copies inside the region)
     e2e = None
     if not args.no_e2e:
         pin = lambda a: torch.from_numpy(a).pin_memory()
@@ -402,8 +424,9 @@ def run_ours(args):
         ems = max_over_ranks(e0.elapsed_time(e1), dev)
         e2e = {"value": aggregate_rate(world, T, ne, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": ne}
+        del qh, kh, vh, shh, ch, oh, lh, ws
 
-    # --- parity spot check of this run's output against the oracle (rank 0)
+    # parity spot check of this run's output against the oracle (rank 0)
     parity = None
     if rank == 0 and not args.no_parity:
         import oracle
@@ -420,52 +443,89 @@ def run_ours(args):
                   "rel_l2": float(np.linalg.norm(d) / np.linalg.norm(ro)), "lse_max_abs": float(np.abs(gl - rl).max())}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, cores, desc = cpu_oracle_rate(w, x, target_s=12.0)
+    if rank == 0 and world == 1 and with_cpu and not args.no_cpu_baseline:
+        rate, cores, desc = cpu_oracle_rate(w, x, target_s=10.0)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+        if w.name in ("swa_sink_T4096_h64_kv8", "tiny_swa_sink_T512_h4_kv1"):
+            r1, _, d1 = cpu_oracle_rate(w, x, target_s=3.0, threads=1)
+            cpu["single_thread"] = {"value": r1, "unit": "tokens/s", "cores": 1, "sample": d1}
+    del sets
+    torch.cuda.empty_cache()
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return 0
-
+    clocks = clk.summary()
     peaks, peak_src = load_peaks()
     flops = flops_per_step(w)
     nbytes = bytes_per_step(w)
     t_s = ms_per_step / 1e3
-    tflops = flops / t_s / 1e12
-    gbs = nbytes / t_s / 1e9
-    tk_s = (kernel_ms if kernel_ms else ms_per_step) / 1e3  # dominant kernel's own launch duration
+    tk_s = (kernel_ms if kernel_ms else ms_per_step) / 1e3  # the attention kernel's own launch duration
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     long_region = ms > 1000.0
     tc_peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
     t_tc = flops / (tc_peak * 1e12)
     kernel = dominant_kernel(w)
-    traffic = recorded_traffic(kernel, w.name)
     if t_hbm >= t_tc:
         ach = nbytes / tk_s / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
     else:
         ach = flops / tk_s / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s", "frac": ach / tc_peak}
-    roof.update({"traffic": traffic, "peak_source": f"{peak_src} ({'sustained' if long_region and roof['bound'] == 'tensor' else 'burst'})",
+        if clocks.get("sm_mhz"):
+            issue_peak = 148 * TC_FLOP_PER_CLK_SM * clocks["sm_mhz"] * 1e6 / 1e12
+            roof["tcgen05_issue_peak"] = {
+                "tflops": issue_peak, "frac": ach / issue_peak,
+                "basis": "148 SMs x 8192 dense BF16 FLOP/clk/SM (M128 N256 K16 MMA in 128 cycles) x the median "
+                         "SM clock sampled in the timed region; a labelled second ratio, not the roofline peak"}
+    roof.update({"traffic": recorded_traffic(kernel, w.name),
+                 "peak_source": f"{peak_src} ({'sustained' if long_region and roof['bound'] == 'tensor' else 'burst'})",
                  "kernel": kernel, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
-                 "kernel_us": tk_s * 1e6, "step_frac": (ms_per_step / 1e3) and tk_s / (ms_per_step / 1e3)})
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                 "kernel_us": tk_s * 1e6, "step_frac": tk_s / t_s})
+    return {
+        "value": aggregate_rate(world, T, args.steps, ms), "ms_per_step": ms_per_step,
+        "per_step_ms": percentiles(per_step), "warm_l2_ms_per_step": warm_ms,
         "config": {**w.describe(), "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"inputs rotated over {n_sets} device buffer sets ({n_sets * set_bytes / 2**20:.0f} MiB > 126 MiB L2), no flush"},
-        "tflops": tflops, "gbs": gbs, "roofline_time_us": max(t_hbm, t_tc) * 1e6,
-        "roofline": roof,
-        "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": args.steps * launches_per_step,
-        "clocks": clk.summary(),
-        "parity": parity,
+                   "l2": f"inputs rotated over {n_sets} device buffer sets ({n_sets * set_bytes / 2**20:.0f} MiB > "
+                         f"126 MiB L2), no flush"},
+        "tflops": flops / t_s / 1e12, "gbs": nbytes / t_s / 1e9, "roofline_time_us": max(t_hbm, t_tc) * 1e6,
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * n_launch,
+        "clocks": clocks, "parity": parity,
     }
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and rank == 0:
+        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    main = measure(args, rank_workload(args.workload, rank), rank, world, dev, with_cpu=True)
+    second = None
+    if args.workload in SECONDARY and not args.no_secondary:
+        second = measure(args, rank_workload(SECONDARY[args.workload], rank), rank, world, dev, with_cpu=True)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": main["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+    }
+    line.update({k: v for k, v in main.items() if k not in ("value", "ms_per_step")})
+    if second is not None:
+        # the other layer kind of the metric, measured the same way in the same run
+        line["gpu_launches"] += second["gpu_launches"]
+        line["global_layer"] = {"metric": METRIC, "unit": "tokens/s", "steps": args.steps, "warmup": args.warmup,
+                                **second}
     print(json.dumps(line), flush=True)
     return 0
 

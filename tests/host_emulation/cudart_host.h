@@ -24,6 +24,7 @@ cudaError_t cudaMemPoolCreate(cudaMemPool_t* p, const struct cudaMemPoolProps*) 
   return cudaSuccess;
 }
 cudaError_t cudaMemPoolSetAttribute(cudaMemPool_t, enum cudaMemPoolAttr, void*) { return cudaSuccess; }
+cudaError_t cudaMemPoolDestroy(cudaMemPool_t) { return cudaSuccess; }
 cudaError_t cudaMallocFromPoolAsync(void** p, size_t n, cudaMemPool_t, cudaStream_t) {
   *p = hemu::guarded_alloc(n);
   return cudaSuccess;
