@@ -42,7 +42,7 @@ FLOPS_PER_PAIR = 2 * 192 + 2 * 128
 # Device code of the two-head kernels: the traffic recorded in profiles/traffic.json is valid
 # only while these files are unchanged.
 KERNEL_SOURCES = ["csrc/sm100.cuh", "csrc/rope_smem.cuh", "csrc/params.cuh", "csrc/rope_k_prepass.cuh",
-                  "csrc/attn_fwd_pipelined.cuh", "csrc/attn_fwd_swa.cuh"]
+                  "csrc/attn_fwd_pipelined.cuh", "csrc/attn_fwd_swa.cuh", "csrc/attn_fwd_swa_packed.cuh"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -95,7 +95,10 @@ def load_peaks():
 
 def dominant_kernel(w) -> str:
     """The attention kernel the library's default choice launches for this shape."""
-    if (w.num_q_heads // w.num_kv_heads) % 2 != 0:
+    group = w.num_q_heads // w.num_kv_heads
+    if w.layer_kind == W.LAYER_SWA and 0 <= w.window <= 128 and group in (4, 8):
+        return "attn_fwd_swa_packed_kernel"
+    if group % 2 != 0:
         return "attn_fwd_simple_kernel"
     if w.layer_kind == W.LAYER_SWA and 0 <= w.window <= 128:
         return "attn_fwd_swa_kernel"

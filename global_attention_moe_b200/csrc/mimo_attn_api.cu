@@ -20,6 +20,7 @@
 #include "attn_fwd_pipelined.cuh"
 #include "attn_fwd_simple.cuh"
 #include "attn_fwd_swa.cuh"
+#include "attn_fwd_swa_packed.cuh"
 #include "attn_decode.cuh"
 #include "attn_decode_tc.cuh"
 #include "attn_bwd_simple.cuh"
@@ -57,6 +58,21 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3-D BF16 view of q [T, Hq, 192] as (dims, heads, tokens) with a {64, G, 128/G} box: one box is a
+// 128-row tile of 128/G tokens x the G query heads of one KV group (heads fastest), 128-byte swizzle.
+bool encode_q_packed(CUtensorMap* m, const void* q, int hq, int total_tokens, int group) {
+  auto enc = tensormap_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kHeadDimQK, (cuuint64_t)hq, (cuuint64_t)total_tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)kHeadDimQK * 2, (cuuint64_t)hq * kHeadDimQK * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)(128 / group)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -117,17 +133,21 @@ void fill_params(FwdParams& P, const float* sink, const int32_t* cu, const mimo_
 
 std::atomic<int> g_kernel_choice{MIMO_KERNEL_AUTO};
 
-enum class Path { Simple, Pipelined, Window };
+enum class Path { Simple, Pipelined, Window, Packed };
 
 // Chooses the kernel for one call from the process-wide choice and the shape.
 int select_path(const FwdParams& P, Path& path) {
   const bool even = P.group % 2 == 0;
   const bool short_window = P.window >= 0 && P.window <= kBlockN;
+  const bool packs = short_window && (P.group == 4 || P.group == 8);
   switch (g_kernel_choice.load()) {
     case MIMO_KERNEL_SIMPLE: path = Path::Simple; return MIMO_OK;
     case MIMO_KERNEL_PIPELINED: path = Path::Pipelined; return even ? MIMO_OK : MIMO_ERR_UNSUPPORTED;
     case MIMO_KERNEL_WINDOW: path = Path::Window; return (even && short_window) ? MIMO_OK : MIMO_ERR_UNSUPPORTED;
-    default: path = !even ? Path::Simple : (short_window ? Path::Window : Path::Pipelined); return MIMO_OK;
+    case MIMO_KERNEL_WINDOW_PACKED: path = Path::Packed; return packs ? MIMO_OK : MIMO_ERR_UNSUPPORTED;
+    default:
+      path = packs ? Path::Packed : !even ? Path::Simple : (short_window ? Path::Window : Path::Pipelined);
+      return MIMO_OK;
   }
 }
 
@@ -139,6 +159,10 @@ bool set_smem_attributes() {
                               pipe::kSmemBytes) == cudaSuccess &&
          cudaFuncSetAttribute(attn_fwd_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               pipe::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(attn_fwd_swa_packed_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              pk::Shape<4>::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(attn_fwd_swa_packed_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              pk::Shape<8>::kSmemBytes) == cudaSuccess &&
          cudaFuncSetAttribute(dec::attn_decode_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               dec::kSmemBytes) == cudaSuccess &&
          cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -175,6 +199,27 @@ void launch_two_head(Path path, int grid, const CUtensorMap& tq, const CUtensorM
     attn_fwd_swa_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tkr, tk, tv, P);
   else
     attn_fwd_pipelined_kernel<<<grid, pipe::kThreads, pipe::kSmemBytes, stream>>>(tq, tkr, tk, tv, P);
+}
+
+// The packed window kernel: no scratch, one persistent CTA per SM (at most one per tile).
+int launch_packed(const void* q, const void* k, const void* v, const FwdParams& P, int sms,
+                  std::pair<cudaEvent_t, cudaEvent_t>* ev, cudaStream_t stream) {
+  const int qt = 128 / P.group;
+  CUtensorMap tq, tk, tv;
+  if (!encode_q_packed(&tq, q, P.hq, P.total_tokens, P.group) ||
+      !encode_2d(&tk, k, (uint64_t)P.hkv * kHeadDimQK, P.total_tokens, pk::kBlk) ||
+      !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, P.total_tokens, pk::kBlk))
+    return MIMO_ERR_CUDA;
+  const long long tiles = (long long)P.hkv * ((long long)P.total_tokens / qt + P.num_seqs);
+  const int grid = (int)std::min<long long>(tiles, sms);
+  if (ev) cudaEventRecord(ev->first, stream);
+  if (P.group == 8)
+    attn_fwd_swa_packed_kernel<8><<<grid, pk::kThreads, pk::Shape<8>::kSmemBytes, stream>>>(tq, tk, tv, P);
+  else
+    attn_fwd_swa_packed_kernel<4><<<grid, pk::kThreads, pk::Shape<4>::kSmemBytes, stream>>>(tq, tk, tv, P);
+  const bool ok = cudaGetLastError() == cudaSuccess;
+  if (ev) cudaEventRecord(ev->second, stream);
+  return ok ? MIMO_OK : MIMO_ERR_CUDA;
 }
 
 // Kernel timing: while enabled, each forward records an event pair around its
@@ -294,6 +339,8 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& P, cuda
   if (P.max_seqlen == 0) return MIMO_OK;
   Path path;
   if (const int sel = select_path(P, path); sel != MIMO_OK) return sel;
+  if (!info->kernels_ready) return MIMO_ERR_CUDA;
+  if (path == Path::Packed) return launch_packed(q, k, v, P, info->sms, profile_slot(dev), stream);
   const bool two_head = path != Path::Simple;
   CUtensorMap tq, tk, tv;
   if (!encode_2d(&tq, q, (uint64_t)P.hq * kHeadDimQK, P.total_tokens) ||
@@ -392,7 +439,7 @@ NoAllocInfo* noalloc_info(int dev) {
 int launch_noalloc(const void* q, const void* k, const void* v, const FwdParams& P, cudaStream_t stream) {
   Path path;
   if (const int sel = select_path(P, path); sel != MIMO_OK) return sel;
-  const bool pipelined = path != Path::Simple;
+  const bool pipelined = path == Path::Pipelined || path == Path::Window;  // the kernels that read pre-rotated K
   const size_t kr_rows = (size_t)P.total_tokens * P.hkv;
   // The size check comes before any CUDA call, so that it holds on a machine without a GPU too.
   if (pipelined && kr_rows * kRopeDims * 2 > kNoAllocScratchBytes) return MIMO_ERR_SCRATCH_LIMIT;
@@ -401,6 +448,7 @@ int launch_noalloc(const void* q, const void* k, const void* v, const FwdParams&
   NoAllocInfo* info = noalloc_info(dev);
   if (!info) return MIMO_ERR_CUDA;
   if (P.max_seqlen == 0) return MIMO_OK;
+  if (path == Path::Packed) return launch_packed(q, k, v, P, info->sms, nullptr, stream);  // needs no scratch
   CUtensorMap tq, tk, tv;
   if (!encode_2d(&tq, q, (uint64_t)P.hq * kHeadDimQK, P.total_tokens) ||
       !encode_2d(&tk, k, (uint64_t)P.hkv * kHeadDimQK, P.total_tokens) ||
@@ -910,7 +958,7 @@ int mimo_attn_set_decode_kernel(int choice) {
 
 int mimo_attn_set_kernel(int choice) {
   if (choice != MIMO_KERNEL_AUTO && choice != MIMO_KERNEL_SIMPLE && choice != MIMO_KERNEL_PIPELINED &&
-      choice != MIMO_KERNEL_WINDOW)
+      choice != MIMO_KERNEL_WINDOW && choice != MIMO_KERNEL_WINDOW_PACKED)
     return MIMO_ERR_INVALID_ARG;
   g_kernel_choice.store(choice);
   return MIMO_OK;

@@ -24,7 +24,7 @@ SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host
            "mimo_attn_profile_stop", "mimo_attn_decode", "mimo_attn_set_decode_kernel", "mimo_attn_version",
            "mimo_attn_bwd", "mimo_fp8_dequant_blockwise", "mimo_qkv_split", "mimo_moe_route",
            "mimo_linear_proj", "mimo_attn_set_bwd_kernel")
-KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED, KERNEL_WINDOW = 0, 1, 2, 3
+KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED, KERNEL_WINDOW, KERNEL_WINDOW_PACKED = 0, 1, 2, 3, 4
 DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR = 0, 1, 2
 
 
@@ -110,7 +110,7 @@ def version() -> tuple[int, int]:
 
 
 def set_kernel(choice: int) -> None:
-    """Select the kernel mimo_attn_fwd launches (KERNEL_AUTO / _SIMPLE / _PIPELINED / _WINDOW)."""
+    """Select the kernel mimo_attn_fwd launches (KERNEL_AUTO / _SIMPLE / _PIPELINED / _WINDOW / _WINDOW_PACKED)."""
     st = LIB.mimo_attn_set_kernel(int(choice))
     if st != OK:
         raise MimoAttnError(st, "mimo_attn_set_kernel")

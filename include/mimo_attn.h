@@ -196,9 +196,10 @@ MIMO_API size_t mimo_attn_noalloc_scratch_bytes(void);
 
 /* Kernel selection for mimo_attn_fwd and mimo_attn_fwd_noalloc (process-wide;
  * default AUTO).
- *   MIMO_KERNEL_AUTO       WINDOW when Hq/Hkv is even and 0 <= window <= 128,
- *                          PIPELINED when Hq/Hkv is even otherwise (the global
- *                          layer, longer windows), else SIMPLE
+ *   MIMO_KERNEL_AUTO       for a sliding-window call with 0 <= window <= 128:
+ *                          WINDOW_PACKED when Hq/Hkv is 4 or 8, else WINDOW when
+ *                          Hq/Hkv is even; PIPELINED when Hq/Hkv is even otherwise
+ *                          (the global layer, longer windows); else SIMPLE
  *   MIMO_KERNEL_SIMPLE     one CTA per (128-query tile, head), every step serialised;
  *                          any Hq/Hkv ratio (the cross-check path)
  *   MIMO_KERNEL_PIPELINED  warp-specialised persistent kernel, two heads per CTA,
@@ -209,6 +210,14 @@ MIMO_API size_t mimo_attn_noalloc_scratch_bytes(void);
  *                          scored first and softmaxed in one pass; Hq/Hkv must be
  *                          even and the call a sliding-window one with
  *                          window <= 128
+ *   MIMO_KERNEL_WINDOW_PACKED  sliding windows of at most 128 keys with the
+ *                          Hq/Hkv query heads of a KV group packed into each
+ *                          128-row tile (128/G tokens x G heads): a tile spans
+ *                          128/G + 128 keys instead of 256, K/V stream through
+ *                          a ring of 16-key blocks, and RoPE of both Q and K is
+ *                          applied in shared memory (no pre-pass, no scratch);
+ *                          Hq/Hkv must be 4 or 8 and the call a sliding-window
+ *                          one with window <= 128
  * A forced choice whose condition fails makes the call return
  * MIMO_ERR_UNSUPPORTED.  Returns MIMO_ERR_INVALID_ARG for any other value.
  * All kernels compute the same operation; they differ only in the order of
@@ -218,15 +227,16 @@ typedef enum {
   MIMO_KERNEL_AUTO = 0,
   MIMO_KERNEL_SIMPLE = 1,
   MIMO_KERNEL_PIPELINED = 2,
-  MIMO_KERNEL_WINDOW = 3
+  MIMO_KERNEL_WINDOW = 3,
+  MIMO_KERNEL_WINDOW_PACKED = 4
 } mimo_kernel_choice;
 MIMO_API int mimo_attn_set_kernel(int choice);
 
 /*
  * Kernel timing for measurement tools.  After mimo_attn_profile_start, every
- * forward that runs a two-head kernel (window or pipelined) records a CUDA
- * event pair (events owned by the library) around that kernel on the call's
- * stream.
+ * forward that runs a persistent kernel (window, packed window or pipelined)
+ * records a CUDA event pair (events owned by the library) around that kernel
+ * on the call's stream.
  * mimo_attn_profile_stop ends recording, waits for the recorded events, and
  * returns how many attention-kernel launches were recorded and their summed
  * duration in milliseconds (the K RoPE pre-pass is excluded).  Process-wide.

@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstdlib>
+
 namespace hemu {
 inline bool g_launch_failed = false;
 CUresult host_encode_tiled(CUtensorMap* m, CUtensorMapDataType dt, cuuint32_t rank, void* base, const cuuint64_t* dims,
@@ -15,7 +17,9 @@ CUresult host_encode_tiled(CUtensorMap* m, CUtensorMapDataType dt, cuuint32_t ra
 extern "C" {
 cudaError_t cudaGetDevice(int* d) { *d = 0; return cudaSuccess; }
 cudaError_t cudaDeviceGetAttribute(int* v, enum cudaDeviceAttr a, int) {
-  *v = a == cudaDevAttrMultiProcessorCount ? 148 : (1 << 20);
+  // HEMU_SMS: fewer SMs, so that the persistent kernels' CTAs walk several work units each
+  const char* sms = std::getenv("HEMU_SMS");
+  *v = a == cudaDevAttrMultiProcessorCount ? (sms ? std::atoi(sms) : 148) : (1 << 20);
   return cudaSuccess;
 }
 cudaError_t cudaFuncSetAttribute(const void*, enum cudaFuncAttribute, int) { return cudaSuccess; }

@@ -138,16 +138,28 @@ struct HostTmap {
   const uint8_t* base;
   uint64_t inner, rows, stride;  // elements, rows, bytes per row
   uint32_t box_inner, box_rows, elem;
+  uint64_t depth = 1, stride2 = 0;  // 3-D maps: extent and byte stride of the outer dimension
+  uint32_t box_depth = 1;
 };
 static_assert(sizeof(HostTmap) <= sizeof(CUtensorMap), "tensor map model too large");
 
 inline void prefetch_tensormap(const CUtensorMap*) {}
 
-inline void tma_box_to_smem(void* dst, const CUtensorMap* map, int32_t x, int32_t y);
+inline void tma_box_to_smem(void* dst, const CUtensorMap* map, int32_t x, int32_t y, int32_t z = 0);
 inline void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y) {
   tma_box_to_smem(dst, map, x, y);
   const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
   mbar_complete_tx(bar, t->box_rows * t->box_inner * t->elem);
+}
+// 3-D box: box_depth x box_rows rows (y fastest), zero fill outside the tensor in any dimension.
+inline void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y, int32_t z) {
+  const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
+  if (t->stride2 == 0) {
+    std::fprintf(stderr, "tcsim: 3-D TMA load through a 2-D tensor map\n");
+    ++hemu::g_errors;
+  }
+  tma_box_to_smem(dst, map, x, y, z);
+  mbar_complete_tx(bar, t->box_depth * t->box_rows * t->box_inner * t->elem);
 }
 // Pair form: the box lands in this CTA's shared memory, its bytes count on the (leader's) barrier.
 inline void tma_load_2d_pair_model(void* dst, const CUtensorMap* map, uint32_t bar, int32_t x, int32_t y) {
@@ -155,7 +167,7 @@ inline void tma_load_2d_pair_model(void* dst, const CUtensorMap* map, uint32_t b
   const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
   mbar_complete_tx_cta(cluster_cta(bar), cluster_off(bar), t->box_rows * t->box_inner * t->elem);
 }
-inline void tma_box_to_smem(void* dst, const CUtensorMap* map, int32_t x, int32_t y) {
+inline void tma_box_to_smem(void* dst, const CUtensorMap* map, int32_t x, int32_t y, int32_t z) {
   const HostTmap* t = reinterpret_cast<const HostTmap*>(map);
   uint8_t* d = static_cast<uint8_t*>(dst);
   const uint32_t rb = t->box_inner * t->elem;
@@ -163,15 +175,21 @@ inline void tma_box_to_smem(void* dst, const CUtensorMap* map, int32_t x, int32_
     std::fprintf(stderr, "tcsim: TMA box of %u bytes per row / x %d not 16-byte aligned\n", rb, x);
     ++hemu::g_errors;
   }
-  for (uint32_t r = 0; r < t->box_rows; ++r) {
+  if ((smem_u32(dst) & 1023u) != 0) {
+    std::fprintf(stderr, "tcsim: 128-byte-swizzled TMA destination not 1024-byte aligned\n");
+    ++hemu::g_errors;
+  }
+  for (uint32_t r = 0; r < t->box_rows * t->box_depth; ++r) {
     uint8_t row[128];
-    const int64_t gy = static_cast<int64_t>(y) + r;
+    const int64_t gy = static_cast<int64_t>(y) + r % t->box_rows;
+    const int64_t gz = static_cast<int64_t>(z) + r / t->box_rows;
     for (uint32_t i = 0; i < t->box_inner; ++i) {
       const int64_t gx = static_cast<int64_t>(x) + i;
-      if (gy < 0 || gy >= static_cast<int64_t>(t->rows) || gx < 0 || gx >= static_cast<int64_t>(t->inner))
+      if (gy < 0 || gy >= static_cast<int64_t>(t->rows) || gx < 0 || gx >= static_cast<int64_t>(t->inner) ||
+          gz < 0 || gz >= static_cast<int64_t>(t->depth))
         std::memset(row + i * t->elem, 0, t->elem);
       else
-        std::memcpy(row + i * t->elem, t->base + gy * t->stride + gx * t->elem, t->elem);
+        std::memcpy(row + i * t->elem, t->base + gz * t->stride2 + gy * t->stride + gx * t->elem, t->elem);
     }
     const uint32_t a = smem_u32(d + r * rb);
     for (uint32_t c = 0; c < 8; ++c) std::memcpy(d + r * rb + ((c ^ ((a >> 7) & 7u)) << 4), row + c * 16, 16);

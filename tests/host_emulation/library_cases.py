@@ -17,7 +17,7 @@ from global_attention_moe_b200 import synth, workloads as W  # noqa: E402
 from decode_helpers import decode_reference  # noqa: E402
 
 TOL_MAX_ABS, TOL_REL_L2, TOL_LSE = 2e-2, 5e-3, 1e-3
-KERNEL = {"auto": 0, "simple": 1, "pipelined": 2, "window": 3}
+KERNEL = {"auto": 0, "simple": 1, "pipelined": 2, "window": 3, "packed": 4}
 DECODE = {"auto": 0, "cuda_cores": 1, "tensor": 2}
 vp = C.c_void_p
 
@@ -198,11 +198,23 @@ CASES = {
         ([300, 129, 17, 1], 8, 2, W.LAYER_SWA, 128, 1e4, True, 41), ([200, 70], 4, 2, W.LAYER_SWA, 0, 1e4, False, 42),
         ([333, 64, 5], 8, 2, W.LAYER_GLOBAL, -1, 1e7, False, 43))],
     "bwd_cuda_cores": lambda H: bwd(H, [300, 129, 17, 1], 8, 2, W.LAYER_SWA, 128, 1e4, True, 41, "cuda_cores", 1e-4),
+    # the packed window kernel (query heads of a KV group in the tile's rows): 32 tokens x 4 heads on the
+    # small config; 16 tokens x 8 heads across ragged and empty sequences, windows 0 .. 128 (run with few
+    # SMs so that each CTA walks several tiles, continuing windows and starting new ones)
+    "fwd_tiny_packed": lambda H: fwd(H, W.tiny_swa(), "packed"),
+    "fwd_packed_g8": lambda H: fwd(H, W.custom("pk8", W.LAYER_SWA, [1, 17, 129, 300, 0, 5, 160], 16, 2, 128, 1e4,
+                                               True, seed=91), "packed"),
+    "fwd_packed_windows": lambda H: [fwd(H, W.custom("pkw", W.LAYER_SWA, [250, 33], 8, 1, win, 1e4, win % 2 == 0,
+                                                     seed=92 + win), "packed") for win in (0, 1, 15, 16, 17, 127)],
+    "fwd_packed_g4_ragged": lambda H: fwd(H, W.custom("pk4", W.LAYER_SWA, [31, 32, 33, 200], 8, 2, 128, 1e4, True,
+                                                      seed=93), "packed"),
     # only for a build whose wait limit is zero
     "fwd_timeout_pipelined": lambda H: fwd_timeout(H, "pipelined"),
     "fwd_timeout_window": lambda H: fwd_timeout(H, "window"),
+    "fwd_timeout_packed": lambda H: fwd_timeout(H, "packed"),
 }
-TIMEOUT_CASES = ("fwd_timeout_pipelined", "fwd_timeout_window")
+TIMEOUT_CASES = ("fwd_timeout_pipelined", "fwd_timeout_window", "fwd_timeout_packed")
+PACKED_CASES = ("fwd_tiny_packed", "fwd_packed_g8", "fwd_packed_windows", "fwd_packed_g4_ragged")
 
 if __name__ == "__main__":
     H = Lib(sys.argv[1])

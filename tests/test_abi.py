@@ -112,9 +112,9 @@ def test_host_entry_checks_cu_seqlens_on_host(M):
 
 
 def test_kernel_choice_values(M):
-    for choice in (M.KERNEL_SIMPLE, M.KERNEL_PIPELINED, M.KERNEL_WINDOW, M.KERNEL_AUTO):
+    for choice in (M.KERNEL_SIMPLE, M.KERNEL_PIPELINED, M.KERNEL_WINDOW, M.KERNEL_WINDOW_PACKED, M.KERNEL_AUTO):
         M.set_kernel(choice)
-    for bad in (-1, 4, 99):
+    for bad in (-1, 5, 99):
         with pytest.raises(M.MimoAttnError) as e:
             M.set_kernel(bad)
         assert e.value.status == M.ERR_INVALID_ARG

@@ -19,15 +19,16 @@ def _cuda():
     assert mimo_attn.check() == mimo_attn.OK
 
 
-KERNELS = {"auto": 0, "simple": 1, "pipelined": 2, "window": 3}
+KERNELS = {"auto": 0, "simple": 1, "pipelined": 2, "window": 3, "packed": 4}
 _current = {"kernel": "auto"}
 
 
-@pytest.fixture(params=["auto", "simple", "pipelined"])
+@pytest.fixture(params=["auto", "simple", "pipelined", "window"])
 def kernel(request):
-    """Run a test with the default kernel choice (the window kernel for short
-    sliding windows, the pipelined one otherwise), with the serialised
-    cross-check kernel, and with the pipelined kernel forced."""
+    """Run a test with the default kernel choice (the packed window kernel for
+    short sliding windows at 4 or 8 query heads per KV head, the pipelined one
+    for the global layer), with the serialised cross-check kernel, and with the
+    pipelined and the two-head window kernels forced."""
     from global_attention_moe_b200 import mimo_attn
     mimo_attn.set_kernel(KERNELS[request.param])
     _current["kernel"] = request.param
@@ -43,6 +44,8 @@ def kernel_supports(name: str, w) -> bool:
         return even
     if name == "window":
         return even and w.layer_kind == W.LAYER_SWA and 0 <= w.window <= 128
+    if name == "packed":
+        return w.num_q_heads // w.num_kv_heads in (4, 8) and w.layer_kind == W.LAYER_SWA and 0 <= w.window <= 128
     return True
 
 
@@ -265,23 +268,24 @@ def test_window_kernel_windows(window, lengths):
         mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
 
 
+@pytest.mark.parametrize("pair", [("window", "pipelined"), ("packed", "pipelined")], ids=lambda p: "-".join(p))
 @pytest.mark.parametrize("name", ["swa4096", "swa_varlen", "swa_long"])
-def test_full_size_window_and_pipelined_agree_on_every_row(name):
-    """At the full workload sizes, every row of the window kernel's output
-    against the pipelined kernel's (two independently written paths with
-    different schedules, tile reuse and softmax passes)."""
+def test_full_size_window_and_pipelined_agree_on_every_row(name, pair):
+    """At the full workload sizes, every row of a window kernel's output
+    against the pipelined kernel's (independently written paths with
+    different schedules, tile shapes, K/V reuse and softmax passes)."""
     from global_attention_moe_b200 import mimo_attn
     w = W.WORKLOADS[name]()
     x = W.make_inputs(w)
     dev = to_device(x)
     res = {}
-    for kname in ("window", "pipelined"):
+    for kname in pair:
         mimo_attn.set_kernel(KERNELS[kname])
         try:
             res[kname] = run_gpu(w, x, dev_inputs=dev)
         finally:
             mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
-    (o1, l1), (o2, l2) = res["window"], res["pipelined"]
+    (o1, l1), (o2, l2) = res[pair[0]], res[pair[1]]
     a, b = o1.float(), o2.float()
     assert bool(torch.isfinite(a).all()) and bool(torch.isfinite(b).all())
     assert float((a - b).abs().max()) <= 2e-2
@@ -337,3 +341,55 @@ def test_pool_scratch_returned_after_synchronize():
     torch.cuda.synchronize()
     free1 = torch.cuda.mem_get_info()[0]
     assert free0 - free1 < 4 * 2 ** 20, (free0, free1)
+
+
+@pytest.mark.parametrize("layer,window,hq,hkv", [(W.LAYER_GLOBAL, -1, 8, 2), (W.LAYER_SWA, 129, 8, 2),
+                                                 (W.LAYER_SWA, 128, 8, 4), (W.LAYER_SWA, 128, 16, 1),
+                                                 (W.LAYER_SWA, 128, 6, 1)])
+def test_forced_packed_kernel_rejects_other_shapes(layer, window, hq, hkv):
+    """The packed window kernel takes sliding windows of at most 128 keys at 4 or 8 query heads per
+    KV head; forced on anything else the call returns UNSUPPORTED before anything is launched."""
+    from global_attention_moe_b200 import mimo_attn
+    w = W.custom("reject_packed", layer, [300], hq, hkv, window, 1e4 if layer == W.LAYER_SWA else 1e7,
+                 layer == W.LAYER_SWA, seed=19)
+    x = W.make_inputs(w)
+    dev = to_device(x)
+    mimo_attn.set_kernel(mimo_attn.KERNEL_WINDOW_PACKED)
+    try:
+        with pytest.raises(mimo_attn.MimoAttnError) as e:
+            run_gpu(w, x, dev_inputs=dev)
+        assert e.value.status == mimo_attn.ERR_UNSUPPORTED
+    finally:
+        mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
+    assert mimo_attn.check() == mimo_attn.OK
+
+
+@pytest.mark.parametrize("window", [0, 1, 15, 16, 17, 31, 64, 127, 128])
+@pytest.mark.parametrize("lengths,hq,hkv", [([1000], 8, 1), ([1, 16, 17, 128, 129, 383, 5], 16, 2),
+                                           ([31, 32, 33, 300], 8, 2)])
+def test_packed_kernel_windows(window, lengths, hq, hkv):
+    """The packed window kernel across windows that move the run across its 16-key ring slots, sequences
+    that end inside a tile and on slot edges, at 8 (16 x 8 tiles) and 4 (32 x 4) query heads per KV head."""
+    from global_attention_moe_b200 import mimo_attn
+    mimo_attn.set_kernel(mimo_attn.KERNEL_WINDOW_PACKED)
+    try:
+        _current["kernel"] = "packed"
+        full_parity(W.custom("pwin", W.LAYER_SWA, lengths, hq, hkv, window, 1e4, window % 2 == 0, seed=20))
+    finally:
+        _current["kernel"] = "auto"
+        mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)
+
+
+def test_packed_kernel_many_tiles_per_cta():
+    """Forty sequences over two KV groups with 16 query heads: every CTA walks many tiles, whose
+    windows continue the previous tile's ring or start afresh at sequence and group changes."""
+    from global_attention_moe_b200 import mimo_attn
+    rng = np.random.default_rng(21)
+    lengths = [int(v) for v in rng.integers(1, 700, size=40)]
+    mimo_attn.set_kernel(mimo_attn.KERNEL_WINDOW_PACKED)
+    try:
+        _current["kernel"] = "packed"
+        full_parity(W.custom("pmany", W.LAYER_SWA, lengths, 16, 2, 128, 1e4, True, seed=21))
+    finally:
+        _current["kernel"] = "auto"
+        mimo_attn.set_kernel(mimo_attn.KERNEL_AUTO)

@@ -15,12 +15,13 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 EMU = os.path.join(HERE, "host_emulation")
 sys.path.insert(0, EMU)
 import build_library  # noqa: E402
-from library_cases import CASES, TIMEOUT_CASES  # noqa: E402
+from library_cases import CASES, PACKED_CASES, TIMEOUT_CASES  # noqa: E402
 
 
-def run_cases(lib, names):
+def run_cases(lib, names, sms=None):
+    env = dict(os.environ, HEMU_SMS=str(sms)) if sms else None
     r = subprocess.run([sys.executable, os.path.join(EMU, "library_cases.py"), lib, *names], capture_output=True,
-                       text=True, timeout=900)
+                       text=True, timeout=900, env=env)
     return r.returncode, (r.stdout + r.stderr)[-2000:]
 
 
@@ -30,7 +31,14 @@ def host_library(tmp_path_factory):
 
 
 def test_library_matches_oracle(host_library):
-    rc, log = run_cases(host_library, [c for c in CASES if c not in TIMEOUT_CASES])
+    rc, log = run_cases(host_library, [c for c in CASES if c not in TIMEOUT_CASES + PACKED_CASES])
+    assert rc == 0, log
+
+
+def test_packed_window_kernel_matches_oracle(host_library):
+    """The packed window kernel with 5 SMs, so that each CTA walks several tiles: windows that continue
+    the previous tile's ring and windows that start afresh at sequence and KV-group changes."""
+    rc, log = run_cases(host_library, list(PACKED_CASES), sms=5)
     assert rc == 0, log
 
 
@@ -55,6 +63,14 @@ PLANTED = [
     ("backward dQ reads dS without its MN-major flag", "attn_bwd_tc.cuh",
      "kIdescDQ = make_idesc_f32acc(1, 1, 128, 192) | (1u << 15);", "kIdescDQ = make_idesc_f32acc(1, 1, 128, 192);",
      "bwd_tensor"),
+    ("packed kernel: score columns mapped to keys one ring slot off", "attn_fwd_swa_packed.cuh",
+     "const int c0 = (base + klo) % S::kN;", "const int c0 = (base + klo + kBlk) % S::kN;", "fwd_packed_g8"),
+    ("packed kernel: K rotated at the next key's position", "attn_fwd_swa_packed.cuh",
+     "* kBlk + r / 4;", "* kBlk + r / 4 + 1;", "fwd_packed_g8"),
+    ("packed kernel: PV reads the V of the slot after each P", "attn_fwd_swa_packed.cuh",
+     "v_lo + s * (kSlot >> 4)", "v_lo + ((s + 1) % S::kR) * (kSlot >> 4)", "fwd_packed_g8"),
+    ("packed kernel: a continuing window re-uses one load too few", "attn_fwd_swa_packed.cuh",
+     "new_from = max(p_blk_hi, blk_lo);", "new_from = max(p_blk_hi - 1, blk_lo);", "fwd_packed_g8"),
     ("scores read from TMEM without waiting for their MMAs", "attn_fwd_simple.cuh",
      "      fail = !mbar_wait(&bars[2], mma_phase, P.wait_limit_ns);\n      mma_phase ^= 1;\n"
      "      if (__syncthreads_or(fail)) { fail = true; break; }\n      tc_fence_after_sync();\n\n      uint32_t s[4][32];",
@@ -66,5 +82,5 @@ PLANTED = [
 @pytest.mark.parametrize("what,file,old,new,case", PLANTED, ids=[p[0] for p in PLANTED])
 def test_planted_kernel_mistake_is_caught(tmp_path, what, file, old, new, case):
     lib = build_library.build(str(tmp_path), mutations=[(file, old, new)])
-    rc, _ = run_cases(lib, [case])
+    rc, _ = run_cases(lib, [case], sms=5 if case in PACKED_CASES else None)
     assert rc != 0, f"not caught: {what}"
