@@ -121,3 +121,10 @@ def test_empty_batch():
                            z(0, 4, 128), lse, z(0, 4, 128))
     assert dq.shape == (0, 4, 192) and dk.shape == (0, 2, 192) and dv.shape == (0, 2, 128)
     assert torch.all(ds.cpu() == 0)
+
+
+def test_full_size_swa_layer():
+    """The sliding-window layer at its full size (4096 tokens, 64 query / 8 KV heads, window 128, sink)
+    against the oracle backward on every element of dq, dk, dv and dsink (the oracle's FP64 backward
+    runs single-threaded here, about a minute)."""
+    run([4096], 64, 8, W.LAYER_SWA, 128, 1e4, True, seed=47)

@@ -70,3 +70,9 @@ def test_tensor_and_cuda_core_kernels_agree():
     M.set_bwd_kernel(M.BWD_TENSOR)
     for a, b in zip(res["tensor"], res["cuda_cores"]):
         assert float((a - b).norm() / b.norm()) <= TOL_TENSOR
+
+
+def test_full_size_swa_layer():
+    """The tensor-core backward on the full-size sliding-window layer (4096 tokens, 64 query / 8 KV
+    heads, window 128, sink), every element of every gradient against the oracle."""
+    B.run([4096], 64, 8, W.LAYER_SWA, 128, 1e4, True, seed=47, tol=TOL_TENSOR)
