@@ -470,7 +470,8 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(s[q][i]));
+          for (int i = 0; i < 32; i += 2)
+            mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(s[q][i]), __uint_as_float(s[q][i + 1]));
       } else {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -496,24 +497,26 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
       const float m_new = grow ? mt : m;
       const float corr = grow ? ex2_approx(m - m_new) : 1.f;  // m = -inf -> 0
       const float base = (m_new == -INFINITY) ? 0.f : m_new;
-      // P = exp2(s * scale - m) as bf16 pairs, stored 32 keys (16 columns) at a time as S registers retire
-      float sm[8];
+      // P = exp2(s * scale - m) as bf16 pairs, stored 32 keys (16 columns) at a time as S registers retire;
+      // the scale-and-shift and the row sum run two lanes per instruction
+      const float2 sl = make_float2(sl2, sl2), nb = make_float2(-base, -base);
+      float2 sm[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) sm[k] = 0.f;
+      for (int k = 0; k < 4; ++k) sm[k] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[q][i]), sl2, -base));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[q][i + 1]), sl2, -base));
-          sm[i & 7] += p0;
-          sm[(i + 1) & 7] += p1;
+          const float2 x = ffma2(make_float2(__uint_as_float(s[q][i]), __uint_as_float(s[q][i + 1])), sl, nb);
+          const float p0 = ex2_approx(x.x);
+          const float p1 = ex2_approx(x.y);
+          sm[(i >> 1) & 3] = fadd2(sm[(i >> 1) & 3], make_float2(p0, p1));
           pk[i >> 1] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + 16 * q, pk);
       }
-      l = l * corr + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+      l = l * corr + (((sm[0].x + sm[0].y) + (sm[1].x + sm[1].y)) + ((sm[2].x + sm[2].y) + (sm[3].x + sm[3].y)));
       m = m_new;
       if (kt != kt_lo && __any_sync(0xffffffffu, grow)) {
         // rescale O; the previous PV has completed (it was issued before this tile's S)

@@ -418,16 +418,19 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
       tmem_ld32(tR + 32 * j, s);
       tmem_ld_wait(s);
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        mx[e & 7] = fmaxf(mx[e & 7], ((run >> e) & 1u) ? __uint_as_float(s[e]) : -INFINITY);
+      for (int e = 0; e < 32; e += 2)
+        mx[(e >> 1) & 7] = fmax3(mx[(e >> 1) & 7], ((run >> e) & 1u) ? __uint_as_float(s[e]) : -INFINITY,
+                                 ((run >> (e + 1)) & 1u) ? __uint_as_float(s[e + 1]) : -INFINITY);
     }
     const float mt =
         fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
     const float m = fmaxf(sink2, mt);  // log2 units
     const float mb = (m == -INFINITY) ? 0.f : m;
-    float sm[8];
+    // P = exp2(s * scale - m) (0 outside the run); scale-and-shift and row sum two lanes per instruction
+    const float2 sl = make_float2(sl2, sl2), nb = make_float2(-mb, -mb);
+    float2 sm[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) sm[k] = 0.f;
+    for (int k = 0; k < 4; ++k) sm[k] = make_float2(0.f, 0.f);
 #pragma unroll 1
     for (int j = 0; j < S::kChunks; ++j) {
       const int a = c0 - 32 * j;
@@ -437,17 +440,17 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        float p0 = ex2_approx(fmaf(__uint_as_float(s[e]), sl2, -mb));
-        float p1 = ex2_approx(fmaf(__uint_as_float(s[e + 1]), sl2, -mb));
-        p0 = ((run >> e) & 1u) ? p0 : 0.f;
-        p1 = ((run >> (e + 1)) & 1u) ? p1 : 0.f;
-        sm[e & 7] += p0;
-        sm[(e + 1) & 7] += p1;
+        const float2 x = ffma2(make_float2(((run >> e) & 1u) ? __uint_as_float(s[e]) : -INFINITY,
+                                           ((run >> (e + 1)) & 1u) ? __uint_as_float(s[e + 1]) : -INFINITY),
+                               sl, nb);
+        const float p0 = ex2_approx(x.x);  // exp2(-inf) = 0
+        const float p1 = ex2_approx(x.y);
+        sm[(e >> 1) & 3] = fadd2(sm[(e >> 1) & 3], make_float2(p0, p1));
         pk[e >> 1] = pack_bf16x2(p0, p1);
       }
       tmem_st16(tR + 16 * j, pk);  // P of the chunk's two slots, onto S columns already read
     }
-    float l = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+    float l = ((sm[0].x + sm[0].y) + (sm[1].x + sm[1].y)) + ((sm[2].x + sm[2].y) + (sm[3].x + sm[3].y));
     if (P.sink != nullptr) l += ex2_approx(sink2 - mb);
     tmem_st_wait();
     tc_fence_before_sync();

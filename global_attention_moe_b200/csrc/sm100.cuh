@@ -379,6 +379,16 @@ __device__ __forceinline__ void st_global_v8(void* dst, uint32_t a0, uint32_t a1
 }
 
 // ---------------------------------------------------------------- math helpers
+// Paired FP32 arithmetic (sm_100: one instruction for two lanes of a float2) and the three-input
+// maximum: the softmax loops issue half as many instructions for these steps.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -22,6 +22,7 @@
 #include <stdint.h>
 
 #include <chrono>
+#include <cmath>
 #include <cstdio>
 #include <unordered_map>
 #include <vector>
@@ -491,6 +492,9 @@ inline void st_global_v8(void* dst, uint32_t a0, uint32_t a1, uint32_t a2, uint3
 }
 
 // ---------------------------------------------------------------- math helpers
+inline float2 ffma2(float2 a, float2 b, float2 c) { return make_float2(std::fma(a.x, b.x, c.x), std::fma(a.y, b.y, c.y)); }
+inline float2 fadd2(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+inline float fmax3(float a, float b, float c) { return std::fmax(a, std::fmax(b, c)); }
 inline float ex2_approx(float x) { return exp2f(x); }
 inline uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
