@@ -690,8 +690,8 @@ def run_step(args):
     peaks, peak_src = load_peaks()
     kind = args.step
     tensor_bwd = kind == "bwd_tc"
-    if tensor_bwd:
-        mimo_attn.set_bwd_kernel(mimo_attn.BWD_TENSOR)
+    if kind in ("bwd", "bwd_tc"):  # bwd: the FP32 CUDA-core kernel; bwd_tc: the tensor-core one (the default)
+        mimo_attn.set_bwd_kernel(mimo_attn.BWD_TENSOR if tensor_bwd else mimo_attn.BWD_CUDA_CORES)
         kind = "bwd"
     if kind == "bwd":
         w = W.WORKLOADS["swa4096"]()

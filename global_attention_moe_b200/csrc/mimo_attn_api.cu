@@ -185,7 +185,7 @@ bool bwd_attributes_ready(int dev) {
 }
 
 std::atomic<int> g_decode_choice{MIMO_DECODE_AUTO};
-std::atomic<int> g_bwd_choice{0};  // 0 auto (CUDA cores), 1 CUDA cores, 2 tensor cores
+std::atomic<int> g_bwd_choice{0};  // 0 auto (tensor cores), 1 CUDA cores, 2 tensor cores
 
 // Persistent grid of the two-head kernels: one CTA per SM, at most one per unit.
 int persistent_grid(const FwdParams& P, int sms) {
@@ -641,7 +641,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const float* sink, c
   if (cudaMallocFromPoolAsync(&scratch, n_d * sizeof(float), info->pool, stream) != cudaSuccess) return MIMO_ERR_CUDA;
   P.D = static_cast<float*>(scratch);
   int st = MIMO_OK;
-  if (g_bwd_choice.load() == 2) {  // tensor cores: dq / dk / dv / dsink accumulate with atomics
+  if (g_bwd_choice.load() != 1) {  // tensor cores: dq / dk / dv / dsink accumulate with atomics
     const size_t T = (size_t)d->total_tokens;
     CUtensorMap tq, tk, tv, to;
     if (cudaMemsetAsync(dq, 0, T * P.hq * kHeadDimQK * 4, stream) != cudaSuccess ||

@@ -27,8 +27,40 @@ namespace nb {
 constexpr int kThreads = 256;
 
 // ---------------------------------------------------------------- FP8 dequant
-// Thread = 16 consecutive codes of one row (N % 16 == 0: 16-byte loads, 32-byte stores).
-// out = bf16_rne(decode(code) * scale_inv[block]) with the product formed exactly in FP64.
+// Thread = 16 consecutive codes of one row (N % 16 == 0: 16-byte loads, 32-byte stores), two such
+// chunks per loop trip with both loads issued first.  out = bf16_rne(decode(code) * scale_inv[block])
+// with the product formed exactly in FP64.  The row's scale block and the (at most two) column blocks
+// a chunk touches are found once per chunk (per-element index divisions dominated an earlier form).
+__device__ __forceinline__ void fp8_dequant_chunk(const uint4 u, const float* __restrict__ srow, int j0, int block_n,
+                                                  uint16_t* __restrict__ dst) {
+  const uint8_t* c = reinterpret_cast<const uint8_t*>(&u);
+  const int b0 = j0 / block_n;
+  const int edge = (b0 + 1) * block_n;  // first column of the next scale block
+  const bool one_block = j0 + 15 < edge;
+  const double s0 = static_cast<double>(__ldg(srow + b0));
+  const double s1 = one_block ? s0 : static_cast<double>(__ldg(srow + (j0 + 15) / block_n));
+  uint32_t w[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    float f[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = j0 + 2 * p + h;
+      // blocks of at least 16 columns: a chunk spans at most two; narrower blocks take the division
+      const double sc = one_block ? s0 : (block_n >= 16 ? (j < edge ? s0 : s1)
+                                                          : static_cast<double>(__ldg(srow + j / block_n)));
+      const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c[2 * p + h]), __NV_E4M3);
+      const float x = __half2float(__half(hr));
+      f[h] = __bfloat162float(__double2bfloat16(static_cast<double>(x) * sc));
+    }
+    const __nv_bfloat162 b2 = __floats2bfloat162_rn(f[0], f[1]);  // exact: both are bf16 values
+    w[p] = *reinterpret_cast<const uint32_t*>(&b2);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 __global__ void __launch_bounds__(kThreads) fp8_dequant_kernel(const uint8_t* __restrict__ codes,
                                                                const float* __restrict__ scale_inv,
                                                                uint16_t* __restrict__ out, int64_t M, int64_t N,
@@ -36,30 +68,23 @@ __global__ void __launch_bounds__(kThreads) fp8_dequant_kernel(const uint8_t* __
   const int64_t per_row = N / 16;
   const int64_t n_vec = M * per_row;
   const int64_t scale_cols = (N + block_n - 1) / block_n;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; e < n_vec;
-       e += static_cast<int64_t>(gridDim.x) * kThreads) {
-    const int64_t i = e / per_row, j0 = (e % per_row) * 16;
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(codes + i * N + j0));
-    const uint8_t* c = reinterpret_cast<const uint8_t*>(&u);
-    uint32_t w[8];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      float f[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int j = static_cast<int>(j0) + 2 * p + h;
-        const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c[2 * p + h]), __NV_E4M3);
-        const float x = __half2float(__half(hr));
-        const double s = static_cast<double>(__ldg(scale_inv + (i / block_m) * scale_cols + j / block_n));
-        const __nv_bfloat16 b = __double2bfloat16(static_cast<double>(x) * s);
-        f[h] = __bfloat162float(b);
-      }
-      const __nv_bfloat162 b2 = __floats2bfloat162_rn(f[0], f[1]);  // exact: both are bf16 values
-      w[p] = *reinterpret_cast<const uint32_t*>(&b2);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; e < n_vec; e += 2 * stride) {
+    const int64_t e2 = e + stride;
+    const bool second = e2 < n_vec;
+    const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(codes) + e);  // chunk e starts at byte 16 e
+    uint4 u1 = make_uint4(0, 0, 0, 0);
+    if (second) u1 = __ldg(reinterpret_cast<const uint4*>(codes) + e2);
+    {
+      const int64_t i = e / per_row;
+      const int j0 = static_cast<int>(e - i * per_row) * 16;
+      fp8_dequant_chunk(u0, scale_inv + (i / block_m) * scale_cols, j0, block_n, out + e * 16);
     }
-    uint4* dst = reinterpret_cast<uint4*>(out + i * N + j0);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    if (second) {
+      const int64_t i = e2 / per_row;
+      const int j0 = static_cast<int>(e2 - i * per_row) * 16;
+      fp8_dequant_chunk(u1, scale_inv + (i / block_m) * scale_cols, j0, block_n, out + e2 * 16);
+    }
   }
 }
 

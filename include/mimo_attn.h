@@ -302,7 +302,8 @@ MIMO_API int mimo_attn_decode(const void* q, const void* k_cache, const void* v_
 typedef enum { MIMO_DECODE_AUTO = 0, MIMO_DECODE_CUDA_CORES = 1, MIMO_DECODE_TENSOR = 2 } mimo_decode_choice;
 MIMO_API int mimo_attn_set_decode_kernel(int choice);
 
-/* Kernel of mimo_attn_bwd: 0 automatic (FP32 CUDA cores), 1 FP32 CUDA cores, 2 tensor cores (BF16
+/* Kernel of mimo_attn_bwd: 0 automatic (tensor cores), 1 FP32 CUDA cores (the cross-check: FP32
+ * throughout, about 4x slower on the sliding layer at 4096 tokens), 2 tensor cores (tcgen05, BF16
  * operands: the rotated Q / K dims, P and dS each rounded once to BF16).  Process-wide. */
 MIMO_API int mimo_attn_set_bwd_kernel(int choice);
 
@@ -314,8 +315,9 @@ MIMO_API int mimo_attn_set_bwd_kernel(int choice);
  * Outputs (device, fp32, overwritten): dq [T, Hq, 192], dk [T, Hkv, 192],
  * dv [T, Hkv, 128] and dsink [Hq] (required iff sink is given).  dL/ds_j =
  * P_j (dout . v_scale v_j - D + dlse) with D = dout . out; the rotation of the
- * first 64 dims is taken back by its transpose.  FP32 on the CUDA cores
- * (accumulation with atomics: the result is not bit-reproducible run to run).
+ * first 64 dims is taken back by its transpose.  By default on the tensor
+ * cores, or in FP32 on the CUDA cores (mimo_attn_set_bwd_kernel); both
+ * accumulate with atomics, so the result is not bit-reproducible run to run.
  * Scratch: Hq * T * 4 bytes from the library's pool.  Does not synchronise.
  */
 MIMO_API int mimo_attn_bwd(const void* q, const void* k, const void* v, const float* sink,

@@ -211,7 +211,9 @@ CASES = {
     "bwd_window31_mqa": lambda H: bwd(H, [90, 33], 4, 1, LAYER_SWA, 31, 1e4, True, 46),
     "bwd_global": lambda H: bwd(H, [333, 64, 5], 8, 2, LAYER_GLOBAL, -1, 1e7, False, 43),
     "bwd_no_dlse": lambda H: bwd(H, [150], 4, 4, LAYER_SWA, 128, 1e4, True, 44, dlse=False),
-    "dequant": lambda H: (dequant(H, (300, 512), (128, 128)), dequant(H, (77, 96), (32, 48))),
+    # 16-code chunks inside one scale block, across two (40-column blocks), and across several (8)
+    "dequant": lambda H: (dequant(H, (300, 512), (128, 128)), dequant(H, (77, 96), (32, 48)),
+                          dequant(H, (45, 160), (16, 40)), dequant(H, (20, 64), (3, 8))),
     "split": lambda H: (split(H, 64, 8, 33), split(H, 6, 2, 9), split(H, 8, 8, 3)),
     "route": lambda H: (route(H, 256, 8, 200), route(H, 64, 8, 33), route(H, 32, 1, 7),
                         route(H, 256, 8, 64, normalize=False), route(H, 96, 32, 40, ties=True)),

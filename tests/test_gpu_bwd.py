@@ -30,9 +30,15 @@ TOL_GPU_STATS = 2e-3
 
 
 @pytest.fixture(scope="module", autouse=True)
-def _cuda():
+def _cuda_core_kernel():
+    """This module checks the FP32 CUDA-core backward (the default is the tensor-core one, checked by
+    tests/test_gpu_bwd_tc.py with these cases at its own tolerance)."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
+    from global_attention_moe_b200 import mimo_attn as M
+    M.set_bwd_kernel(M.BWD_CUDA_CORES)
+    yield
+    M.set_bwd_kernel(M.BWD_AUTO)
 
 
 def f64_to_bf16_bits(x):

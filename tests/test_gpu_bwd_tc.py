@@ -1,4 +1,4 @@
-"""GPU parity of the tensor-core backward (mimo_attn_set_bwd_kernel(2)) against the FP64 oracle
+"""GPU parity of the tensor-core backward (the default; mimo_attn_set_bwd_kernel(2)) against the FP64 oracle
 backward, on the cases of tests/test_gpu_bwd.py and with the same dLSE shift (the kernel forms
 D = dO . out from the stored BF16 out).
 
@@ -24,6 +24,31 @@ def _tensor_kernel():
     M.set_bwd_kernel(M.BWD_TENSOR)
     yield
     M.set_bwd_kernel(M.BWD_AUTO)
+
+
+def test_default_is_the_tensor_core_kernel():
+    """BWD_AUTO runs the tensor-core kernel: its result matches the forced tensor-core kernel up to
+    the order of the atomic adds (1e-5), and differs from the FP32 CUDA-core kernel's by the BF16
+    rounding of the operands (well above 1e-4)."""
+    import numpy as np
+    from global_attention_moe_b200 import mimo_attn as M, synth
+    rng = np.random.default_rng(48)
+    T = 300
+    cu = torch.tensor([0, T], dtype=torch.int32).cuda()
+    dev = lambda a: torch.from_numpy(synth.f32_to_bf16_bits(a.astype(np.float32)).view(np.int16)).cuda().view(torch.bfloat16)
+    q, k, v = dev(rng.standard_normal((T, 4, 192))), dev(rng.standard_normal((T, 1, 192))), dev(rng.standard_normal((T, 1, 128)))
+    go = dev(rng.standard_normal((T, 4, 128)))
+    out, lse = M.fwd(q, k, v, None, cu, T, W.LAYER_SWA, 128, 1e4)
+    res = {}
+    for name, choice in (("auto", M.BWD_AUTO), ("tensor", M.BWD_TENSOR), ("cuda_cores", M.BWD_CUDA_CORES)):
+        M.set_bwd_kernel(choice)
+        res[name] = M.bwd(q, k, v, None, cu, T, W.LAYER_SWA, 128, 1e4, out, lse, go)
+        assert M.check() == M.OK
+    M.set_bwd_kernel(M.BWD_TENSOR)
+    rel = lambda a, b: float((a - b).norm() / b.norm())
+    for i in range(3):  # dq, dk, dv
+        assert rel(res["auto"][i], res["tensor"][i]) <= 1e-5
+        assert rel(res["auto"][i], res["cuda_cores"][i]) >= 1e-4
 
 
 @pytest.mark.parametrize("hq,hkv", [(8, 2), (4, 1), (4, 4)])

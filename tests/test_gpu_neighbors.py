@@ -26,7 +26,8 @@ def f64_to_bf16_bits(x):
     return (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
 
 
-@pytest.mark.parametrize("shape,block", [((300, 512), (128, 128)), ((128, 16), (128, 128)), ((77, 96), (32, 48))])
+@pytest.mark.parametrize("shape,block", [((300, 512), (128, 128)), ((128, 16), (128, 128)), ((77, 96), (32, 48)),
+                                         ((45, 160), (16, 40)), ((20, 64), (3, 8))])
 def test_fp8_dequant_bit_exact(shape, block):
     from global_attention_moe_b200 import mimo_attn as M
     rng = np.random.default_rng(51)
