@@ -68,7 +68,8 @@ constexpr uint32_t kCtrlBytes = 3072;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kRopeBarId = 1;
-constexpr uint32_t kRegsCtl = 96, kRegsSoftmax = 152, kRegsRope = 112;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8 between rescales
+constexpr uint32_t kRegsCtl = 64, kRegsSoftmax = 168, kRegsRope = 112;  // no spills in any role
 static_assert(128 * kRegsCtl + 256 * kRegsSoftmax + 128 * kRegsRope <= 65536, "register split exceeds the launch");
 
 template <int G>
@@ -102,9 +103,12 @@ struct Ctrl {
 };
 static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
 
-// Bounded wait that also gives up once another role has aborted (kept inline:
-// the roles run under different setmaxnreg budgets).
-__device__ __forceinline__ bool pk_wait_slow(Ctrl* C, uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+// Bounded wait that also gives up once another role has aborted.  The slow
+// path is out of line, one copy per role (Role is only a tag): the roles run
+// under different setmaxnreg budgets, which one shared function could not
+// satisfy, and keeping it out of the roles' loops keeps their code small.
+template <int Role>
+__device__ __noinline__ bool pk_wait_slow(Ctrl* C, uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSliceNs)) return true;
@@ -117,9 +121,10 @@ __device__ __forceinline__ bool pk_wait_slow(Ctrl* C, uint64_t* bar, uint32_t pa
   }
 }
 
+template <int Role>
 __device__ __forceinline__ bool pk_wait(Ctrl* C, uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  return pk_wait_slow(C, bar, parity, limit_ns);
+  return pk_wait_slow<Role>(C, bar, parity, limit_ns);
 }
 
 // Bits lo..hi of a 32-bit chunk (bounds relative to the chunk; empty when lo > hi).
@@ -253,7 +258,7 @@ __device__ void role_q_loader(uint8_t* smem, Ctrl* C, const CUtensorMap* tm_q, c
   TileWalk<G> W(P, C->total_tiles);
   for (uint32_t t = 0; W.next(); ++t) {
     const uint32_t buf = t & 1u;
-    if (t >= 2 && !pk_wait(C, &C->q_empty[buf], ((t >> 1) - 1) & 1u, P.wait_limit_ns)) return;
+    if (t >= 2 && !pk_wait<0>(C, &C->q_empty[buf], ((t >> 1) - 1) & 1u, P.wait_limit_ns)) return;
     mbar_arrive_expect_tx(&C->q_full[buf], 3 * kChunk);
 #pragma unroll
     for (int c = 0; c < 3; ++c)
@@ -274,7 +279,7 @@ __device__ void role_kv_loader(uint8_t* smem, Ctrl* C, const CUtensorMap* tm_k, 
 #pragma unroll 1
     for (uint32_t n = W.n_new; n < W.n_hi; ++n) {
       const uint32_t s = n % S::kR;
-      if (n >= S::kR && !pk_wait(C, &C->k_empty[s], ((n / S::kR) - 1) & 1u, lim)) return;
+      if (n >= S::kR && !pk_wait<1>(C, &C->k_empty[s], ((n / S::kR) - 1) & 1u, lim)) return;
       const int row = W.s_b + (W.blk_lo + static_cast<int>(n - W.n_lo)) * kBlk;
       mbar_arrive_expect_tx(&C->k_full[s], 3 * kSlot);
 #pragma unroll
@@ -284,7 +289,7 @@ __device__ void role_kv_loader(uint8_t* smem, Ctrl* C, const CUtensorMap* tm_k, 
 #pragma unroll 1
     for (uint32_t n = W.n_new; n < W.n_hi; ++n) {
       const uint32_t s = n % S::kR;
-      if (n >= S::kR && !pk_wait(C, &C->v_empty[s], ((n / S::kR) - 1) & 1u, lim)) return;
+      if (n >= S::kR && !pk_wait<1>(C, &C->v_empty[s], ((n / S::kR) - 1) & 1u, lim)) return;
       const int row = W.s_b + (W.blk_lo + static_cast<int>(n - W.n_lo)) * kBlk;
       mbar_arrive_expect_tx(&C->v_full[s], 2 * kSlot);
 #pragma unroll
@@ -341,11 +346,11 @@ __device__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, const FwdParams&
   for (uint32_t t = 0; has; ++t) {
     const uint32_t buf = t & 1u;
     const bool has_next = Wn.next();  // Wn: the tile after t
-    if (!pk_wait(C, &C->q_ready[buf], (t >> 1) & 1u, lim)) return;
-    if (t >= 2 && !pk_wait(C, &C->o_empty[buf], ((t >> 1) - 1) & 1u, lim)) return;
+    if (!pk_wait<2>(C, &C->q_ready[buf], (t >> 1) & 1u, lim)) return;
+    if (t >= 2 && !pk_wait<2>(C, &C->o_empty[buf], ((t >> 1) - 1) & 1u, lim)) return;
 #pragma unroll 1
     for (uint32_t n = W.n_new; n < W.n_hi; ++n)
-      if (!pk_wait(C, &C->k_ready[n % S::kR], (n / S::kR) & 1u, lim)) return;
+      if (!pk_wait<2>(C, &C->k_ready[n % S::kR], (n / S::kR) & 1u, lim)) return;
     tc_fence_after_sync();
     issue_s<G>(tmem + buf * kRegion, q_lo + buf * 3 * (kChunk >> 4), k_lo);
     tc_commit(&C->s_full[buf]);
@@ -356,10 +361,10 @@ __device__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, const FwdParams&
     for (uint32_t n = W.n_lo; n < k_dead_hi; ++n) tc_commit(&C->k_empty[n % S::kR]);
     if (t >= 1) {  // PV of the previous tile
       const uint32_t pbuf = buf ^ 1u;
-      if (!pk_wait(C, &C->p_full[pbuf], ((t - 1) >> 1) & 1u, lim)) return;
+      if (!pk_wait<2>(C, &C->p_full[pbuf], ((t - 1) >> 1) & 1u, lim)) return;
 #pragma unroll 1
       for (uint32_t n = max(v_wait, p_lo); n < p_hi; ++n)
-        if (!pk_wait(C, &C->v_full[n % S::kR], (n / S::kR) & 1u, lim)) return;
+        if (!pk_wait<2>(C, &C->v_full[n % S::kR], (n / S::kR) & 1u, lim)) return;
       v_wait = p_hi;
       tc_fence_after_sync();
       issue_pv<G>(tmem + pbuf * kRegion, v_lo, p_lo, p_hi);
@@ -370,10 +375,10 @@ __device__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, const FwdParams&
     p_lo = W.n_lo;
     p_hi = W.n_hi;
     if (!has_next) {  // PV of the last tile
-      if (!pk_wait(C, &C->p_full[buf], (t >> 1) & 1u, lim)) return;
+      if (!pk_wait<2>(C, &C->p_full[buf], (t >> 1) & 1u, lim)) return;
 #pragma unroll 1
       for (uint32_t n = max(v_wait, p_lo); n < p_hi; ++n)
-        if (!pk_wait(C, &C->v_full[n % S::kR], (n / S::kR) & 1u, lim)) return;
+        if (!pk_wait<2>(C, &C->v_full[n % S::kR], (n / S::kR) & 1u, lim)) return;
       tc_fence_after_sync();
       issue_pv<G>(tmem + buf * kRegion, v_lo, p_lo, p_hi);
       tc_commit(&C->o_full[buf]);
@@ -383,7 +388,10 @@ __device__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, const FwdParams&
   }
 }
 
-// Softmax + epilogue of the tiles with parity hw; thread r of the warpgroup owns MMA row r.
+// Softmax + epilogue of the tiles with parity hw; thread r of the warpgroup owns MMA row r.  One
+// pass over the score columns (one TMEM load per 32 columns): the row's run of allowed keys is
+// selected (others become -inf), and P = exp2(s * scale - m) is formed against a running max m that
+// is updated lazily (P stays below 2^8).
 template <int G>
 __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw, int r, int wq) {
   using S = Shape<G>;
@@ -405,29 +413,13 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
     float sink2 = -INFINITY;
     if (P.sink != nullptr) sink2 = (P.hq <= kMaxStagedSinks ? C->sink[head] : __ldg(P.sink + head)) * kLog2e;
 
-    if (!pk_wait(C, &C->s_full[hw], (t >> 1) & 1u, lim)) return;
+    if (!pk_wait<3>(C, &C->s_full[hw], (t >> 1) & 1u, lim)) return;
     tc_fence_after_sync();
-    uint32_t s[32];
-    float mx[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
-#pragma unroll 1
-    for (int j = 0; j < S::kChunks; ++j) {
-      const int a = c0 - 32 * j;
-      const uint32_t run = bits(a, a + len - 1) | bits(a - S::kN, a - S::kN + len - 1);
-      tmem_ld32(tR + 32 * j, s);
-      tmem_ld_wait(s);
-#pragma unroll
-      for (int e = 0; e < 32; e += 2)
-        mx[(e >> 1) & 7] = fmax3(mx[(e >> 1) & 7], ((run >> e) & 1u) ? __uint_as_float(s[e]) : -INFINITY,
-                                 ((run >> (e + 1)) & 1u) ? __uint_as_float(s[e + 1]) : -INFINITY);
-    }
-    const float mt =
-        fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-    const float m = fmaxf(sink2, mt);  // log2 units
-    const float mb = (m == -INFINITY) ? 0.f : m;
-    // P = exp2(s * scale - m) (0 outside the run); scale-and-shift and row sum two lanes per instruction
-    const float2 sl = make_float2(sl2, sl2), nb = make_float2(-mb, -mb);
+    // One pass over S with a lazily updated running max m (log2 units): P = exp2(s * scale - m) stays
+    // below 2^8, and when a chunk's max passes m + 8 the P columns already written (a rare event)
+    // are scaled down to the new m before going on.  The sink starts the running max and sum.
+    float m = sink2, l = (P.sink != nullptr) ? 1.f : 0.f;
+    const float2 sl = make_float2(sl2, sl2);
     float2 sm[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) sm[k] = make_float2(0.f, 0.f);
@@ -435,29 +427,60 @@ __device__ void role_softmax(Ctrl* C, uint32_t tmem, const FwdParams& P, int hw,
     for (int j = 0; j < S::kChunks; ++j) {
       const int a = c0 - 32 * j;
       const uint32_t run = bits(a, a + len - 1) | bits(a - S::kN, a - S::kN + len - 1);
+      uint32_t s[32];
       tmem_ld32(tR + 32 * j, s);
       tmem_ld_wait(s);
+      float mx[8];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const float v0 = ((run >> e) & 1u) ? __uint_as_float(s[e]) : -INFINITY;
+        const float v1 = ((run >> (e + 1)) & 1u) ? __uint_as_float(s[e + 1]) : -INFINITY;
+        s[e] = __float_as_uint(v0);
+        s[e + 1] = __float_as_uint(v1);
+        mx[(e >> 1) & 7] = (e < 16) ? fmaxf(v0, v1) : fmax3(mx[(e >> 1) & 7], v0, v1);
+      }
+      const float cm = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
+      const bool grow = cm > m + kRescaleThreshold;
+      if (__any_sync(0xffffffffu, grow)) {  // warp-uniform: TMEM access is warp-collective
+        const float m_new = grow ? cm : m;
+        const float corr = grow ? ex2_approx(m - m_new) : 1.f;  // m = -inf -> 0
+        l *= corr;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sm[k] = make_float2(sm[k].x * corr, sm[k].y * corr);
+#pragma unroll 1
+        for (int jj = 0; jj < j; ++jj) {  // P columns written so far
+          uint32_t pk[16];
+          tmem_ld16(tR + 16 * jj, pk);
+          tmem_ld16_wait(pk);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 f = unpack_bf16x2(pk[e]);
+            pk[e] = pack_bf16x2(f.x * corr, f.y * corr);
+          }
+          tmem_st16(tR + 16 * jj, pk);
+        }
+        m = m_new;
+      }
+      const float mb = (m == -INFINITY) ? 0.f : m;
+      const float2 nb = make_float2(-mb, -mb);
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        const float2 x = ffma2(make_float2(((run >> e) & 1u) ? __uint_as_float(s[e]) : -INFINITY,
-                                           ((run >> (e + 1)) & 1u) ? __uint_as_float(s[e + 1]) : -INFINITY),
-                               sl, nb);
-        const float p0 = ex2_approx(x.x);  // exp2(-inf) = 0
+        const float2 x = ffma2(make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl, nb);
+        const float p0 = ex2_approx(x.x);  // exp2(-inf) = 0 outside the run
         const float p1 = ex2_approx(x.y);
         sm[(e >> 1) & 3] = fadd2(sm[(e >> 1) & 3], make_float2(p0, p1));
         pk[e >> 1] = pack_bf16x2(p0, p1);
       }
       tmem_st16(tR + 16 * j, pk);  // P of the chunk's two slots, onto S columns already read
     }
-    float l = ((sm[0].x + sm[0].y) + (sm[1].x + sm[1].y)) + ((sm[2].x + sm[2].y) + (sm[3].x + sm[3].y));
-    if (P.sink != nullptr) l += ex2_approx(sink2 - mb);
+    l += ((sm[0].x + sm[0].y) + (sm[1].x + sm[1].y)) + ((sm[2].x + sm[2].y) + (sm[3].x + sm[3].y));
     tmem_st_wait();
     tc_fence_before_sync();
     mbar_arrive(&C->p_full[hw]);
 
     // epilogue: O / l times the V scale, BF16 rows; the FP32 LSE
-    if (!pk_wait(C, &C->o_full[hw], (t >> 1) & 1u, lim)) return;
+    if (!pk_wait<3>(C, &C->o_full[hw], (t >> 1) & 1u, lim)) return;
     tc_fence_after_sync();
     uint32_t o[4][32];
 #pragma unroll
@@ -543,7 +566,7 @@ __device__ void role_rope(uint8_t* smem, Ctrl* C, const FwdParams& P, int r) {
 #pragma unroll 1
     for (uint32_t n = W.n_new; ok && n < W.n_hi; ++n) {
       const uint32_t s = n % S::kR;
-      const bool got = pk_wait(C, &C->k_full[s], (n / S::kR) & 1u, lim);
+      const bool got = pk_wait<4>(C, &C->k_full[s], (n / S::kR) & 1u, lim);
       if (got && r < 64) {
         const int pos = (W.blk_lo + static_cast<int>(n - W.n_lo)) * kBlk + r / 4;
         const float a = rope_rotate_chunk_pair(smem + S::kKOff + s * kSlot, r / 4, r % 4, pos, C->theta);
@@ -560,7 +583,7 @@ __device__ void role_rope(uint8_t* smem, Ctrl* C, const FwdParams& P, int r) {
       rope_sincos(W.i * S::kQT, C->theta[r], sn, cs);
       C->base_q[r] = make_float2(cs, sn);
     }
-    const bool got = pk_wait(C, &C->q_full[buf], (t >> 1) & 1u, lim);
+    const bool got = pk_wait<4>(C, &C->q_full[buf], (t >> 1) & 1u, lim);
     named_bar_sync(kRopeBarId, 128);  // base_q written
     if (got) {
       const float a = rope_q_row(smem + S::kQOff + 3 * buf * kChunk, r, C->base_q, oc, os);

@@ -462,6 +462,12 @@ inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   for (int j = 0; j < 32; ++j) r[j] = g_tmem_all[hemu::g_cur_cta][lane][col + j];
 }
 inline void tmem_ld_wait(uint32_t (&)[32]) {}
+inline void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  tmem_lane_check(taddr);
+  const uint32_t lane = (taddr >> 16) + hemu::lin_tid() % 32, col = taddr & 0xFFFFu;
+  for (int j = 0; j < 16; ++j) r[j] = g_tmem_all[hemu::g_cur_cta][lane][col + j];
+}
+inline void tmem_ld16_wait(uint32_t (&)[16]) {}
 inline void reg_fence(uint32_t (&)[32]) {}
 inline void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   tmem_lane_check(taddr);
@@ -496,6 +502,13 @@ inline float2 ffma2(float2 a, float2 b, float2 c) { return make_float2(std::fma(
 inline float2 fadd2(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
 inline float fmax3(float a, float b, float c) { return std::fmax(a, std::fmax(b, c)); }
 inline float ex2_approx(float x) { return exp2f(x); }
+inline float2 unpack_bf16x2(uint32_t w) {
+  const uint32_t lo = w << 16, hi = w & 0xffff0000u;
+  float a, b;
+  std::memcpy(&a, &lo, 4);
+  std::memcpy(&b, &hi, 4);
+  return make_float2(a, b);
+}
 inline uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   uint32_t u;

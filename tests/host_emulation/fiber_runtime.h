@@ -40,6 +40,8 @@
 #undef __host__
 #define __host__
 #define __launch_bounds__(...)
+#undef __noinline__
+#define __noinline__
 #define __cluster_dims__(...)
 #define __grid_constant__
 #undef __shared__

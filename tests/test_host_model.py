@@ -42,6 +42,28 @@ def test_packed_window_kernel_matches_oracle(host_library):
     assert rc == 0, log
 
 
+def test_packed_window_kernel_rescale_path(tmp_path):
+    """The packed kernel's softmax keeps a lazily updated running max and rescales the P it has
+    already written when a later score chunk passes it by more than the threshold -- rare with these
+    inputs.  A build with threshold 0 rescales at every increase of the running max: the results
+    must still match the oracle."""
+    lib = build_library.build(str(tmp_path), mutations=[(
+        "attn_fwd_swa_packed.cuh", "constexpr float kRescaleThreshold = 8.0f;",
+        "constexpr float kRescaleThreshold = 0.0f;")])
+    rc, log = run_cases(lib, list(PACKED_CASES), sms=5)
+    assert rc == 0, log
+
+
+def test_packed_window_kernel_rescale_mistake_is_caught(tmp_path):
+    """The same threshold-0 build with the rescale of written P left out must fail."""
+    lib = build_library.build(str(tmp_path), mutations=[
+        ("attn_fwd_swa_packed.cuh", "constexpr float kRescaleThreshold = 8.0f;",
+         "constexpr float kRescaleThreshold = 0.0f;"),
+        ("attn_fwd_swa_packed.cuh", "pk[e] = pack_bf16x2(f.x * corr, f.y * corr);", "pk[e] = pack_bf16x2(f.x, f.y);")])
+    rc, _ = run_cases(lib, ["fwd_packed_windows"], sms=5)
+    assert rc != 0, "not caught: written P not rescaled when the running max grows"
+
+
 def test_timed_out_waits_end_cleanly(tmp_path):
     """A build whose bounded waits have a zero limit: the forward kernels' roles give up on each other,
     record a timeout and leave without a deadlock or a warp-collective instruction with exited lanes."""
