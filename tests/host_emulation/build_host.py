@@ -20,7 +20,7 @@ CS = os.path.join(ROOT, "global_attention_moe_b200", "csrc")
 SMS = 148  # grid sizes of the grid-stride kernels follow the B200's SM count
 
 ENTRY_POINTS = ("mimo_attn_bwd", "mimo_fp8_dequant_blockwise", "mimo_qkv_split", "mimo_moe_route",
-                "mimo_attn_decode", "mimo_attn_set_decode_kernel")
+                "mimo_attn_decode", "mimo_attn_set_decode_kernel", "mimo_attn_set_bwd_kernel")
 
 
 def _read(name):

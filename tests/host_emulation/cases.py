@@ -59,6 +59,8 @@ class Host:
         L.mimo_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, C.POINTER(DecodeDims), C.c_int, C.c_int,
                                        C.c_double, C.c_int, C.c_float, vp, vp, vp]
         L.mimo_attn_set_decode_kernel.argtypes = [C.c_int]
+        L.mimo_attn_set_bwd_kernel.argtypes = [C.c_int]
+        assert L.mimo_attn_set_bwd_kernel(1) == 0  # the CUDA-core backward: the one this library holds
         self.live = []
 
     def put(self, a):
