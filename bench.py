@@ -39,10 +39,14 @@ from global_attention_moe_b200 import workloads as W  # noqa: E402
 METRIC = "attn fwd tokens/s and TFLOP/s on 1 B200 (SWA-sink and global); % of roofline"
 L2_BYTES = 126 * 2 ** 20
 FLOPS_PER_PAIR = 2 * 192 + 2 * 128
-# Device code of the two-head kernels: the traffic recorded in profiles/traffic.json is valid
-# only while these files are unchanged.
-KERNEL_SOURCES = ["csrc/sm100.cuh", "csrc/rope_smem.cuh", "csrc/params.cuh", "csrc/rope_k_prepass.cuh",
-                  "csrc/attn_fwd_pipelined.cuh", "csrc/attn_fwd_swa.cuh", "csrc/attn_fwd_swa_packed.cuh"]
+# Device code of each forward kernel: the traffic recorded in profiles/traffic.json for a kernel is
+# valid only while its files are unchanged.
+_COMMON_SOURCES = ["csrc/sm100.cuh", "csrc/rope_smem.cuh", "csrc/params.cuh"]
+KERNEL_SOURCES = {
+    "attn_fwd_pipelined_kernel": _COMMON_SOURCES + ["csrc/attn_fwd_pipelined.cuh"],
+    "attn_fwd_swa_kernel": _COMMON_SOURCES + ["csrc/rope_k_prepass.cuh", "csrc/attn_fwd_swa.cuh"],
+    "attn_fwd_swa_packed_kernel": _COMMON_SOURCES + ["csrc/attn_fwd_swa_packed.cuh"],
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -105,9 +109,9 @@ def dominant_kernel(w) -> str:
     return "attn_fwd_pipelined_kernel"
 
 
-def kernel_sources_sha() -> str:
+def kernel_sources_sha(kernel: str) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "global_attention_moe_b200", rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -122,7 +126,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel, {}).get(workload)
-    if not e or e.get("sources_sha") != kernel_sources_sha():
+    if not e or kernel not in KERNEL_SOURCES or e.get("sources_sha") != kernel_sources_sha(kernel):
         return None
     return float(e["dram_bytes_per_launch"])
 

@@ -12,10 +12,11 @@
 //     dV += P^T dO and dK~ += dS^T Q~ accumulate in TMEM (columns 192..319, 320..511) across the
 //     query tiles: A = P / dS K-major (rows = keys), B = dO / Q~ MN-major (their row-major tiles);
 //     dQ~ = dS K~ for this query tile (columns 0..191, reusing S / dP): A = the same dS buffer read
-//     MN-major (M = queries), B = K~ MN-major; each query row adds R(-pos) scale dQ~ to dq with FP32
-//     atomics (other key tiles add theirs).
-//   at the end each key row adds v_scale dV and R(-pos) scale dK~ to dv / dk with FP32 atomics (the
-//   query heads of a KV group add to the same rows).
+//     MN-major (M = queries), B = K~ MN-major; the tile's R(-pos) scale dQ~ rows are staged in shared
+//     memory and added to dq with 16-byte vector reductions along each row (other key tiles add
+//     theirs).
+//   at the end v_scale dV and R(-pos) scale dK~ of the key rows are added to dv / dk the same way
+//   (the query heads of a KV group add to the same rows).
 // The rotated Q / K dims enter the MMAs as BF16 (one rounding of the rotation), P and dS as BF16.
 // bwdtc_prep_kernel: D - dLSE per (token, head) and the sink gradient (dq, dk, dv, dsink zeroed by
 // the host before).  The work is serialised inside a CTA (load, MMA, softmax-side math, MMA);
@@ -41,6 +42,12 @@ constexpr uint32_t kOffS = 12 * kBox;       // dS^T [keys][queries]: 2 boxes
 constexpr uint32_t kOffRow = 14 * kBox;     // lse (log2 units) [128], D - dLSE [128]
 constexpr uint32_t kOffBar = kOffRow + 1024;
 constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;  // + slack to align the base to 1024
+// Gradient rows staged for the vector reductions: row per thread, 4 floats of padding per row (so the
+// threads' 16-byte writes spread over the banks), over the Q / dO / P boxes (free once the MMAs that
+// read them have completed).
+constexpr uint32_t kOffStage = kOffQ;
+constexpr int kStrideQK = kHeadDimQK + 4, kStrideV = kHeadDimV + 4;
+static_assert(kOffStage + 128 * kStrideQK * 4 <= kOffS, "staging overlaps dS");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 64, kColDQ = 0, kColDV = 192, kColDK = 320;
 constexpr uint32_t kIdescS = make_idesc_f32acc(1, 0, 128, 64);       // S^T / dP^T halves
@@ -80,6 +87,57 @@ __device__ __forceinline__ void store_chunk(uint8_t* box, int r, int q8, const u
 }
 
 __device__ __forceinline__ uint64_t desc(uint32_t saddr, uint32_t lbo) { return sdesc_sw128(saddr, lbo, 1024); }
+
+// Row r of a staged tile (kCols floats, stride kCols + 4): the thread that owns the row writes it
+// 4 floats at a time.
+template <int kCols>
+__device__ __forceinline__ void stage4(float* stage, int r, int c4, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(stage + r * (kCols + 4) + 4 * c4) = make_float4(a, b, c, d);
+}
+
+// Adds the first nrows staged rows to global rows dst0 + r * row_stride: warp w takes rows w, w + 4,
+// ..., its lanes 16-byte pieces of the row, so each reduction instruction covers consecutive floats.
+template <int kCols>
+__device__ __forceinline__ void flush_rows(const float* stage, int nrows, float* dst0, size_t row_stride, int warp,
+                                           int lane) {
+  for (int r = warp; r < nrows; r += 4) {
+    const float* src = stage + r * (kCols + 4);
+    float* dst = dst0 + r * row_stride;
+#pragma unroll
+    for (int c = lane; c < kCols / 4; c += 32) {
+      const float4 v = *reinterpret_cast<const float4*>(src + 4 * c);
+      red_add_f32x4(dst + 4 * c, v.x, v.y, v.z, v.w);
+    }
+  }
+}
+
+// Stages this thread's gradient row R(-pos) scale x (x: 6 x 32 TMEM words, the 192 Q/K dims; the
+// rotate-half pairs (i, i + 32) of the first 64 are turned back by -pos).
+__device__ __forceinline__ void stage_rotated_row(float* stage, int r, const uint32_t (&x)[6][32], int pos,
+                                                  float scale, const double* theta) {
+#pragma unroll
+  for (int c4 = 0; c4 < 8; ++c4) {
+    float lo[4], hi[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = 4 * c4 + u;
+      float sn, cs;
+      rope_sincos(pos, theta[i], sn, cs);
+      const float a = __uint_as_float(x[0][i]) * scale, b = __uint_as_float(x[1][i]) * scale;
+      lo[u] = a * cs + b * sn;
+      hi[u] = b * cs - a * sn;
+    }
+    stage4<kHeadDimQK>(stage, r, c4, lo[0], lo[1], lo[2], lo[3]);
+    stage4<kHeadDimQK>(stage, r, 8 + c4, hi[0], hi[1], hi[2], hi[3]);
+  }
+#pragma unroll
+  for (int j = 2; j < 6; ++j)
+#pragma unroll
+    for (int c4 = 0; c4 < 8; ++c4)
+      stage4<kHeadDimQK>(stage, r, 8 * j + c4, __uint_as_float(x[j][4 * c4]) * scale,
+                         __uint_as_float(x[j][4 * c4 + 1]) * scale, __uint_as_float(x[j][4 * c4 + 2]) * scale,
+                         __uint_as_float(x[j][4 * c4 + 3]) * scale);
+}
 
 }  // namespace bwdtc
 
@@ -273,7 +331,7 @@ __global__ void __launch_bounds__(bwdtc::kThreads, 1)
       mma_phase ^= 1;
       if (__syncthreads_or(fail)) { fail = true; break; }
       tc_fence_after_sync();
-      // dq for this thread's query row (TMEM lane = query): R(-pos) scale dQ~
+      // dq for the tile's query rows (TMEM lane = query): R(-pos) scale dQ~, staged then added row-wise
       {
         uint32_t r[6][32];
 #pragma unroll
@@ -281,29 +339,20 @@ __global__ void __launch_bounds__(bwdtc::kThreads, 1)
         tmem_ld_wait(r[0]);
 #pragma unroll
         for (int j = 1; j < 6; ++j) reg_fence(r[j]);
-        if (tid < nq) {
-          float* dst = P.dq + (static_cast<size_t>(s_b + q0 + tid) * P.hq + h) * kHeadDimQK;
-          const int pos = q0 + tid;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float sn, cs;
-            rope_sincos(pos, P.theta[i], sn, cs);
-            const float x = __uint_as_float(r[0][i]) * P.scale, y = __uint_as_float(r[1][i]) * P.scale;
-            atomicAdd(dst + i, x * cs + y * sn);
-            atomicAdd(dst + i + 32, y * cs - x * sn);
-          }
-#pragma unroll
-          for (int j = 2; j < 6; ++j)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) atomicAdd(dst + 32 * j + i, __uint_as_float(r[j][i]) * P.scale);
-        }
+        float* stage = reinterpret_cast<float*>(sm + kOffStage);
+        stage_rotated_row(stage, tid, r, q0 + tid, P.scale, P.theta);
+        __syncthreads();
+        flush_rows<kHeadDimQK>(stage, nq, P.dq + (static_cast<size_t>(s_b + q0) * P.hq + h) * kHeadDimQK,
+                               static_cast<size_t>(P.hq) * kHeadDimQK, warp, tid & 31);
       }
       tc_fence_before_sync();
     }
     if (fail) break;
 
-    // dV and R(-pos) scale dK~ for this thread's key row
+    // dV and R(-pos) scale dK~ of the tile's key rows, staged then added row-wise
     tc_fence_after_sync();
+    float* stage = reinterpret_cast<float*>(sm + kOffStage);
+    __syncthreads();  // every warp has read the last dq rows out of the staging area
     {
       uint32_t r[4][32];
 #pragma unroll
@@ -311,13 +360,17 @@ __global__ void __launch_bounds__(bwdtc::kThreads, 1)
       tmem_ld_wait(r[0]);
 #pragma unroll
       for (int j = 1; j < 4; ++j) reg_fence(r[j]);
-      if (tid < nk) {
-        float* dst = P.dv + (static_cast<size_t>(s_b + key) * P.hkv + g) * kHeadDimV;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) atomicAdd(dst + 32 * j + i, __uint_as_float(r[j][i]) * P.v_scale);
-      }
+        for (int c4 = 0; c4 < 8; ++c4)
+          stage4<kHeadDimV>(stage, tid, 8 * j + c4, __uint_as_float(r[j][4 * c4]) * P.v_scale,
+                            __uint_as_float(r[j][4 * c4 + 1]) * P.v_scale, __uint_as_float(r[j][4 * c4 + 2]) * P.v_scale,
+                            __uint_as_float(r[j][4 * c4 + 3]) * P.v_scale);
+      __syncthreads();
+      flush_rows<kHeadDimV>(stage, nk, P.dv + (static_cast<size_t>(s_b + k0) * P.hkv + g) * kHeadDimV,
+                            static_cast<size_t>(P.hkv) * kHeadDimV, warp, tid & 31);
+      __syncthreads();
     }
     {
       uint32_t r[6][32];
@@ -326,21 +379,10 @@ __global__ void __launch_bounds__(bwdtc::kThreads, 1)
       tmem_ld_wait(r[0]);
 #pragma unroll
       for (int j = 1; j < 6; ++j) reg_fence(r[j]);
-      if (tid < nk) {
-        float* dst = P.dk + (static_cast<size_t>(s_b + key) * P.hkv + g) * kHeadDimQK;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float sn, cs;
-          rope_sincos(key, P.theta[i], sn, cs);
-          const float x = __uint_as_float(r[0][i]) * P.scale, y = __uint_as_float(r[1][i]) * P.scale;
-          atomicAdd(dst + i, x * cs + y * sn);
-          atomicAdd(dst + i + 32, y * cs - x * sn);
-        }
-#pragma unroll
-        for (int j = 2; j < 6; ++j)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) atomicAdd(dst + 32 * j + i, __uint_as_float(r[j][i]) * P.scale);
-      }
+      stage_rotated_row(stage, tid, r, key, P.scale, P.theta);
+      __syncthreads();
+      flush_rows<kHeadDimQK>(stage, nk, P.dk + (static_cast<size_t>(s_b + k0) * P.hkv + g) * kHeadDimQK,
+                             static_cast<size_t>(P.hkv) * kHeadDimQK, warp, tid & 31);
     }
   } while (0);
 

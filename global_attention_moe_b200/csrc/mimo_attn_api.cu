@@ -923,7 +923,7 @@ int mimo_moe_route(const float* logits, const float* bias, int64_t tokens, int n
   if (!info) return MIMO_ERR_CUDA;
   const long long warps_per_cta = nb::kThreads / 32;
   const unsigned grid = (unsigned)std::min<long long>((tokens + warps_per_cta - 1) / warps_per_cta, 16LL * info->sms);
-  nb::route_kernel<8><<<grid, nb::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+  nb::route_kernel<8><<<grid, nb::kThreads, nb::kRouteSmemBytes, static_cast<cudaStream_t>(stream)>>>(
       logits, bias, ids, weights, tokens, num_experts, top_k, normalize ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }

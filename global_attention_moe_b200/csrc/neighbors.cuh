@@ -121,75 +121,202 @@ __global__ void __launch_bounds__(kThreads) qkv_split_kernel(const uint16_t* __r
 // One warp per token (E <= 256, E % 32 == 0): lane holds experts lane + 32 m.  The choice is taken on
 // FP32 keys fp32(sigmoid) + bias with the sigmoid formed in FP64; the weights are the chosen FP64
 // scores normalised in FP64, stored as FP32.
+//
+// Only the keys near the top k decide anything, so the FP64 sigmoid is formed for those alone:
+//   1. approximate keys from an FP32 sigmoid whose error is bounded (below);
+//   2. a lower bound L on the k-th largest approximate key: the k-th largest of the lanes' maxima
+//      (k of the keys are at least that);
+//   3. candidates: experts whose approximate key is at least L less the error margin.  Every
+//      expert of the exact top k is one: an expert below that has k exact keys strictly above it;
+//   4. exact keys for the candidates (FP64 sigmoid, the same expression as the exact loop), then
+//      each candidate's rank by (key descending, expert ascending).
+// A token with more than 32 candidates (many keys within the margin of L) or a NaN among them takes
+// the exact loop over all its experts, which gives the same result by definition.
+
+__device__ __forceinline__ double route_sigmoid_f64(double x) {
+  return x >= 0 ? 1.0 / (1.0 + exp(-x)) : exp(x) / (1.0 + exp(x));
+}
+
+// Approximate sigmoid: e = __expf(-|x|) is within (2 + 1.173 |x|) ulp of exp(-|x|) and
+// __fdividef within 2 ulp (CUDA's documented bounds), so the absolute error is at most
+// e (2 + 1.173 |x|) 2^-23 + 2^-24 + 2^-22 <= 2^-20.5 (e (2 + 1.173 |x|) <= 2 for all x).
+__device__ __forceinline__ float route_sigmoid_approx(float x) {
+  const float e = __expf(-fabsf(x));
+  return __fdividef(x >= 0.f ? 1.f : e, 1.f + e);
+}
+
+// The exact choice for one token over all its experts.
+template <int kMaxPerLane>
+__device__ __forceinline__ void route_token_exact(const float* __restrict__ lrow, const float* __restrict__ bias,
+                                                  int per_lane, int lane, int top_k, int normalize,
+                                                  int32_t* __restrict__ ids, float* __restrict__ weights) {
+  double sc[kMaxPerLane];
+  float key[kMaxPerLane];
+#pragma unroll
+  for (int m = 0; m < kMaxPerLane; ++m) {
+    if (m < per_lane) {
+      const int e = lane + 32 * m;
+      sc[m] = route_sigmoid_f64(static_cast<double>(__ldg(lrow + e)));
+      key[m] = static_cast<float>(sc[m]) + __ldg(bias + e);
+    } else {
+      sc[m] = 0.0;
+      key[m] = -INFINITY;
+    }
+  }
+  double chosen = 0.0, total = 0.0;
+  int my_id = -1;  // lane k keeps choice k
+  uint32_t taken = 0;
+#pragma unroll 1
+  for (int c = 0; c < top_k; ++c) {
+    // this lane's best remaining (largest key, then lowest expert)
+    float bk = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int m = 0; m < kMaxPerLane; ++m) {
+      const int e = lane + 32 * m;
+      if (m < per_lane && !((taken >> m) & 1u) && (key[m] > bk || (key[m] == bk && e < be))) {
+        bk = key[m];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+      }
+    }
+    // the owner marks it and broadcasts its score
+    double s = 0.0;
+    if ((be & 31) == lane) {
+      const int m = be >> 5;
+#pragma unroll
+      for (int mm = 0; mm < kMaxPerLane; ++mm)
+        if (mm == m) s = sc[mm];
+      taken |= 1u << m;
+    }
+    s = __shfl_sync(0xffffffffu, s, be & 31);
+    total += s;
+    if (lane == c) {
+      my_id = be;
+      chosen = s;
+    }
+  }
+  if (lane < top_k) {
+    ids[lane] = my_id;
+    weights[lane] = static_cast<float>(normalize ? chosen / total : chosen);
+  }
+}
+
 template <int kMaxPerLane>
 __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
                                                          int32_t* __restrict__ ids, float* __restrict__ weights,
                                                          int64_t T, int E, int top_k, int normalize) {
+  extern __shared__ __align__(16) float sm[];  // per warp: 32 candidates' logits, experts, exact keys
   const int lane = threadIdx.x & 31;
+  float* c_x = sm + (threadIdx.x >> 5) * 96;
+  int* c_id = reinterpret_cast<int*>(c_x + 32);
+  float* c_key = c_x + 64;
   const int per_lane = E / 32;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-  for (int64_t t = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5; t < T; t += warps) {
-    double sc[kMaxPerLane];
-    float key[kMaxPerLane];
+  float bl[kMaxPerLane], xn[kMaxPerLane];  // this lane's biases; the next token's logits
+#pragma unroll
+  for (int m = 0; m < kMaxPerLane; ++m) bl[m] = m < per_lane ? __ldg(bias + lane + 32 * m) : 0.f;
+  int64_t t = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+#pragma unroll
+  for (int m = 0; m < kMaxPerLane; ++m) xn[m] = (t < T && m < per_lane) ? __ldg(logits + t * E + lane + 32 * m) : 0.f;
+  for (; t < T; t += warps) {
+    const float* lrow = logits + t * E;
+    float x[kMaxPerLane], ka[kMaxPerLane];
+    const int64_t tn = t + warps;
 #pragma unroll
     for (int m = 0; m < kMaxPerLane; ++m) {
-      if (m < per_lane) {
-        const int e = lane + 32 * m;
-        const double x = static_cast<double>(__ldg(logits + t * E + e));
-        sc[m] = x >= 0 ? 1.0 / (1.0 + exp(-x)) : exp(x) / (1.0 + exp(x));
-        key[m] = static_cast<float>(sc[m]) + __ldg(bias + e);
-      } else {
-        sc[m] = 0.0;
-        key[m] = -INFINITY;
-      }
+      x[m] = xn[m];
+      xn[m] = (tn < T && m < per_lane) ? __ldg(logits + tn * E + lane + 32 * m) : 0.f;  // in flight meanwhile
     }
-    double chosen = 0.0, total = 0.0;
-    int my_id = -1;  // lane k keeps choice k
-    uint32_t taken = 0;
-#pragma unroll 1
-    for (int c = 0; c < top_k; ++c) {
-      // this lane's best remaining (largest key, then lowest expert)
-      float bk = -INFINITY;
-      int be = 0x7fffffff;
+    float lmax = -INFINITY;
+#pragma unroll
+    for (int m = 0; m < kMaxPerLane; ++m) {
+      ka[m] = -INFINITY;
+      if (m < per_lane) {
+        const float k = route_sigmoid_approx(x[m]) + bl[m];
+        ka[m] = (k == k) ? k : -INFINITY;  // a NaN key is never a candidate here
+      }
+      lmax = fmaxf(lmax, ka[m]);
+    }
+    // L: the k-th largest lane maximum (bitonic sort of the 32 maxima, descending)
+    float v = lmax;
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, v, stride);
+        v = (((lane & stride) == 0) == ((lane & size) == 0)) ? fmaxf(v, o) : fminf(v, o);
+      }
+    const float kth = __shfl_sync(0xffffffffu, v, top_k - 1);
+    // candidates: an exact key differs from its approximate one by at most 2^-19 + 2^-22 |key| (the
+    // sigmoid bound, the FP32 rounding of the exact sigmoid and of the sum), so twice that, with room,
+    // is the margin
+    const float cut = kth - (0x1p-17f + 0x1p-19f * fabsf(kth));
+    unsigned cand[kMaxPerLane];
+    int n_cand = 0;
+#pragma unroll
+    for (int m = 0; m < kMaxPerLane; ++m) {
+      cand[m] = __ballot_sync(0xffffffffu, ka[m] >= cut);
+      n_cand += __popc(cand[m]);
+    }
+    bool fast = n_cand >= top_k && n_cand <= 32;  // warp-uniform
+    if (fast) {
+      int at = 0;
 #pragma unroll
       for (int m = 0; m < kMaxPerLane; ++m) {
-        const int e = lane + 32 * m;
-        if (m < per_lane && !((taken >> m) & 1u) && (key[m] > bk || (key[m] == bk && e < be))) {
-          bk = key[m];
-          be = e;
+        if ((cand[m] >> lane) & 1u) {
+          const int pos = at + __popc(cand[m] & ((1u << lane) - 1u));
+          c_x[pos] = x[m];
+          c_id[pos] = lane + 32 * m;
+        }
+        at += __popc(cand[m]);
+      }
+      __syncwarp();
+      double sc = 0.0;
+      float key = -INFINITY;
+      int id = 0;
+      if (lane < n_cand) {
+        id = c_id[lane];
+        sc = route_sigmoid_f64(static_cast<double>(c_x[lane]));
+        key = static_cast<float>(sc) + __ldg(bias + id);  // as in the exact loop
+        c_key[lane] = key;
+      }
+      __syncwarp();
+      fast = !__any_sync(0xffffffffu, lane < n_cand && key != key);
+      if (fast) {
+        int rank = 0;
+        if (lane < n_cand)
+          for (int j = 0; j < n_cand; ++j) {
+            const float kj = c_key[j];
+            rank += (kj > key || (kj == key && c_id[j] < id)) ? 1 : 0;
+          }
+        const bool chosen = lane < n_cand && rank < top_k;
+        double total = chosen ? sc : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+        if (chosen) {
+          ids[t * top_k + rank] = id;
+          weights[t * top_k + rank] = static_cast<float>(normalize ? sc / total : sc);
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ok > bk || (ok == bk && oe < be)) {
-          bk = ok;
-          be = oe;
-        }
-      }
-      // the owner marks it and broadcasts its score
-      double s = 0.0;
-      if ((be & 31) == lane) {
-        const int m = be >> 5;
-#pragma unroll
-        for (int mm = 0; mm < kMaxPerLane; ++mm)
-          if (mm == m) s = sc[mm];
-        taken |= 1u << m;
-      }
-      s = __shfl_sync(0xffffffffu, s, be & 31);
-      total += s;
-      if (lane == c) {
-        my_id = be;
-        chosen = s;
-      }
+      __syncwarp();  // the candidate buffers are rewritten for the next token
     }
-    if (lane < top_k) {
-      ids[t * top_k + lane] = my_id;
-      weights[t * top_k + lane] = static_cast<float>(normalize ? chosen / total : chosen);
-    }
+    if (!fast)
+      route_token_exact<kMaxPerLane>(lrow, bias, per_lane, lane, top_k, normalize, ids + t * top_k,
+                                     weights + t * top_k);
   }
 }
+
+// Dynamic shared memory of route_kernel: per warp 32 logits, 32 expert indices and 32 keys.
+constexpr uint32_t kRouteSmemBytes = (kThreads / 32) * 96 * 4;
 
 }  // namespace nb
 }  // namespace mimo

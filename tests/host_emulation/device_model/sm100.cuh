@@ -24,6 +24,7 @@
 #include <chrono>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <unordered_map>
 #include <vector>
 
@@ -495,6 +496,17 @@ inline void st_global_v8(void* dst, uint32_t a0, uint32_t a1, uint32_t a2, uint3
                          uint32_t a6, uint32_t a7) {
   const uint32_t v[8] = {a0, a1, a2, a3, a4, a5, a6, a7};
   std::memcpy(dst, v, 32);
+}
+
+inline void red_add_f32x4(float* p, float a, float b, float c, float d) {
+  if (reinterpret_cast<uintptr_t>(p) & 15u) {
+    std::fprintf(stderr, "emu: vector reduction at a misaligned address\n");
+    std::abort();
+  }
+  p[0] += a;
+  p[1] += b;
+  p[2] += c;
+  p[3] += d;
 }
 
 // ---------------------------------------------------------------- math helpers

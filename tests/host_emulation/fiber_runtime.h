@@ -386,6 +386,20 @@ inline bool __any_sync(unsigned, int pred) {
   hemu::syncwarp();
   return r;
 }
+inline unsigned __ballot_sync(unsigned, int pred) {
+  const int l = hemu::lin_tid() % 32, w = hemu::warp_slot();
+  hemu::g_xch[w][l] = pred != 0;
+  hemu::syncwarp();
+  unsigned r = 0;
+  for (int i = 0; i < 32; ++i) r |= (hemu::g_xch[w][i] != 0 ? 1u : 0u) << i;
+  hemu::syncwarp();
+  return r;
+}
+inline int __popc(unsigned v) { return __builtin_popcount(v); }
+inline int __ffs(unsigned v) { return __builtin_ffs(static_cast<int>(v)); }
+inline float __fdiv_rn(float a, float b) { return a / b; }
+inline float __fdividef(float a, float b) { return a / b; }
+inline float __expf(float x) { return std::exp(x); }
 inline int __syncthreads_or(int pred) { return hemu::syncthreads_or(pred != 0); }
 inline uint32_t __float_as_uint(float f) {
   uint32_t u;

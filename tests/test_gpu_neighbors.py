@@ -107,6 +107,30 @@ def test_route_exact_ties_take_lower_experts():
     assert np.allclose(w.cpu().numpy(), 1.0 / 8, rtol=0, atol=1e-7)
 
 
+@pytest.mark.parametrize("E,k", [(256, 8), (64, 32)])
+def test_route_tied_pairs(E, k):
+    """Every key twice (experts e and e + E/2 share logit and bias): the top k are pairs of exact
+    ties, each ordered by the lower expert first, and the ids match the oracle row for row."""
+    from global_attention_moe_b200 import mimo_attn as M
+    rng = np.random.default_rng(57)
+    logits = (rng.standard_normal((300, E)) * 2).astype(np.float32)
+    logits[:, E // 2:] = logits[:, :E // 2]
+    bias = (rng.standard_normal(E) * 0.1).astype(np.float32)
+    bias[E // 2:] = bias[:E // 2]
+    ids, w = M.moe_route(torch.from_numpy(logits).cuda(), torch.from_numpy(bias).cuda(), k)
+    assert M.check() == M.OK
+    ids, w = ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+    rid, rw, key = NB.route(logits, bias, k)
+    same = np.all(ids == rid, axis=1)
+    assert same.mean() > 0.99
+    assert np.max(np.abs(w[same] - rw[same])) <= 1e-6
+    for t in range(len(ids)):  # within every pair of equal keys the lower expert comes first
+        kk = key[t, ids[t]]
+        for a in range(k - 1):
+            if kk[a] == kk[a + 1]:
+                assert ids[t, a] < ids[t, a + 1]
+
+
 def test_empty_inputs():
     """Zero tokens / rows: nothing to launch, empty results."""
     from global_attention_moe_b200 import mimo_attn as M

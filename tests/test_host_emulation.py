@@ -46,6 +46,10 @@ PLANTED = [
      "    for (int e = tid; e < kChunk * (kRopeDims / 2); e += kThreads) {", "bwd_window0"),
     ("window mask one key short", "pos - kpos <= P.window", "pos - kpos < P.window", "bwd_window31_mqa"),
     ("router ties to the higher expert", "(ok == bk && oe < be)", "(ok == bk && oe > be)", "route"),
+    ("router ranks tied candidates by the higher expert", "(kj == key && c_id[j] < id)",
+     "(kj == key && c_id[j] > id)", "route"),
+    ("router candidates all written to the first slot", "const int pos = at + __popc(cand[m] & ((1u << lane) - 1u));",
+     "const int pos = at;", "route"),
     ("decode row tiles all start at row 0", "const int row0 = kMaxRows * qt;", "const int row0 = 0;",
      "decode_tiles_swa"),
     ("decode combine reads splits before the tile's keys", "const int s_lo = (lo_t - lo) / P.split_keys,",
