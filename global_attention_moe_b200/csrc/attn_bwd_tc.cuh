@@ -141,29 +141,33 @@ __device__ __forceinline__ void stage_rotated_row(float* stage, int r, const uin
 
 }  // namespace bwdtc
 
-// D - dLSE per (token, head) into P.D, and dL/dsink_h += exp(sigma_h - lse)(dLSE - D).
+// D - dLSE per (token, head) into P.D, and dL/dsink_h += exp(sigma_h - lse)(dLSE - D).  Work items are
+// (head, token stride class): a warp keeps one head, sums its tokens' sink terms in a register and adds
+// them with one atomic per item (atomics per token and head would all land on Hq addresses).
 __global__ void __launch_bounds__(256) bwdtc_prep_kernel(const __grid_constant__ bwd::BwdParams P) {
-  const long long gtid = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
-  const long long nthreads = static_cast<long long>(gridDim.x) * 256;
+  const long long warp = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  const long long nwarps = static_cast<long long>(gridDim.x) * 8;
   const long long T = P.total_tokens;
   const int lane = threadIdx.x & 31;
-  for (long long w = gtid >> 5; w < T * P.hq; w += nthreads >> 5) {
-    const long long t = w / P.hq;
-    const int h = static_cast<int>(w % P.hq);
-    const size_t base = (static_cast<size_t>(t) * P.hq + h) * kHeadDimV;
-    float acc = 0.f;
+  const long long classes = nwarps / P.hq > 0 ? nwarps / P.hq : 1;  // token stride classes per head
+  const bool sink = P.sink != nullptr && P.dsink != nullptr;
+  for (long long item = warp; item < classes * P.hq; item += nwarps) {
+    const int h = static_cast<int>(item / classes);
+    float ds = 0.f;
+    for (long long t = item % classes; t < T; t += classes) {
+      const size_t base = (static_cast<size_t>(t) * P.hq + h) * kHeadDimV;
+      float acc = 0.f;
 #pragma unroll
-    for (int d = 0; d < kHeadDimV / 32; ++d)
-      acc += bwd::bf(P.dout[base + lane + 32 * d]) * bwd::bf(P.out[base + lane + 32 * d]);
+      for (int d = 0; d < kHeadDimV / 32; ++d)
+        acc += bwd::bf(P.dout[base + lane + 32 * d]) * bwd::bf(P.out[base + lane + 32 * d]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       const size_t i = static_cast<size_t>(h) * T + t;
       const float dl = P.dlse != nullptr ? P.dlse[i] : 0.f;
-      P.D[i] = acc - dl;
-      if (P.sink != nullptr && P.dsink != nullptr)
-        atomicAdd(P.dsink + h, ex2_approx((P.sink[h] - P.lse[i]) * bwdtc::kLog2e) * (dl - acc));
+      if (lane == 0) P.D[i] = acc - dl;
+      if (sink) ds += ex2_approx((P.sink[h] - P.lse[i]) * bwdtc::kLog2e) * (dl - acc);
     }
+    if (sink && lane == 0) atomicAdd(P.dsink + h, ds);
   }
 }
 
