@@ -132,12 +132,25 @@ def bwd(H, lens, hq, hkv, layer, window, base, has_sink, seed, dlse=True):
         assert rel <= TOL_BWD, f"{name}: rel-L2 {rel:.2e}"
 
 
-def dequant(H, shape, block, seed=51):
+# Scales for the rounding of the dequant products (a product rounded to FP32 first and then to BF16
+# differs from the single rounding on the first kind).
+TIE_SCALES = np.concatenate([
+    # FP32 scales whose products with 32-45 of the E4M3 values lie just beside a BF16 midpoint, closer
+    # than half an FP32 ulp (found by comparing both roundings over 2e6 random scales)
+    np.array([1070475106, 1071501685, 1070290262, 1072649557, 1068944589, 1068420301], dtype=np.uint32)
+    .view(np.float32),
+    # products exactly on midpoints (ties to even), and far below the normal range (the FP64 path)
+    np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -9, 2.0 ** -110, 3 * 2.0 ** -112], dtype=np.float32)])
+
+
+def dequant(H, shape, block, seed=51, ties=False):
     rng = np.random.default_rng(seed)
     codes = rng.integers(0, 256, size=shape).astype(np.uint8)
     codes[(codes & 0x7F) == 0x7F] = 0x3F  # no NaN codes
     gs = (-(-shape[0] // block[0]), -(-shape[1] // block[1]))
     scale = (np.exp2(rng.integers(-8, 8, size=gs)) * rng.uniform(1, 2, size=gs)).astype(np.float32)
+    if ties:
+        scale = TIE_SCALES[rng.integers(0, len(TIE_SCALES), size=gs)]
     po = H.empty(shape, np.uint16)
     st = H.L.mimo_fp8_dequant_blockwise(H.put(codes), H.put(scale), shape[0], shape[1], block[0], block[1], po, None)
     got = H.get(po, shape, np.uint16)
@@ -218,7 +231,8 @@ CASES = {
     "bwd_no_dlse": lambda H: bwd(H, [150], 4, 4, LAYER_SWA, 128, 1e4, True, 44, dlse=False),
     # 16-code chunks inside one scale block, across two (40-column blocks), and across several (8)
     "dequant": lambda H: (dequant(H, (300, 512), (128, 128)), dequant(H, (77, 96), (32, 48)),
-                          dequant(H, (45, 160), (16, 40)), dequant(H, (20, 64), (3, 8))),
+                          dequant(H, (45, 160), (16, 40)), dequant(H, (20, 64), (3, 8)),
+                          dequant(H, (64, 256), (4, 16), ties=True), dequant(H, (40, 96), (1, 1), ties=True)),
     "split": lambda H: (split(H, 64, 8, 33), split(H, 6, 2, 9), split(H, 8, 8, 3)),
     "route": lambda H: (route(H, 256, 8, 200), route(H, 64, 8, 33), route(H, 32, 1, 7),
                         route(H, 256, 8, 64, normalize=False), route(H, 96, 32, 40, ties=True),

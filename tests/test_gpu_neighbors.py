@@ -29,12 +29,34 @@ def f64_to_bf16_bits(x):
 @pytest.mark.parametrize("shape,block", [((300, 512), (128, 128)), ((128, 16), (128, 128)), ((77, 96), (32, 48)),
                                          ((45, 160), (16, 40)), ((20, 64), (3, 8))])
 def test_fp8_dequant_bit_exact(shape, block):
+    _dequant_case(shape, block, False)
+
+
+# Scales for the rounding of the dequant products (a product rounded to FP32 first and then to BF16
+# differs from the single rounding on the first kind).
+TIE_SCALES = np.concatenate([
+    # FP32 scales whose products with 32-45 of the E4M3 values lie just beside a BF16 midpoint, closer
+    # than half an FP32 ulp (found by comparing both roundings over 2e6 random scales)
+    np.array([1070475106, 1071501685, 1070290262, 1072649557, 1068944589, 1068420301], dtype=np.uint32)
+    .view(np.float32),
+    # products exactly on midpoints (ties to even), and far below the normal range (the FP64 path)
+    np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -9, 2.0 ** -110, 3 * 2.0 ** -112], dtype=np.float32)])
+
+
+@pytest.mark.parametrize("shape,block", [((256, 512), (8, 16)), ((40, 96), (1, 1))])
+def test_fp8_dequant_rounding_midpoints(shape, block):
+    _dequant_case(shape, block, True)
+
+
+def _dequant_case(shape, block, ties):
     from global_attention_moe_b200 import mimo_attn as M
     rng = np.random.default_rng(51)
     codes = rng.integers(0, 256, size=shape).astype(np.uint8)
     codes[(codes & 0x7F) == 0x7F] = 0x3F  # no NaN codes
     gs = (-(-shape[0] // block[0]), -(-shape[1] // block[1]))
     scale = (np.exp2(rng.integers(-8, 8, size=gs)) * rng.uniform(1, 2, size=gs)).astype(np.float32)
+    if ties:
+        scale = TIE_SCALES[rng.integers(0, len(TIE_SCALES), size=gs)]
     out = M.fp8_dequant_blockwise(torch.from_numpy(codes).cuda(), torch.from_numpy(scale).cuda(), block)
     got = out.view(torch.int16).cpu().numpy().view(np.uint16)
     want = f64_to_bf16_bits(NB.dequant_fp8_blockwise(codes, scale.astype(np.float64), block))

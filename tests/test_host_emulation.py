@@ -39,6 +39,9 @@ def test_kernels_match_oracle(host_lib, mode):
 # Mistakes planted in the host copy of the kernels, each of which the cases above must catch.
 PLANTED = [
     ("one vector read past the end of the codes", "e < n_vec;", "e <= n_vec;", "dequant"),
+    ("dequant rounds the product to FP32 before BF16",
+     "f[h] = __bfloat162float(__double2bfloat16(static_cast<double>(x) * sc));",
+     "f[h] = __bfloat162float(__float2bfloat16(x * static_cast<float>(sc)));", "dequant"),
     ("shared-memory block one row-vector short", "kRows * kPS + 2 * kRows) * 4;", "kRows * kPS + kRows) * 4;",
      "bwd_window0"),
     ("barrier between the K/V load and its rotation dropped",
