@@ -227,6 +227,8 @@ int launch_packed(const void* q, const void* k, const void* v, const FwdParams& 
 struct ProfileState {
   std::mutex mu;
   bool enabled = false;
+  int stride = 1;         // record every stride-th launch
+  long long launches = 0;  // launches seen since profiling started
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pairs[64];
   size_t used[64] = {};
 };
@@ -240,6 +242,7 @@ std::pair<cudaEvent_t, cudaEvent_t>* profile_slot(int dev) {
   ProfileState& st = profile_state();
   std::lock_guard<std::mutex> lock(st.mu);
   if (!st.enabled || dev < 0 || dev >= 64) return nullptr;
+  if (st.launches++ % st.stride != 0) return nullptr;
   auto& v = st.pairs[dev];
   if (st.used[dev] == v.size()) {
     cudaEvent_t a, b;
@@ -813,10 +816,19 @@ const char* mimo_attn_status_string(int status) {
   }
 }
 
+int mimo_attn_profile_set_stride(int stride) {
+  if (stride < 1) return MIMO_ERR_INVALID_ARG;
+  ProfileState& st = profile_state();
+  std::lock_guard<std::mutex> lock(st.mu);
+  st.stride = stride;
+  return MIMO_OK;
+}
+
 int mimo_attn_profile_start(void) {
   ProfileState& st = profile_state();
   std::lock_guard<std::mutex> lock(st.mu);
   st.enabled = true;
+  st.launches = 0;
   for (auto& u : st.used) u = 0;
   return MIMO_OK;
 }

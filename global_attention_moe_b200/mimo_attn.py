@@ -21,7 +21,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BAD_
 SYMBOLS = ("mimo_attn_fwd", "mimo_attn_host_workspace_size", "mimo_attn_fwd_host", "mimo_attn_check",
            "mimo_attn_selftest_wait_timeout", "mimo_attn_status_string", "mimo_attn_fwd_noalloc",
            "mimo_attn_noalloc_scratch_bytes", "mimo_attn_set_kernel", "mimo_attn_profile_start",
-           "mimo_attn_profile_stop", "mimo_attn_decode", "mimo_attn_set_decode_kernel", "mimo_attn_version",
+           "mimo_attn_profile_stop", "mimo_attn_profile_set_stride", "mimo_attn_decode", "mimo_attn_set_decode_kernel", "mimo_attn_version",
            "mimo_attn_bwd", "mimo_fp8_dequant_blockwise", "mimo_qkv_split", "mimo_moe_route",
            "mimo_linear_proj", "mimo_attn_set_bwd_kernel")
 KERNEL_AUTO, KERNEL_SIMPLE, KERNEL_PIPELINED, KERNEL_WINDOW, KERNEL_WINDOW_PACKED = 0, 1, 2, 3, 4
@@ -71,6 +71,8 @@ def _load():
     lib.mimo_attn_noalloc_scratch_bytes.argtypes = []
     lib.mimo_attn_profile_start.restype = I
     lib.mimo_attn_profile_start.argtypes = []
+    lib.mimo_attn_profile_set_stride.restype = I
+    lib.mimo_attn_profile_set_stride.argtypes = [I]
     lib.mimo_attn_profile_stop.restype = I
     lib.mimo_attn_profile_stop.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
     lib.mimo_attn_set_kernel.restype = I
@@ -218,6 +220,13 @@ def moe_route(logits, bias, top_k=8, normalize=True, stream=None):
 def profile_start() -> None:
     """Record the attention kernel's duration on every following forward (see profile_stop)."""
     LIB.mimo_attn_profile_start()
+
+
+def profile_set_stride(stride: int) -> None:
+    """Record only every stride-th attention-kernel launch while profiling (1: every launch)."""
+    st = LIB.mimo_attn_profile_set_stride(stride)
+    if st != OK:
+        raise MimoAttnError(st, "profile_set_stride")
 
 
 def profile_stop() -> tuple[int, float]:

@@ -243,6 +243,13 @@ MIMO_API int mimo_attn_set_kernel(int choice);
  */
 MIMO_API int mimo_attn_profile_start(void);
 MIMO_API int mimo_attn_profile_stop(int* launches, double* total_ms);
+/*
+ * Records the event pair around every stride-th attention-kernel launch only
+ * (stride >= 1; 1, the default, records every launch), so that the events can
+ * sit inside a timed region with little effect on it.  The count restarts at
+ * mimo_attn_profile_start.  MIMO_ERR_INVALID_ARG for stride < 1.
+ */
+MIMO_API int mimo_attn_profile_set_stride(int stride);
 
 /*
  * Attention of new query tokens against a KV cache with page size 1: decode,

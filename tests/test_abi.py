@@ -184,3 +184,13 @@ def test_noalloc_rejects_problems_beyond_its_scratch(M):
                                      FAKE, FAKE, None)
     assert st == M.ERR_SCRATCH_LIMIT
     assert "scratch" in M.status_string(st)
+
+
+def test_profile_stride_values(M):
+    for good in (1, 16):
+        M.profile_set_stride(good)
+    for bad in (0, -3):
+        with pytest.raises(M.MimoAttnError) as e:
+            M.profile_set_stride(bad)
+        assert e.value.status == M.ERR_INVALID_ARG
+    M.profile_set_stride(1)
