@@ -35,6 +35,13 @@ def test_library_matches_oracle(host_library):
     assert rc == 0, log
 
 
+def test_backward_with_two_sms(host_library):
+    """The tensor-core backward on a 2-SM grid: the prep kernel's warps then walk many tokens of a head
+    each (several four-token trips, a ragged last one), and each SM runs many key tiles in turn."""
+    rc, log = run_cases(host_library, ["bwd_tensor"], sms=2)
+    assert rc == 0, log
+
+
 def test_packed_window_kernel_matches_oracle(host_library):
     """The packed window kernel with 5 SMs, so that each CTA walks several tiles: windows that continue
     the previous tile's ring and windows that start afresh at sequence and KV-group changes."""
