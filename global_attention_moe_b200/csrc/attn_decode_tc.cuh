@@ -33,11 +33,13 @@
 //   warp 8      TMEM owner; lane 0 issues the MMAs over the CTA's chunk stream
 //               (t counts chunks over all items):
 //               S(0) | S(1) PV(0) | S(2) PV(1) | ... | PV(T-1)
-//               so the score of the next chunk overlaps the softmax of this one
+//               so the score of the next chunk overlaps the softmax of this one; at an item
+//               boundary the previous chunk's PV goes first (the new item's S waits for its Q)
 //   warps 9-12  lander: per item, once the previous item's last S has read Q,
 //               loads and rotates the item's Q (its own cp.async groups); then,
 //               per landed chunk, rotates the first 64 dims of K at the key
-//               positions (BF16 -> FP16 in place) and signals the MMA issuer
+//               positions (BF16 -> FP16 in place; angle addition from the
+//               chunk's first position) and signals the MMA issuer
 //   warp 13     item producer (lane 0)
 // Fetching and landing are separate warps, so a chunk is signalled as soon as
 // it lands, whatever the fetcher is waiting for: chunk f waits for PV(f-4) to
@@ -103,6 +105,7 @@ struct Ctrl {
   uint64_t item_full[kRing], item_empty[kRing];
   Work ring[kRing];  // n < 0: no more items
   double theta[kRopeDims / 2];  // RoPE inverse frequencies, staged once per CTA
+  float2 k_base[2][kRopeDims / 2];  // cos / sin of theta_i x (first key position of the chunk), by chunk parity
 };
 static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
 
@@ -276,6 +279,40 @@ __device__ __forceinline__ void role_fetcher(uint8_t* smem, Ctrl* C, const dec::
   if (bad) atomicOr(&g_mimo_error, kErrSeqlens);
 }
 
+// Rotates the chunk pair (c, c + 4) of key row r of a landed stage by angles given as cos / sin pairs:
+// base[i] of the chunk's first key position and off[e] of the row's offset from it (frequencies 8c ..
+// 8c + 7), combined by angle addition.  Returns the largest |rotated value|.
+__device__ __forceinline__ float rope_rotate_chunk_pair_add(uint8_t* block, int r, int c, const float2* base,
+                                                           const float2 (&off)[8]) {
+  uint8_t* row = block + r * 128;
+  uint4* plo = reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4));
+  uint4* phi = reinterpret_cast<uint4*>(row + (((c + 4) ^ (r & 7)) << 4));
+  const uint4 lo = *plo, hi = *phi;
+  const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lo);
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hi);
+  uint4 olo, ohi;
+  __half2* ol = reinterpret_cast<__half2*>(&olo);
+  __half2* oh = reinterpret_cast<__half2*>(&ohi);
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 x = __bfloat1622float2(l2[e]);
+    const float2 y = __bfloat1622float2(h2[e]);
+    const float2 b0 = base[8 * c + 2 * e], b1 = base[8 * c + 2 * e + 1];
+    const float2 o0 = off[2 * e], o1 = off[2 * e + 1];
+    const float c0 = b0.x * o0.x - b0.y * o0.y, s0 = b0.y * o0.x + b0.x * o0.y;
+    const float c1 = b1.x * o1.x - b1.y * o1.y, s1 = b1.y * o1.x + b1.x * o1.y;
+    const float a0 = x.x * c0 - y.x * s0, d0 = y.x * c0 + x.x * s0;
+    const float a1 = x.y * c1 - y.y * s1, d1 = y.y * c1 + x.y * s1;
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(a0), fabsf(d0)), fmaxf(fabsf(a1), fabsf(d1))));
+    ol[e] = __floats2half2_rn(a0, a1);
+    oh[e] = __floats2half2_rn(d0, d1);
+  }
+  *plo = olo;
+  *phi = ohi;
+  return amax;
+}
+
 // Per item: Q (once the previous item's last S has read Q), then every chunk as it lands.
 __device__ __forceinline__ void role_lander(uint8_t* smem, Ctrl* C, const dec::DecParams& P, int qt) {
   const uint64_t lim = P.wait_limit_ns;
@@ -286,6 +323,16 @@ __device__ __forceinline__ void role_lander(uint8_t* smem, Ctrl* C, const dec::D
   float amax = 0.f;
   uint32_t landed = 0;
   bool ok = true;
+  // cos / sin of theta_i x (this thread's key row within a chunk), for its two chunk pairs' frequencies
+  float2 off[2][8];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float sn, cs;
+      rope_sincos(qt & 63, C->theta[8 * (2 * (qt >> 6) + h) + e], sn, cs);
+      off[h][e] = make_float2(cs, sn);
+    }
 #pragma unroll 1
   for (uint32_t item = 0;; ++item) {
     bool failed = false;
@@ -313,17 +360,24 @@ __device__ __forceinline__ void role_lander(uint8_t* smem, Ctrl* C, const dec::D
     for (int c = 0; c < 4; ++c) amax = fmaxf(amax, rope_rotate_chunk_pair(smem + kQOff, qt, c, pos, C->theta));
     fence_proxy_async_smem();
     mbar_arrive(&C->q_ready);
-    // the item's chunks: rotated dims of the 64 keys, two chunk pairs per thread
+    // the item's chunks: rotated dims of the 64 keys, two chunk pairs per thread, at angles
+    // base (the chunk's first key position, FP64-reduced by 32 threads per chunk) + off (the row's offset)
     const int r = qt & 63, c0 = 2 * (qt >> 6);
 #pragma unroll 1
     for (int c = 0; c < w.n; ++c, ++landed) {
       const int stage = static_cast<int>(landed % kStages);
+      float2* base = C->k_base[landed & 1];
+      if (qt < kRopeDims / 2) {
+        float sn, cs;
+        rope_sincos(w.k_beg + c * kChunk, C->theta[qt], sn, cs);
+        base[qt] = make_float2(cs, sn);
+      }
+      named_bar_sync(kQBar, 128);  // this chunk's bases written; the bases of two chunks back are read
       if (ok) ok = dwait(C, &C->landed[stage], (landed / kStages) & 1, lim);
       if (!ok) continue;  // the same trips as the others, without the work, up to the barrier above
       uint8_t* kr = smem + kStageOff + stage * kStageBytes;
-      const int kpos = w.k_beg + c * kChunk + r;
-      amax = fmaxf(amax, rope_rotate_chunk_pair(kr, r, c0, kpos, C->theta));
-      amax = fmaxf(amax, rope_rotate_chunk_pair(kr, r, c0 + 1, kpos, C->theta));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) amax = fmaxf(amax, rope_rotate_chunk_pair_add(kr, r, c0 + h, base, off[h]));
       fence_proxy_async_smem();  // the fetcher's copies and these writes, before the MMA reads the stage
       mbar_arrive(&C->full[stage]);
     }
@@ -352,6 +406,23 @@ __device__ __forceinline__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, 
       c = 0;
       if (have) ++item;
     }
+    // PV of the previous chunk; at an item boundary it goes before the new item's first score, so that
+    // the previous item's epilogue does not wait for this item's Q to load and rotate
+    auto pv_prev = [&]() -> bool {
+      const uint32_t u = t - 1;
+      const int s = static_cast<int>(u % kStages);
+      if (!dwait(C, &C->p_full[u & 1], (u >> 1) & 1, lim)) return false;
+      if (prev_first && prev_item > 1 && !dwait(C, &C->o_empty, (prev_item - 2) & 1, lim)) return false;
+      tc_fence_after_sync();
+      issue_pv_half(tmem + kColO, tmem + 64u * (u & 1),
+                    sdesc_lo(smem_u32(smem + kStageOff + s * kStageBytes + kVOff), kKUnit), prev_first);
+      tc_commit(&C->pv_done);
+      tc_commit(&C->empty[s]);
+      if (prev_last) tc_commit(&C->o_full);
+      return true;
+    };
+    const bool pv_first = prev && (!have || c == 0);
+    if (pv_first && !pv_prev()) return;
     if (have) {
       if (c == 0) {
         if (!dwait(C, &C->q_ready, (item - 1) & 1, lim)) return;
@@ -364,18 +435,7 @@ __device__ __forceinline__ void role_mma(uint8_t* smem, Ctrl* C, uint32_t tmem, 
       tc_commit(&C->s_full[t & 1]);
       if (c == w.n - 1) tc_commit(&C->q_empty);  // the item's last S has read Q
     }
-    if (prev) {
-      const uint32_t u = t - 1;
-      const int s = static_cast<int>(u % kStages);
-      if (!dwait(C, &C->p_full[u & 1], (u >> 1) & 1, lim)) return;
-      if (prev_first && prev_item > 1 && !dwait(C, &C->o_empty, (prev_item - 2) & 1, lim)) return;
-      tc_fence_after_sync();
-      issue_pv_half(tmem + kColO, tmem + 64u * (u & 1),
-                    sdesc_lo(smem_u32(smem + kStageOff + s * kStageBytes + kVOff), kKUnit), prev_first);
-      tc_commit(&C->pv_done);
-      tc_commit(&C->empty[s]);
-      if (prev_last) tc_commit(&C->o_full);
-    }
+    if (prev && !pv_first && !pv_prev()) return;
     if (!have) break;
     prev = true;
     prev_first = c == 0;

@@ -35,6 +35,16 @@ def test_library_matches_oracle(host_library):
     assert rc == 0, log
 
 
+def test_decode_kernel_with_one_and_two_sms(host_library):
+    """The persistent KV-cache kernel on 1 and 2 SMs: every CTA then takes many items in turn, so the
+    item boundaries (the previous item's last PV before the next item's first score, Q reloaded once
+    the last score has read it) and the lander's per-chunk angle tables turn over many times."""
+    for sms in (1, 2):
+        rc, log = run_cases(host_library, ["decode_tensor", "decode_tensor_tiles_swa", "decode_tensor_tiles_global"],
+                            sms=sms)
+        assert rc == 0, log
+
+
 def test_backward_with_two_sms(host_library):
     """The tensor-core backward on a 2-SM grid: the prep kernel's warps then walk many tokens of a head
     each (several four-token trips, a ragged last one), and each SM runs many key tiles in turn."""
@@ -89,6 +99,12 @@ PLANTED = [
      "v_lo + kk * (2048 >> 4)", "v_lo + kk * (1024 >> 4)", "fwd_tiny_pipelined"),
     ("KV-cache row tiles all start at row 0", "attn_decode_tc.cuh", "w.row0 = 128 * qt;", "w.row0 = 0;",
      "decode_tensor_tiles_swa"),
+    ("KV-cache lander reads the previous chunk's angle table", "attn_decode_tc.cuh",
+     "rope_rotate_chunk_pair_add(kr, r, c0 + h, base, off[h])",
+     "rope_rotate_chunk_pair_add(kr, r, c0 + h, C->k_base[(landed + 1) & 1], off[h])",
+     "decode_tensor_tiles_global"),
+    ("KV-cache lander offsets each key row by one position too many", "attn_decode_tc.cuh",
+     "rope_sincos(qt & 63, C->theta", "rope_sincos((qt & 63) + 1, C->theta", "decode_tensor"),
     ("backward dQ reads dS without its MN-major flag", "attn_bwd_tc.cuh",
      "kIdescDQ = make_idesc_f32acc(1, 1, 128, 192) | (1u << 15);", "kIdescDQ = make_idesc_f32acc(1, 1, 128, 192);",
      "bwd_tensor"),
