@@ -47,7 +47,7 @@ def test_decode_kernel_with_one_and_two_sms(host_library):
 
 def test_backward_with_two_sms(host_library):
     """The tensor-core backward on a 2-SM grid: the prep kernel's warps then walk many tokens of a head
-    each (several four-token trips, a ragged last one), and each SM runs many key tiles in turn."""
+    each, and each SM runs many key tiles in turn."""
     rc, log = run_cases(host_library, ["bwd_tensor"], sms=2)
     assert rc == 0, log
 
@@ -79,6 +79,21 @@ def test_packed_window_kernel_rescale_mistake_is_caught(tmp_path):
         ("attn_fwd_swa_packed.cuh", "pk[e] = pack_bf16x2(f.x * corr, f.y * corr);", "pk[e] = pack_bf16x2(f.x, f.y);")])
     rc, _ = run_cases(lib, ["fwd_packed_windows"], sms=5)
     assert rc != 0, "not caught: written P not rescaled when the running max grows"
+
+
+def test_pipelined_kernel_rescale_path(tmp_path):
+    """The pipelined kernel's softmax raises its running max lazily (when a tile's max passes it by
+    more than the threshold) and then rescales O.  Under threshold 0 it rescales at every increase:
+    the results must still match the oracle, and leaving the O rescale out must not."""
+    thr = ("attn_fwd_pipelined.cuh", "constexpr float kRescaleThreshold = 8.0f;", "constexpr float kRescaleThreshold = 0.0f;")
+    cases = ["fwd_global", "fwd_tiny_pipelined"]
+    lib = build_library.build(str(tmp_path / "ok"), mutations=[thr])
+    rc, log = run_cases(lib, cases)
+    assert rc == 0, log
+    lib = build_library.build(str(tmp_path / "no_o"), mutations=[thr, (
+        "attn_fwd_pipelined.cuh", "o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);", "o[i] = o[i];")])
+    rc, _ = run_cases(lib, cases)
+    assert rc != 0, "not caught: O not rescaled"
 
 
 def test_timed_out_waits_end_cleanly(tmp_path):
