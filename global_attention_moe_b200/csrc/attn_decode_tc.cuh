@@ -541,6 +541,40 @@ __device__ __forceinline__ void role_softmax(Ctrl* C, uint32_t tmem, const dec::
     }
     if (!__all_sync(0xffffffffu, dwait(C, &C->o_full, item & 1, lim))) return;
     tc_fence_after_sync();
+    if (P.splits == 1) {
+      // One split: the item holds every key its rows see, so the row's output and LSE are final here,
+      // with the sink folded into the running max and sum as the combine kernel would (no combine).
+      const int i = (w.row0 + r) / P.group, head = w.g * P.group + (w.row0 + r) % P.group;
+      const float sg = P.sink != nullptr ? __ldg(P.sink + head) * dec::kLog2e : -INFINITY;
+      const float M = fmaxf(m, sg);
+      const float mb = (M == -INFINITY) ? 0.f : M;
+      const float wgt = ex2_approx(m - mb);  // m = -inf -> 0
+      const float L = l * wgt + (P.sink != nullptr ? ex2_approx(sg - mb) : 0.f);
+      const float scale = P.v_scale * wgt / L;
+      uint16_t* dst = valid ? P.out + (static_cast<size_t>(w.q_beg + i) * P.hq + head) * kHeadDimV : nullptr;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {  // 32 columns at a time (warp-collective loads: every row takes part)
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * q, o);
+        tmem_ld_wait(o);
+        if (valid) {
+#pragma unroll
+          for (int hv = 0; hv < 2; ++hv) {
+            uint32_t b[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              b[e] = pack_bf16x2(__uint_as_float(o[16 * hv + 2 * e]) * scale,
+                                 __uint_as_float(o[16 * hv + 2 * e + 1]) * scale);
+            st_global_v8(dst + 32 * q + 16 * hv, b[0], b[1], b[2], b[3], b[4], b[5], b[6], b[7]);
+          }
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&C->o_empty);  // the next item's first PV may overwrite O
+      if (valid) P.lse[static_cast<size_t>(head) * P.total_q + w.q_beg + i] = (M + log2f(L)) * dec::kLn2;
+      ++item;
+      continue;
+    }
     size_t slot = 0;
     float4* dst = valid ? partial_row(P, w, r, slot) : nullptr;
 #pragma unroll 1

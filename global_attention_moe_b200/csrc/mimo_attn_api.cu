@@ -79,6 +79,7 @@ bool encode_q_packed(CUtensorMap* m, const void* q, int hq, int total_tokens, in
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }  // 32-byte row stores
 
 int validate(const void* q, const void* k, const void* v, const float* sink, const int32_t* cu,
              const mimo_attn_dims* d, int layer_kind, int window, double rope_base, int rope_dims, float v_scale,
@@ -104,7 +105,7 @@ int validate(const void* q, const void* k, const void* v, const float* sink, con
   if (!cu) return MIMO_ERR_INVALID_ARG;
   if (d->total_tokens > 0) {
     if (!q || !k || !v || !out || !lse) return MIMO_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(out) || !aligned16(lse))
       return MIMO_ERR_INVALID_ARG;
   }
   if (sink && (reinterpret_cast<uintptr_t>(sink) & 3u)) return MIMO_ERR_INVALID_ARG;
@@ -513,7 +514,7 @@ int validate_decode(const void* q, const void* kc, const void* vc, const int32_t
   if (!indptr || !cu_q) return MIMO_ERR_INVALID_ARG;
   if (d->total_q > 0) {
     if (!q || !out || !lse || (d->total_kv > 0 && (!kc || !vc || !idx))) return MIMO_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || (kc && !aligned16(kc)) || (vc && !aligned16(vc)))
+    if (!aligned16(q) || !aligned32(out) || !aligned16(lse) || (kc && !aligned16(kc)) || (vc && !aligned16(vc)))
       return MIMO_ERR_INVALID_ARG;
   }
   if (sink && (reinterpret_cast<uintptr_t>(sink) & 3u)) return MIMO_ERR_INVALID_ARG;
@@ -595,7 +596,8 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
   }
   const long long warps = (long long)d->total_q * P.hq;
-  if (st == MIMO_OK) {
+  // with one key split the tensor-core kernel writes the final rows itself (no partials to merge)
+  if (st == MIMO_OK && !(tensor && splits == 1)) {
     dec::attn_decode_combine_kernel<<<(unsigned)((warps * 32 + dec::kThreads - 1) / dec::kThreads), dec::kThreads,
                                       0, stream>>>(P);
     if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;

@@ -30,7 +30,10 @@
  *   - Return values are mimo_status codes.  Argument checks happen before any
  *     CUDA call, so a rejected call has no side effect.
  *   - All tensors are dense, row-major and contiguous in THD layout
- *     (tokens, heads, dims).  Every device pointer must be 16-byte aligned.
+ *     (tokens, heads, dims).  Every device pointer must be 16-byte aligned,
+ *     and the attention output `out` of the forward and KV-cache entry
+ *     points 32-byte aligned (its rows are written with 32-byte stores);
+ *     otherwise MIMO_ERR_INVALID_ARG.
  */
 #ifndef MIMO_ATTN_H_
 #define MIMO_ATTN_H_
@@ -280,7 +283,10 @@ MIMO_API int mimo_attn_profile_set_stride(int stride);
  * recorded as MIMO_ERR_BAD_SEQLENS for mimo_attn_check (such rows are left
  * unwritten; an index outside the cache is never dereferenced).  Scratch: a
  * partial result per key split, total_q * Hq * splits * 520 bytes (plus 512
- * bytes) from the library's stream-ordered pool.  Does not synchronise.  (The pages give no
+ * bytes) from the library's stream-ordered pool; with one split (the keys a
+ * row sees fit one split: always on sliding-window layers) the tensor-core
+ * kernel writes out and lse directly and the partials go unused.  Does not
+ * synchronise.  (The pages give no
  * interface; this one mirrors mimo_attn_fwd.)
  */
 typedef struct {

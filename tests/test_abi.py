@@ -62,6 +62,7 @@ def call(M, dims, layer=0, window=128, base=1e4, rope_dims=64, sink=None, q=FAKE
     (dict(base=float("nan")), 1),
     (dict(q=FAKE + 8), 1),                          # misaligned
     (dict(out=0), 1),                               # null output
+    (dict(out=FAKE + 16), 1),                       # output rows are written with 32-byte stores
     (dict(dims=dict(num_seqs=0)), 1),
     (dict(dims=dict(max_seqlen=10 ** 6)), 1),       # max_seqlen > total tokens
 ])
@@ -142,17 +143,18 @@ def test_decode_kernel_choice_values(M):
     (dict(window=-1), 1),
     (dict(layer=1, sink=FAKE), 1),
     (dict(q=FAKE + 8), 1),
+    (dict(out=FAKE + 16), 1),               # output rows are written with 32-byte stores
 ])
 def test_decode_validation_rejects(M, case, expect):
     d = dict(num_seqs=2, total_q=4, total_kv=100, cache_rows=128, max_q_len=2, max_kv_len=60, hq=8, hkv=2,
              dqk=192, dv=128)
-    args = dict(layer=0, window=128, rope_dims=64, sink=None, q=FAKE)
+    args = dict(layer=0, window=128, rope_dims=64, sink=None, q=FAKE, out=FAKE)
     for key in list(case):
         (d if key in d else args)[key] = case[key]
     dims = M.make_decode_dims(d["num_seqs"], d["total_q"], d["total_kv"], d["cache_rows"], d["max_q_len"],
                               d["max_kv_len"], d["hq"], d["hkv"], d["dqk"], d["dv"])
     st = M.decode_raw(args["q"], FAKE, FAKE, FAKE, FAKE, FAKE, args["sink"], dims, args["layer"], args["window"],
-                      1e4, args["rope_dims"], 0.707, FAKE, FAKE, None)
+                      1e4, args["rope_dims"], 0.707, args["out"], FAKE, None)
     assert st == expect
 
 
