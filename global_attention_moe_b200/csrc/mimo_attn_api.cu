@@ -879,7 +879,7 @@ int mimo_attn_bwd(const void* q, const void* k, const void* v, const float* sink
 int mimo_fp8_dequant_blockwise(const void* codes, const float* scale_inv, int64_t rows, int64_t cols, int block_rows,
                                int block_cols, void* out, void* stream) {
   if (rows < 0 || cols < 0 || block_rows < 1 || block_cols < 1) return MIMO_ERR_INVALID_ARG;
-  if (cols % 16 != 0) return MIMO_ERR_UNSUPPORTED;
+  if (cols % 16 != 0 || cols > 0x7FFFFFFFLL) return MIMO_ERR_UNSUPPORTED;
   if (rows == 0 || cols == 0) return MIMO_OK;
   if (!codes || !scale_inv || !out || !aligned16(codes) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(scale_inv) & 3u))

@@ -27,63 +27,134 @@ namespace nb {
 constexpr int kThreads = 256;
 
 // ---------------------------------------------------------------- FP8 dequant
-// Thread = 16 consecutive codes of one row (N % 16 == 0: 16-byte loads, 32-byte stores), two such
-// chunks per loop trip with both loads issued first.  out = bf16_rne(decode(code) * scale_inv[block])
-// with the product formed exactly in FP64.  The row's scale block and the (at most two) column blocks
-// a chunk touches are found once per chunk (per-element index divisions dominated an earlier form).
-__device__ __forceinline__ void fp8_dequant_chunk(const uint4 u, const float* __restrict__ srow, int j0, int block_n,
-                                                  uint16_t* __restrict__ dst) {
-  const uint8_t* c = reinterpret_cast<const uint8_t*>(&u);
-  const int b0 = j0 / block_n;
-  const int edge = (b0 + 1) * block_n;  // first column of the next scale block
-  const bool one_block = j0 + 15 < edge;
-  const double s0 = static_cast<double>(__ldg(srow + b0));
-  const double s1 = one_block ? s0 : static_cast<double>(__ldg(srow + (j0 + 15) / block_n));
+// out = bf16_rne(decode(code) * scale_inv[block]), the exact product rounded once.  The product is
+// formed in FP32 (round to nearest) and rounded to BF16 two at a time.  Every BF16 midpoint is an
+// FP32 number, so rounding to FP32 first cannot carry the product across one: the two roundings
+// differ only when the FP32 product lands exactly on a midpoint (its low 16 bits 0x8000) without
+// being exact.  A chunk with such a product forms its products in FP64 instead.  Codes are decoded
+// through a 256-entry table in shared memory.
+
+// The scale blocks a chunk of 16 columns starting at j0 touches: b0 (and b1 when it crosses into the
+// next block at column `edge`; blocks of at least 16 columns give at most two).
+struct DequantCols {
+  int j0, b0, b1, edge;
+  bool one_block;
+};
+
+__device__ __forceinline__ DequantCols dequant_cols(int j0, int block_n) {
+  DequantCols c;
+  c.j0 = j0;
+  c.b0 = j0 / block_n;
+  c.edge = (c.b0 + 1) * block_n;
+  c.one_block = j0 + 15 < c.edge;
+  c.b1 = c.one_block ? c.b0 : (j0 + 15) / block_n;
+  return c;
+}
+
+__device__ __forceinline__ float dequant_code(const float* lut, uint32_t word, int byte) {
+  return lut[(word >> (8 * byte)) & 0xFFu];
+}
+
+// Thread = 16 consecutive codes of one row (N % 16 == 0: 16-byte loads, 32-byte stores).
+__device__ __forceinline__ void fp8_dequant_chunk(const uint4 u, const float* __restrict__ srow, const DequantCols& c,
+                                                  int block_n, const float* lut, uint16_t* __restrict__ dst) {
+  const uint32_t cw[4] = {u.x, u.y, u.z, u.w};
+  const float s0 = __ldg(srow + c.b0);
   uint32_t w[8];
+  bool mid = false;
+  if (c.one_block) {
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    float f[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int j = j0 + 2 * p + h;
-      // blocks of at least 16 columns: a chunk spans at most two; narrower blocks take the division
-      const double sc = one_block ? s0 : (block_n >= 16 ? (j < edge ? s0 : s1)
-                                                          : static_cast<double>(__ldg(srow + j / block_n)));
-      const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c[2 * p + h]), __NV_E4M3);
-      const float x = __half2float(__half(hr));
-      f[h] = __bfloat162float(__double2bfloat16(static_cast<double>(x) * sc));
+    for (int p = 0; p < 8; ++p) {
+      const float a = __fmul_rn(dequant_code(lut, cw[p >> 1], 2 * (p & 1)), s0);
+      const float b = __fmul_rn(dequant_code(lut, cw[p >> 1], 2 * (p & 1) + 1), s0);
+      mid |= (__float_as_uint(a) & 0xFFFFu) == 0x8000u;
+      mid |= (__float_as_uint(b) & 0xFFFFu) == 0x8000u;
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(a, b);
+      w[p] = *reinterpret_cast<const uint32_t*>(&b2);
     }
-    const __nv_bfloat162 b2 = __floats2bfloat162_rn(f[0], f[1]);  // exact: both are bf16 values
-    w[p] = *reinterpret_cast<const uint32_t*>(&b2);
+  } else {
+    mid = true;  // a chunk across a block edge (only with blocks that are not multiples of 16 wide)
+  }
+  if (mid) {
+    const float s1 = __ldg(srow + c.b1);
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      uint32_t h[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int jj = 2 * p + k;
+        const int j = c.j0 + jj;
+        // narrower blocks than 16 columns take the division per column
+        const float sc = c.one_block ? s0 : (block_n >= 16 ? (j < c.edge ? s0 : s1) : __ldg(srow + j / block_n));
+        const __nv_bfloat16 r = __double2bfloat16(static_cast<double>(dequant_code(lut, cw[jj >> 2], jj & 3)) *
+                                                  static_cast<double>(sc));
+        h[k] = *reinterpret_cast<const uint16_t*>(&r);
+      }
+      w[p] = h[0] | (h[1] << 16);
+    }
   }
   uint4* d = reinterpret_cast<uint4*>(dst);
   d[0] = make_uint4(w[0], w[1], w[2], w[3]);
   d[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
+// Rows of at most kThreads chunks: a CTA takes G = kThreads / chunks-per-row whole rows per step, so
+// every thread keeps one column chunk (its scale-block columns found once) and walks rows; two row
+// groups per loop trip with both loads issued first.  Wider rows: a CTA walks rows, its threads the
+// row's chunks.  The only per-chunk index arithmetic left is the row's scale row, i / block_m, in
+// 32 bits while M allows.
 __global__ void __launch_bounds__(kThreads) fp8_dequant_kernel(const uint8_t* __restrict__ codes,
                                                                const float* __restrict__ scale_inv,
                                                                uint16_t* __restrict__ out, int64_t M, int64_t N,
                                                                int block_m, int block_n) {
+  static_assert(kThreads == 256, "one decode-table entry per thread");
+  __shared__ float lut[256];
+  lut[threadIdx.x] = __half2float(__half(__nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(threadIdx.x),
+                                                                 __NV_E4M3)));
+  __syncthreads();
   const int64_t per_row = N / 16;
-  const int64_t n_vec = M * per_row;
   const int64_t scale_cols = (N + block_n - 1) / block_n;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; e < n_vec; e += 2 * stride) {
-    const int64_t e2 = e + stride;
-    const bool second = e2 < n_vec;
-    const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(codes) + e);  // chunk e starts at byte 16 e
-    uint4 u1 = make_uint4(0, 0, 0, 0);
-    if (second) u1 = __ldg(reinterpret_cast<const uint4*>(codes) + e2);
-    {
-      const int64_t i = e / per_row;
-      const int j0 = static_cast<int>(e - i * per_row) * 16;
-      fp8_dequant_chunk(u0, scale_inv + (i / block_m) * scale_cols, j0, block_n, out + e * 16);
+  const bool m32 = M <= 0x7FFFFFFF;
+  auto scale_row = [&](int64_t i) {
+    const int64_t r = m32 ? static_cast<int64_t>(static_cast<uint32_t>(i) / static_cast<uint32_t>(block_m))
+                          : i / block_m;
+    return scale_inv + r * scale_cols;
+  };
+  const uint4* src = reinterpret_cast<const uint4*>(codes);  // chunk e starts at byte 16 e
+  if (per_row <= kThreads) {
+    const int pr = static_cast<int>(per_row);
+    const int G = kThreads / pr;
+    const int r_off = static_cast<int>(threadIdx.x) / pr;
+    if (r_off >= G) return;  // no CTA-wide synchronisation follows
+    const int jc = static_cast<int>(threadIdx.x) - r_off * pr;
+    const DequantCols cols = dequant_cols(16 * jc, block_n);
+    const int64_t groups = (M + G - 1) / G;
+    const int64_t gstep = gridDim.x;
+    for (int64_t g = blockIdx.x; g < groups; g += 2 * gstep) {
+      const int64_t i0 = g * G + r_off, i1 = (g + gstep) * G + r_off;
+      const int64_t e0 = i0 * per_row + jc, e1 = i1 * per_row + jc;
+      const bool has0 = i0 < M, has1 = i1 < M;
+      uint4 u0 = make_uint4(0, 0, 0, 0), u1 = make_uint4(0, 0, 0, 0);
+      if (has0) u0 = __ldg(src + e0);
+      if (has1) u1 = __ldg(src + e1);
+      if (has0) fp8_dequant_chunk(u0, scale_row(i0), cols, block_n, lut, out + e0 * 16);
+      if (has1) fp8_dequant_chunk(u1, scale_row(i1), cols, block_n, lut, out + e1 * 16);
     }
-    if (second) {
-      const int64_t i = e2 / per_row;
-      const int j0 = static_cast<int>(e2 - i * per_row) * 16;
-      fp8_dequant_chunk(u1, scale_inv + (i / block_m) * scale_cols, j0, block_n, out + e2 * 16);
+  } else {
+    for (int64_t i = blockIdx.x; i < M; i += gridDim.x) {
+      const float* srow = scale_row(i);
+      for (int64_t jc = threadIdx.x; jc < per_row; jc += 2 * kThreads) {
+        const int64_t jc1 = jc + kThreads;
+        const bool has1 = jc1 < per_row;
+        const uint4 u0 = __ldg(src + i * per_row + jc);
+        uint4 u1 = make_uint4(0, 0, 0, 0);
+        if (has1) u1 = __ldg(src + i * per_row + jc1);
+        fp8_dequant_chunk(u0, srow, dequant_cols(static_cast<int>(16 * jc), block_n), block_n, lut,
+                          out + (i * per_row + jc) * 16);
+        if (has1)
+          fp8_dequant_chunk(u1, srow, dequant_cols(static_cast<int>(16 * jc1), block_n), block_n, lut,
+                            out + (i * per_row + jc1) * 16);
+      }
     }
   }
 }

@@ -347,7 +347,10 @@ MIMO_API int mimo_attn_bwd(const void* q, const void* k, const void* v, const fl
  * aligned, cols a multiple of 16); scale_inv: fp32 [ceil(rows / block_rows),
  * ceil(cols / block_cols)] (device); out: bf16 [rows, cols] (device), each the
  * round-to-nearest-even of the exact product.  The pages do not give the block
- * size (128 x 128 is the usual one).  Does not synchronise.
+ * size (128 x 128 is the usual one).  cols not a multiple of 16 or above
+ * 2^31 - 1: MIMO_ERR_UNSUPPORTED; negative sizes, block sizes below 1, null
+ * or misaligned pointers: MIMO_ERR_INVALID_ARG; no rows or no columns: nothing
+ * to do.  Does not synchronise.
  */
 MIMO_API int mimo_fp8_dequant_blockwise(const void* codes, const float* scale_inv, int64_t rows, int64_t cols,
                                         int block_rows, int block_cols, void* out, void* stream);

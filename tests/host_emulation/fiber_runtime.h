@@ -398,6 +398,7 @@ inline unsigned __ballot_sync(unsigned, int pred) {
 inline int __popc(unsigned v) { return __builtin_popcount(v); }
 inline int __ffs(unsigned v) { return __builtin_ffs(static_cast<int>(v)); }
 inline float __fdiv_rn(float a, float b) { return a / b; }
+inline float __fmul_rn(float a, float b) { return a * b; }  // SSE: one IEEE rounding, subnormals kept
 
 inline float __fdividef(float a, float b) { return a / b; }
 inline float __expf(float x) { return std::exp(x); }

@@ -196,3 +196,21 @@ def test_profile_stride_values(M):
             M.profile_set_stride(bad)
         assert e.value.status == M.ERR_INVALID_ARG
     M.profile_set_stride(1)
+
+
+@pytest.mark.parametrize("args,expect", [
+    (dict(rows=-1), 1),                        # negative size
+    (dict(bm=0), 1),                           # empty scale blocks
+    (dict(bn=-4), 1),
+    (dict(cols=40), 2),                        # rows not made of 16-byte chunks
+    (dict(cols=1 << 31), 2),                   # beyond the kernel's 32-bit column index
+    (dict(codes=FAKE + 8), 1),                 # misaligned
+    (dict(scale=FAKE + 2), 1),
+    (dict(out=None), 1),                       # missing output
+    (dict(rows=0, codes=None, scale=None, out=None), 0),  # nothing to do: no pointer is needed
+])
+def test_fp8_dequant_validation(M, args, expect):
+    a = dict(codes=FAKE, scale=FAKE, rows=256, cols=4096, bm=128, bn=128, out=FAKE)
+    a.update(args)
+    assert M.LIB.mimo_fp8_dequant_blockwise(a["codes"], a["scale"], a["rows"], a["cols"], a["bm"], a["bn"],
+                                            a["out"], None) == expect

@@ -42,12 +42,19 @@ def _cuda_core_kernel():
 
 
 def f64_to_bf16_bits(x):
-    """Round-to-nearest-even of FP64 values to BF16 (one rounding; finite values in FP32 range)."""
-    b = np.asarray(x, dtype=np.float64).view(np.uint64)
+    """Round-to-nearest-even of FP64 values to BF16, one rounding: 8 significant bits in the normal
+    range, the fixed grid of 2^-133 below 2^-126 (subnormals), infinity past the largest finite value."""
+    x = np.asarray(x, dtype=np.float64)
+    b = x.view(np.uint64)
     lsb = (b >> np.uint64(45)) & np.uint64(1)
     r = (b + np.uint64((1 << 44) - 1) + lsb) & ~np.uint64((1 << 45) - 1)  # 8 significant bits left
-    f32 = r.view(np.float64).astype(np.float32)  # exact: at most 8 significant bits
-    return (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    with np.errstate(over="ignore"):
+        f32 = r.view(np.float64).astype(np.float32)  # exact: at most 8 significant bits
+    out = (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    sub = np.abs(x) < 2.0 ** -126
+    m = np.rint(np.abs(x[sub]) * 2.0 ** 133).astype(np.uint16)  # rint rounds halves to even
+    out[sub] = m | (np.signbit(x[sub]).astype(np.uint16) << np.uint16(15))
+    return out
 
 
 def run(lens, hq, hkv, layer, window, base, has_sink, seed, dlse=True, stats="oracle", tol=None):

@@ -18,16 +18,24 @@ def _cuda():
 
 
 def f64_to_bf16_bits(x):
-    """Round-to-nearest-even of FP64 values to BF16 (one rounding; finite values in FP32 range)."""
-    b = np.asarray(x, dtype=np.float64).view(np.uint64)
+    """Round-to-nearest-even of FP64 values to BF16, one rounding: 8 significant bits in the normal
+    range, the fixed grid of 2^-133 below 2^-126 (subnormals), infinity past the largest finite value."""
+    x = np.asarray(x, dtype=np.float64)
+    b = x.view(np.uint64)
     lsb = (b >> np.uint64(45)) & np.uint64(1)
     r = (b + np.uint64((1 << 44) - 1) + lsb) & ~np.uint64((1 << 45) - 1)  # 8 significant bits left
-    f32 = r.view(np.float64).astype(np.float32)  # exact: at most 8 significant bits
-    return (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    with np.errstate(over="ignore"):
+        f32 = r.view(np.float64).astype(np.float32)  # exact: at most 8 significant bits
+    out = (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    sub = np.abs(x) < 2.0 ** -126
+    m = np.rint(np.abs(x[sub]) * 2.0 ** 133).astype(np.uint16)  # rint rounds halves to even
+    out[sub] = m | (np.signbit(x[sub]).astype(np.uint16) << np.uint16(15))
+    return out
 
 
 @pytest.mark.parametrize("shape,block", [((300, 512), (128, 128)), ((128, 16), (128, 128)), ((77, 96), (32, 48)),
-                                         ((45, 160), (16, 40)), ((20, 64), (3, 8))])
+                                         ((45, 160), (16, 40)), ((20, 64), (3, 8)),
+                                         ((5, 4352), (2, 128)), ((3, 8224), (1, 48))])
 def test_fp8_dequant_bit_exact(shape, block):
     _dequant_case(shape, block, False)
 
@@ -39,8 +47,13 @@ TIE_SCALES = np.concatenate([
     # than half an FP32 ulp (found by comparing both roundings over 2e6 random scales)
     np.array([1070475106, 1071501685, 1070290262, 1072649557, 1068944589, 1068420301], dtype=np.uint32)
     .view(np.float32),
-    # products exactly on midpoints (ties to even), and far below the normal range (the FP64 path)
-    np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -9, 2.0 ** -110, 3 * 2.0 ** -112], dtype=np.float32)])
+    # 8883769 * 2^-149, near the bottom of FP32's normal range: its product with 1.125 lies 2^-152 above
+    # a BF16 midpoint, below FP32's smallest subnormal, so an FP32 error term would lose that sticky bit
+    np.array([8883769], dtype=np.uint32).view(np.float32),
+    # products exactly on midpoints (ties to even), far below the normal range (the FP64 path), either
+    # side of 2^-96, past the largest finite value (infinity), and of both signs
+    np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -9, 2.0 ** -110, 3 * 2.0 ** -112, 1.37 * 2.0 ** -100, 1.5 * 2.0 ** 120,
+              -1.3], dtype=np.float32)])
 
 
 @pytest.mark.parametrize("shape,block", [((256, 512), (8, 16)), ((40, 96), (1, 1))])

@@ -38,10 +38,15 @@ def test_kernels_match_oracle(host_lib, mode):
 
 # Mistakes planted in the host copy of the kernels, each of which the cases above must catch.
 PLANTED = [
-    ("one vector read past the end of the codes", "e < n_vec;", "e <= n_vec;", "dequant"),
-    ("dequant rounds the product to FP32 before BF16",
-     "f[h] = __bfloat162float(__double2bfloat16(static_cast<double>(x) * sc));",
-     "f[h] = __bfloat162float(__float2bfloat16(x * static_cast<float>(sc)));", "dequant"),
+    ("dequant reads and writes one row past the end", "has1 = i1 < M;", "has1 = i1 <= M;", "dequant"),
+    ("dequant rounds the FP32 product to BF16 without the midpoint check",
+     "      mid |= (__float_as_uint(b) & 0xFFFFu) == 0x8000u;\n", "", "dequant"),
+    ("dequant takes the first block's scale one column past its edge", "(j < c.edge ? s0 : s1)",
+     "(j <= c.edge ? s0 : s1)", "dequant"),
+    ("dequant's exact path rounds the product to FP32 first",
+     "static_cast<double>(dequant_code(lut, cw[jj >> 2], jj & 3)) *\n                                                  static_cast<double>(sc)",
+     "static_cast<float>(dequant_code(lut, cw[jj >> 2], jj & 3)) *\n                                                  static_cast<float>(sc)",
+     "dequant"),
     ("shared-memory block one row-vector short", "kRows * kPS + 2 * kRows) * 4;", "kRows * kPS + kRows) * 4;",
      "bwd_window0"),
     ("barrier between the K/V load and its rotation dropped",
