@@ -936,9 +936,17 @@ int mimo_moe_route(const float* logits, const float* bias, int64_t tokens, int n
   DeviceInfo* info = device_info(dev);
   if (!info) return MIMO_ERR_CUDA;
   const long long warps_per_cta = nb::kThreads / 32;
-  const unsigned grid = (unsigned)std::min<long long>((tokens + warps_per_cta - 1) / warps_per_cta, 16LL * info->sms);
-  nb::route_kernel<8><<<grid, nb::kThreads, nb::kRouteSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      logits, bias, ids, weights, tokens, num_experts, top_k, normalize ? 1 : 0);
+  if (top_k <= 16) {  // two tokens per warp
+    const long long pairs = (tokens + 1) / 2;
+    const unsigned grid = (unsigned)std::min<long long>((pairs + warps_per_cta - 1) / warps_per_cta, 16LL * info->sms);
+    nb::route_pair_kernel<16><<<grid, nb::kThreads, nb::kRoutePairSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+        logits, bias, ids, weights, tokens, num_experts, top_k, normalize ? 1 : 0);
+  } else {
+    const unsigned grid =
+        (unsigned)std::min<long long>((tokens + warps_per_cta - 1) / warps_per_cta, 16LL * info->sms);
+    nb::route_kernel<8><<<grid, nb::kThreads, nb::kRouteSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+        logits, bias, ids, weights, tokens, num_experts, top_k, normalize ? 1 : 0);
+  }
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 

@@ -386,6 +386,126 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
   }
 }
 
+// Two tokens per warp (top_k <= 16), one per half-warp: lane hl = lane & 15 of half h holds experts
+// hl + 16 m.  The steps of route_kernel on 16 lanes: the threshold is the k-th largest of the half's
+// 16 lane maxima, and a token takes the fast path with at most 16 candidates (one per lane of its
+// half for the FP64 sigmoid).  The warp-wide steps -- the sort of the lane maxima, the FP64 sigmoid,
+// the rank loop and the sums -- then serve both tokens at once.  Each lane packs its candidates as a
+// bit mask; a scan over the half gives each lane its slot, and the candidates' logits are read again
+// (from L1) by the lanes that evaluate them.  A token with more than 16 candidates, fewer than k, or
+// a NaN among their keys takes the exact loop over all its experts, run by the whole warp.
+template <int kMaxPerLane>
+__global__ void __launch_bounds__(kThreads) route_pair_kernel(const float* __restrict__ logits,
+                                                              const float* __restrict__ bias,
+                                                              int32_t* __restrict__ ids, float* __restrict__ weights,
+                                                              int64_t T, int E, int top_k, int normalize) {
+  // per half-warp: 16 candidates' experts, then their keys; after all warps' buffers, the E biases
+  extern __shared__ __align__(16) float sm[];
+  float* s_bias = sm + (kThreads / 32) * 64;
+  for (int e = threadIdx.x; e < E; e += kThreads) s_bias[e] = __ldg(bias + e);
+  __syncthreads();  // the only CTA-wide barrier
+  const int lane = threadIdx.x & 31;
+  const int hl = lane & 15, hbase = lane & 16;
+  int* c_id = reinterpret_cast<int*>(sm) + (threadIdx.x >> 5) * 64 + 2 * hbase;
+  float* c_key = reinterpret_cast<float*>(c_id + 16);
+  const int per_lane = E / 16;
+  const int64_t pair_step = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  float xn[kMaxPerLane];  // the next token's logits
+  int64_t pr = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;  // warp-uniform
+  {
+    const int64_t t = 2 * pr + (hbase >> 4);
+#pragma unroll
+    for (int m = 0; m < kMaxPerLane; ++m)
+      xn[m] = (t < T && m < per_lane) ? __ldg(logits + t * E + hl + 16 * m) : 0.f;
+  }
+  for (; 2 * pr < T; pr += pair_step) {
+    const int64_t t = 2 * pr + (hbase >> 4);
+    const bool live = t < T;
+    const int64_t tn = t + 2 * pair_step;
+    float ka[kMaxPerLane];
+    float lmax = -INFINITY;
+#pragma unroll
+    for (int m = 0; m < kMaxPerLane; ++m) {
+      const float x = xn[m];
+      xn[m] = (tn < T && m < per_lane) ? __ldg(logits + tn * E + hl + 16 * m) : 0.f;  // in flight meanwhile
+      // a NaN key compares false below: never a candidate, and fmaxf passes it over
+      ka[m] = m < per_lane ? route_sigmoid_approx(x) + s_bias[hl + 16 * m] : -INFINITY;
+      lmax = fmaxf(lmax, ka[m]);
+    }
+    // L: the k-th largest lane maximum of the half (bitonic sort of its 16 maxima, descending)
+    float v = lmax;
+#pragma unroll
+    for (int size = 2; size <= 16; size <<= 1)
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, v, stride);
+        v = (((hl & stride) == 0) == ((hl & size) == 0)) ? fmaxf(v, o) : fminf(v, o);
+      }
+    const float kth = __shfl_sync(0xffffffffu, v, hbase + top_k - 1);
+    // the margin of route_kernel: twice the bound on |exact key - approximate key|, with room
+    const float cut = kth - (0x1p-17f + 0x1p-19f * fabsf(kth));
+    uint32_t mask = 0;
+#pragma unroll
+    for (int m = 0; m < kMaxPerLane; ++m)
+      if (ka[m] >= cut) mask |= 1u << m;
+    if (!live) mask = 0;
+    // this lane's first slot: an exclusive scan of the candidate counts over the half
+    const int cnt = __popc(mask);
+    int scan = cnt;
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, scan, o);
+      if (hl >= o) scan += y;
+    }
+    const int n_cand = __shfl_sync(0xffffffffu, scan, hbase + 15);
+    bool fast = live && n_cand >= top_k && n_cand <= 16;
+    if (fast) {
+      int pos = scan - cnt;
+      for (uint32_t mm = mask; mm; mm &= mm - 1) c_id[pos++] = hl + 16 * (__ffs(mm) - 1);
+    }
+    __syncwarp();
+    const bool mine = fast && hl < n_cand;
+    double sc = 0.0;
+    float key = -INFINITY;
+    int id = 0;
+    if (mine) {
+      id = c_id[hl];
+      sc = route_sigmoid_f64(static_cast<double>(__ldg(logits + t * E + id)));
+      key = static_cast<float>(sc) + s_bias[id];  // as in the exact loop
+      c_key[hl] = key;
+    }
+    __syncwarp();
+    if ((__ballot_sync(0xffffffffu, mine && key != key) >> hbase) & 0xFFFFu) fast = false;
+    int rank = 0;
+    if (mine)
+      for (int j = 0; j < n_cand; ++j) {
+        const float kj = c_key[j];
+        rank += (kj > key || (kj == key && c_id[j] < id)) ? 1 : 0;
+      }
+    const bool chosen = fast && mine && rank < top_k;
+    double total = chosen ? sc : 0.0;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+    if (chosen) {
+      ids[t * top_k + rank] = id;
+      weights[t * top_k + rank] = static_cast<float>(normalize ? sc / total : sc);
+    }
+    const uint32_t slow = __ballot_sync(0xffffffffu, live && !fast);
+    __syncwarp();  // the candidate buffers are rewritten for the next pair
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh)
+      if ((slow >> (16 * hh)) & 0xFFFFu) {
+        const int64_t ts = 2 * pr + hh;
+        route_token_exact<(kMaxPerLane + 1) / 2>(logits + ts * E, bias, E / 32, lane, top_k, normalize,
+                                                 ids + ts * top_k, weights + ts * top_k);
+      }
+  }
+}
+
+// Dynamic shared memory of route_pair_kernel: per warp two halves of 16 experts and 16 keys, then
+// the biases of at most 256 experts.
+constexpr uint32_t kRoutePairSmemBytes = ((kThreads / 32) * 64 + 256) * 4;
+
 // Dynamic shared memory of route_kernel: per warp 32 logits, 32 expert indices and 32 keys.
 constexpr uint32_t kRouteSmemBytes = (kThreads / 32) * 96 * 4;
 

@@ -182,7 +182,7 @@ def split(H, hq, hkv, T, seed=52):
         assert np.array_equal(a, r.reshape(a.shape))
 
 
-def route(H, E, k, T, normalize=True, ties=False, pairs=False, seed=53):
+def route(H, E, k, T, normalize=True, ties=False, pairs=False, adjacent=False, seed=53):
     rng = np.random.default_rng(seed)
     logits = (rng.standard_normal((T, E)) * 2).astype(np.float32)
     bias = (rng.standard_normal(E) * 0.1).astype(np.float32)
@@ -192,6 +192,9 @@ def route(H, E, k, T, normalize=True, ties=False, pairs=False, seed=53):
     if pairs:  # every key twice (experts e and e + E/2): the top k are pairs of exact ties
         logits[:, E // 2:] = logits[:, :E // 2]
         bias[E // 2:] = bias[:E // 2]
+    if adjacent:  # every key twice (experts 2i and 2i + 1, held by different lanes): pairs of exact ties
+        logits[:, 1::2] = logits[:, 0::2]
+        bias[1::2] = bias[0::2]
     pi, pw = H.empty((T, k), np.int32), H.empty((T, k), np.float32)
     st = H.L.mimo_moe_route(H.put(logits), H.put(bias), T, E, k, int(normalize), pi, pw, None)
     ids, w = H.get(pi, (T, k), np.int32), H.get(pw, (T, k), np.float32).astype(np.float64)
@@ -250,7 +253,8 @@ CASES = {
     "route": lambda H: (route(H, 256, 8, 200), route(H, 64, 8, 33), route(H, 32, 1, 7),
                         route(H, 256, 8, 64, normalize=False), route(H, 96, 32, 40, ties=True),
                         route(H, 32, 8, 12, ties=True), route(H, 256, 8, 50, pairs=True),
-                        route(H, 64, 32, 20, pairs=True)),
+                        route(H, 64, 32, 20, pairs=True), route(H, 256, 17, 40), route(H, 256, 20, 40, adjacent=True),
+                        route(H, 256, 8, 40, adjacent=True)),
     # 40 new tokens x 4 heads = 160 rows (two tiles) beside one-tile sequences; keys clipped per tile
     "decode_tiles_swa": lambda H: decode(H, [300, 90, 20], [40, 20, 20], 8, 2, LAYER_SWA, 128, 1e4, True, 61,
                                          choice=DECODE_CUDA_CORES),

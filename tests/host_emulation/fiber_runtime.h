@@ -363,6 +363,11 @@ inline T __shfl_xor_sync(unsigned, T v, int o) { return hemu::shfl_idx(v, (hemu:
 template <class T>
 inline T __shfl_sync(unsigned, T v, int src) { return hemu::shfl_idx(v, src); }
 template <class T>
+inline T __shfl_up_sync(unsigned, T v, int d) {  // lanes below d keep their own value
+  const int l = hemu::lin_tid() % 32;
+  return hemu::shfl_idx(v, l >= d ? l - d : l);
+}
+template <class T>
 inline T atomicAdd(T* p, T v) {
   const T o = *p;
   *p = o + v;

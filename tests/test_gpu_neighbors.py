@@ -88,7 +88,8 @@ def test_qkv_split_bit_exact(hq, hkv, T):
         assert np.array_equal(a.view(torch.int16).cpu().numpy().view(np.uint16), r)
 
 
-@pytest.mark.parametrize("E,k,T", [(256, 8, 4099), (64, 8, 33), (32, 1, 7)])
+@pytest.mark.parametrize("E,k,T", [(256, 8, 4099), (64, 8, 33), (32, 1, 7), (256, 16, 1001), (256, 17, 999),
+                                   (256, 20, 513)])
 def test_route(E, k, T):
     from global_attention_moe_b200 import mimo_attn as M
     rng = np.random.default_rng(53)
@@ -142,16 +143,21 @@ def test_route_exact_ties_take_lower_experts():
     assert np.allclose(w.cpu().numpy(), 1.0 / 8, rtol=0, atol=1e-7)
 
 
-@pytest.mark.parametrize("E,k", [(256, 8), (64, 32)])
-def test_route_tied_pairs(E, k):
-    """Every key twice (experts e and e + E/2 share logit and bias): the top k are pairs of exact
-    ties, each ordered by the lower expert first, and the ids match the oracle row for row."""
+@pytest.mark.parametrize("E,k,adjacent", [(256, 8, False), (64, 32, False), (256, 8, True), (256, 20, True)])
+def test_route_tied_pairs(E, k, adjacent):
+    """Every key twice (experts e and e + E/2, or 2i and 2i + 1, share logit and bias): the top k are
+    pairs of exact ties, each ordered by the lower expert first, and the ids match the oracle row for
+    row."""
     from global_attention_moe_b200 import mimo_attn as M
     rng = np.random.default_rng(57)
-    logits = (rng.standard_normal((300, E)) * 2).astype(np.float32)
-    logits[:, E // 2:] = logits[:, :E // 2]
+    logits = (rng.standard_normal((301, E)) * 2).astype(np.float32)
     bias = (rng.standard_normal(E) * 0.1).astype(np.float32)
-    bias[E // 2:] = bias[:E // 2]
+    if adjacent:
+        logits[:, 1::2] = logits[:, 0::2]
+        bias[1::2] = bias[0::2]
+    else:
+        logits[:, E // 2:] = logits[:, :E // 2]
+        bias[E // 2:] = bias[:E // 2]
     ids, w = M.moe_route(torch.from_numpy(logits).cuda(), torch.from_numpy(bias).cuda(), k)
     assert M.check() == M.OK
     ids, w = ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
