@@ -208,13 +208,14 @@ __device__ __forceinline__ double route_sigmoid_f64(double x) {
   return x >= 0 ? 1.0 / (1.0 + exp(-x)) : exp(x) / (1.0 + exp(x));
 }
 
-// Approximate sigmoid: e = __expf(-|x|) is within (2 + 1.173 |x|) ulp of exp(-|x|) and
-// __fdividef within 2 ulp (CUDA's documented bounds), so the absolute error is at most
-// e (2 + 1.173 |x|) 2^-23 + 2^-24 + 2^-22 <= 2^-20.5 (e (2 + 1.173 |x|) <= 2 for all x).
-__device__ __forceinline__ float route_sigmoid_approx(float x) {
-  const float e = __expf(-fabsf(x));
-  return __fdividef(x >= 0.f ? 1.f : e, 1.f + e);
-}
+// Approximate sigmoid 1 / (1 + e), e = __expf(-x): e is within (2 + 1.173 |x|) ulp of exp(-x) and
+// __fdividef within 2 ulp for divisors up to 2^126 (CUDA's documented bounds).  With s the exact
+// sigmoid, e's relative error d moves the result by at most s d e / (1 + e): for x >= 0 that is
+// (2 + 1.173 x) e^-x / (1 + e^-x)^2 2^-23 <= 0.65 2^-23; for x < 0 it is below (2 + 1.173 |x|) /
+// (1 + e^|x|) 2^-23 <= 2^-23.  The rounding of 1 + e adds at most 2^-24 and the division 2 ulp of s
+// (<= 2^-23), so the absolute error is below 2^-21.  Past the divisor's range (x below about -87)
+// the result is 0 against an exact value below 2^-126.
+__device__ __forceinline__ float route_sigmoid_approx(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
 // The exact choice for one token over all its experts.
 template <int kMaxPerLane>
@@ -401,13 +402,14 @@ __global__ void __launch_bounds__(kThreads) route_pair_kernel(const float* __res
                                                               int64_t T, int E, int top_k, int normalize) {
   // per half-warp: 16 candidates' experts, then their keys; after all warps' buffers, the E biases
   extern __shared__ __align__(16) float sm[];
-  float* s_bias = sm + (kThreads / 32) * 64;
+  float* s_bias = sm + (kThreads / 32) * 96;
   for (int e = threadIdx.x; e < E; e += kThreads) s_bias[e] = __ldg(bias + e);
   __syncthreads();  // the only CTA-wide barrier
   const int lane = threadIdx.x & 31;
   const int hl = lane & 15, hbase = lane & 16;
-  int* c_id = reinterpret_cast<int*>(sm) + (threadIdx.x >> 5) * 64 + 2 * hbase;
-  float* c_key = reinterpret_cast<float*>(c_id + 16);
+  int* c_id = reinterpret_cast<int*>(sm) + (threadIdx.x >> 5) * 96 + 3 * hbase;
+  // a candidate's (key, expert) as one integer that orders like (key descending, expert ascending)
+  unsigned long long* c_ord = reinterpret_cast<unsigned long long*>(c_id + 16);
   const int per_lane = E / 16;
   const int64_t pair_step = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
   float xn[kMaxPerLane];  // the next token's logits
@@ -472,16 +474,18 @@ __global__ void __launch_bounds__(kThreads) route_pair_kernel(const float* __res
       id = c_id[hl];
       sc = route_sigmoid_f64(static_cast<double>(__ldg(logits + t * E + id)));
       key = static_cast<float>(sc) + s_bias[id];  // as in the exact loop
-      c_key[hl] = key;
     }
+    // the key's bits made order-preserving as an unsigned integer (-0 taken as +0, which the FP32
+    // comparisons of the exact loop treat as equal), above the complemented expert index
+    const uint32_t kb = __float_as_uint(key + 0.f);
+    const uint32_t ko = (kb & 0x80000000u) ? ~kb : (kb | 0x80000000u);
+    const unsigned long long ord = (static_cast<unsigned long long>(ko) << 32) | static_cast<uint32_t>(~id);
+    if (mine) c_ord[hl] = ord;
     __syncwarp();
     if ((__ballot_sync(0xffffffffu, mine && key != key) >> hbase) & 0xFFFFu) fast = false;
     int rank = 0;
     if (mine)
-      for (int j = 0; j < n_cand; ++j) {
-        const float kj = c_key[j];
-        rank += (kj > key || (kj == key && c_id[j] < id)) ? 1 : 0;
-      }
+      for (int j = 0; j < n_cand; ++j) rank += c_ord[j] > ord ? 1 : 0;
     const bool chosen = fast && mine && rank < top_k;
     double total = chosen ? sc : 0.0;
 #pragma unroll
@@ -502,9 +506,9 @@ __global__ void __launch_bounds__(kThreads) route_pair_kernel(const float* __res
   }
 }
 
-// Dynamic shared memory of route_pair_kernel: per warp two halves of 16 experts and 16 keys, then
-// the biases of at most 256 experts.
-constexpr uint32_t kRoutePairSmemBytes = ((kThreads / 32) * 64 + 256) * 4;
+// Dynamic shared memory of route_pair_kernel: per warp two halves of 16 experts and 16 ordering
+// keys (8 bytes each), then the biases of at most 256 experts.
+constexpr uint32_t kRoutePairSmemBytes = ((kThreads / 32) * 96 + 256) * 4;
 
 // Dynamic shared memory of route_kernel: per warp 32 logits, 32 expert indices and 32 keys.
 constexpr uint32_t kRouteSmemBytes = (kThreads / 32) * 96 * 4;

@@ -182,10 +182,10 @@ def split(H, hq, hkv, T, seed=52):
         assert np.array_equal(a, r.reshape(a.shape))
 
 
-def route(H, E, k, T, normalize=True, ties=False, pairs=False, adjacent=False, seed=53):
+def route(H, E, k, T, normalize=True, ties=False, pairs=False, adjacent=False, shift=0.0, seed=53):
     rng = np.random.default_rng(seed)
     logits = (rng.standard_normal((T, E)) * 2).astype(np.float32)
-    bias = (rng.standard_normal(E) * 0.1).astype(np.float32)
+    bias = (rng.standard_normal(E) * 0.1 + shift).astype(np.float32)  # shift -2: every key negative
     if ties:  # rows of equal logits with a zero bias: the choice is the k lowest expert indices
         logits[::3] = 0.5
         bias[:] = 0
@@ -254,7 +254,8 @@ CASES = {
                         route(H, 256, 8, 64, normalize=False), route(H, 96, 32, 40, ties=True),
                         route(H, 32, 8, 12, ties=True), route(H, 256, 8, 50, pairs=True),
                         route(H, 64, 32, 20, pairs=True), route(H, 256, 17, 40), route(H, 256, 20, 40, adjacent=True),
-                        route(H, 256, 8, 40, adjacent=True)),
+                        route(H, 256, 8, 40, adjacent=True), route(H, 256, 8, 40, shift=-2.0),
+                        route(H, 64, 20, 30, shift=-2.0)),
     # 40 new tokens x 4 heads = 160 rows (two tiles) beside one-tile sequences; keys clipped per tile
     "decode_tiles_swa": lambda H: decode(H, [300, 90, 20], [40, 20, 20], 8, 2, LAYER_SWA, 128, 1e4, True, 61,
                                          choice=DECODE_CUDA_CORES),

@@ -88,13 +88,15 @@ def test_qkv_split_bit_exact(hq, hkv, T):
         assert np.array_equal(a.view(torch.int16).cpu().numpy().view(np.uint16), r)
 
 
-@pytest.mark.parametrize("E,k,T", [(256, 8, 4099), (64, 8, 33), (32, 1, 7), (256, 16, 1001), (256, 17, 999),
-                                   (256, 20, 513)])
-def test_route(E, k, T):
+@pytest.mark.parametrize("E,k,T,shift", [(256, 8, 4099, 0.0), (64, 8, 33, 0.0), (32, 1, 7, 0.0), (256, 16, 1001, 0.0),
+                                         (256, 17, 999, 0.0), (256, 20, 513, 0.0), (256, 8, 777, -2.0),
+                                         (64, 20, 301, -2.0)])
+def test_route(E, k, T, shift):
+    """Ids equal to the oracle's up to FP32 key ties; with the bias shifted by -2 every key is negative."""
     from global_attention_moe_b200 import mimo_attn as M
     rng = np.random.default_rng(53)
     logits = (rng.standard_normal((T, E)) * 2).astype(np.float32)
-    bias = (rng.standard_normal(E) * 0.1).astype(np.float32)
+    bias = (rng.standard_normal(E) * 0.1 + shift).astype(np.float32)
     ids, w = M.moe_route(torch.from_numpy(logits).cuda(), torch.from_numpy(bias).cuda(), k)
     ids, w = ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
     rid, rw, key = NB.route(logits, bias, k)

@@ -54,8 +54,8 @@ PLANTED = [
      "    for (int e = tid; e < kChunk * (kRopeDims / 2); e += kThreads) {", "bwd_window0"),
     ("window mask one key short", "pos - kpos <= P.window", "pos - kpos < P.window", "bwd_window31_mqa"),
     ("router ties to the higher expert", "(ok == bk && oe < be)", "(ok == bk && oe > be)", "route"),
-    ("two-token router: the halves' candidate buffers overlap", "(threadIdx.x >> 5) * 64 + 2 * hbase;",
-     "(threadIdx.x >> 5) * 64 + hbase;", "route"),
+    ("two-token router: the halves' candidate buffers overlap", "(threadIdx.x >> 5) * 96 + 3 * hbase;",
+     "(threadIdx.x >> 5) * 96 + hbase;", "route"),
     ("two-token router: slot scan skips one lane's count", "if (hl >= o) scan += y;", "if (hl > o) scan += y;",
      "route"),
     ("two-token router: the exact loop runs for the first token of the pair", "const int64_t ts = 2 * pr + hh;",
@@ -63,8 +63,9 @@ PLANTED = [
     ("router ranks tied candidates by the higher expert", "\n            rank += (kj > key || (kj == key && c_id[j] < id))",
      "\n            rank += (kj > key || (kj == key && c_id[j] > id))", "route"),
     ("two-token router ranks tied candidates by the higher expert",
-     "\n        rank += (kj > key || (kj == key && c_id[j] < id))",
-     "\n        rank += (kj > key || (kj == key && c_id[j] > id))", "route"),
+     "| static_cast<uint32_t>(~id);", "| static_cast<uint32_t>(id);", "route"),
+    ("two-token router orders negative keys as unsigned bits", "(kb & 0x80000000u) ? ~kb : (kb | 0x80000000u)",
+     "kb", "route"),
     ("router candidates all written to the first slot", "const int pos = at + __popc(cand[m] & ((1u << lane) - 1u));",
      "const int pos = at;", "route"),
     ("decode row tiles all start at row 0", "const int row0 = kMaxRows * qt;", "const int row0 = 0;",
