@@ -111,32 +111,48 @@ __device__ __forceinline__ void flush_rows(const float* stage, int nrows, float*
   }
 }
 
-// Stages this thread's gradient row R(-pos) scale x (x: 6 x 32 TMEM words, the 192 Q/K dims; the
-// rotate-half pairs (i, i + 32) of the first 64 are turned back by -pos).
-__device__ __forceinline__ void stage_rotated_row(float* stage, int r, const uint32_t (&x)[6][32], int pos,
-                                                  float scale, const double* theta) {
+// Stages this thread's gradient row R(-pos) scale x, x read from its TMEM lane at columns taddr ..
+// taddr + 191 (the 192 Q/K dims) 64 columns at a time; the rotate-half pairs (i, i + 32) of the first
+// 64 are turned back by -pos.
+__device__ __forceinline__ void stage_rotated_row(float* stage, int r, uint32_t taddr, int pos, float scale,
+                                                  const double* theta) {
+  {
+    uint32_t x[2][32];
+    tmem_ld32(taddr, x[0]);
+    tmem_ld32(taddr + 32, x[1]);
+    tmem_ld_wait(x[0]);
+    reg_fence(x[1]);
 #pragma unroll
-  for (int c4 = 0; c4 < 8; ++c4) {
-    float lo[4], hi[4];
+    for (int c4 = 0; c4 < 8; ++c4) {
+      float lo[4], hi[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = 4 * c4 + u;
-      float sn, cs;
-      rope_sincos(pos, theta[i], sn, cs);
-      const float a = __uint_as_float(x[0][i]) * scale, b = __uint_as_float(x[1][i]) * scale;
-      lo[u] = a * cs + b * sn;
-      hi[u] = b * cs - a * sn;
+      for (int u = 0; u < 4; ++u) {
+        const int i = 4 * c4 + u;
+        float sn, cs;
+        rope_sincos(pos, theta[i], sn, cs);
+        const float a = __uint_as_float(x[0][i]) * scale, b = __uint_as_float(x[1][i]) * scale;
+        lo[u] = a * cs + b * sn;
+        hi[u] = b * cs - a * sn;
+      }
+      stage4<kHeadDimQK>(stage, r, c4, lo[0], lo[1], lo[2], lo[3]);
+      stage4<kHeadDimQK>(stage, r, 8 + c4, hi[0], hi[1], hi[2], hi[3]);
     }
-    stage4<kHeadDimQK>(stage, r, c4, lo[0], lo[1], lo[2], lo[3]);
-    stage4<kHeadDimQK>(stage, r, 8 + c4, hi[0], hi[1], hi[2], hi[3]);
   }
 #pragma unroll
-  for (int j = 2; j < 6; ++j)
+  for (int j = 2; j < 6; j += 2) {
+    uint32_t x[2][32];
+    tmem_ld32(taddr + 32 * j, x[0]);
+    tmem_ld32(taddr + 32 * (j + 1), x[1]);
+    tmem_ld_wait(x[0]);
+    reg_fence(x[1]);
 #pragma unroll
-    for (int c4 = 0; c4 < 8; ++c4)
-      stage4<kHeadDimQK>(stage, r, 8 * j + c4, __uint_as_float(x[j][4 * c4]) * scale,
-                         __uint_as_float(x[j][4 * c4 + 1]) * scale, __uint_as_float(x[j][4 * c4 + 2]) * scale,
-                         __uint_as_float(x[j][4 * c4 + 3]) * scale);
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4)
+        stage4<kHeadDimQK>(stage, r, 8 * (j + h) + c4, __uint_as_float(x[h][4 * c4]) * scale,
+                           __uint_as_float(x[h][4 * c4 + 1]) * scale, __uint_as_float(x[h][4 * c4 + 2]) * scale,
+                           __uint_as_float(x[h][4 * c4 + 3]) * scale);
+  }
 }
 
 }  // namespace bwdtc
@@ -174,7 +190,8 @@ __global__ void __launch_bounds__(256) bwdtc_prep_kernel(const __grid_constant__
 __global__ void __launch_bounds__(bwdtc::kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                       const __grid_constant__ bwd::BwdParams P, const uint64_t wait_limit_ns) {
+                       const __grid_constant__ bwd::BwdParams P, const int heads_per_cta,
+                       const uint64_t wait_limit_ns) {
   using namespace bwdtc;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~uintptr_t(1023));
@@ -184,17 +201,19 @@ __global__ void __launch_bounds__(bwdtc::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int kt = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
+  // heads h0 .. h0 + heads_per_cta - 1, all of KV group g: K / V loaded and rotated once, dK / dV
+  // accumulated over them in TMEM and added to global memory once
+  const int kt = blockIdx.x, b = blockIdx.y, h0 = blockIdx.z * heads_per_cta;
   const int s_b = __ldg(P.cu_seqlens + b), e_b = __ldg(P.cu_seqlens + b + 1);
   if (s_b < 0 || e_b < s_b || e_b > P.total_tokens) {
-    if (tid == 0 && kt == 0 && h == 0) atomicOr(&g_mimo_error, kErrSeqlens);
+    if (tid == 0 && kt == 0 && h0 == 0) atomicOr(&g_mimo_error, kErrSeqlens);
     return;
   }
   const int L = e_b - s_b;
   const int k0 = kt * 128;
   if (k0 >= L) return;
   const int nk = min(128, L - k0);
-  const int g = h / P.group;
+  const int g = h0 / P.group;
   const uint32_t base = smem_u32(sm);
 
   if (tid == 0) {
@@ -229,7 +248,9 @@ __global__ void __launch_bounds__(bwdtc::kThreads, 1)
     const int q_last = P.window >= 0 ? min(L - 1, k0 + nk - 1 + P.window) : L - 1;
     const int key = k0 + tid;  // this thread's key (S / dP / dV / dK rows)
     const float sl2 = P.scale * kLog2e;
-    for (int q0 = k0 / 128 * 128, first = 1; q0 <= q_last; q0 += 128, first = 0) {
+#pragma unroll 1
+    for (int h = h0; h < h0 + heads_per_cta; ++h) {
+    for (int q0 = k0 / 128 * 128, first = h == h0; q0 <= q_last; q0 += 128, first = 0) {
       const int nq = min(128, L - q0);
       fence_proxy_async_smem();
       __syncthreads();  // the previous tile's MMAs and reads are done; K~ rotated (first pass)
@@ -337,19 +358,15 @@ __global__ void __launch_bounds__(bwdtc::kThreads, 1)
       tc_fence_after_sync();
       // dq for the tile's query rows (TMEM lane = query): R(-pos) scale dQ~, staged then added row-wise
       {
-        uint32_t r[6][32];
-#pragma unroll
-        for (int j = 0; j < 6; ++j) tmem_ld32(tmem + lane_base + kColDQ + 32 * j, r[j]);
-        tmem_ld_wait(r[0]);
-#pragma unroll
-        for (int j = 1; j < 6; ++j) reg_fence(r[j]);
         float* stage = reinterpret_cast<float*>(sm + kOffStage);
-        stage_rotated_row(stage, tid, r, q0 + tid, P.scale, P.theta);
+        stage_rotated_row(stage, tid, tmem + lane_base + kColDQ, q0 + tid, P.scale, P.theta);
         __syncthreads();
         flush_rows<kHeadDimQK>(stage, nq, P.dq + (static_cast<size_t>(s_b + q0) * P.hq + h) * kHeadDimQK,
                                static_cast<size_t>(P.hq) * kHeadDimQK, warp, tid & 31);
       }
       tc_fence_before_sync();
+    }
+    if (fail) break;
     }
     if (fail) break;
 
@@ -377,13 +394,7 @@ __global__ void __launch_bounds__(bwdtc::kThreads, 1)
       __syncthreads();
     }
     {
-      uint32_t r[6][32];
-#pragma unroll
-      for (int j = 0; j < 6; ++j) tmem_ld32(tmem + lane_base + kColDK + 32 * j, r[j]);
-      tmem_ld_wait(r[0]);
-#pragma unroll
-      for (int j = 1; j < 6; ++j) reg_fence(r[j]);
-      stage_rotated_row(stage, tid, r, key, P.scale, P.theta);
+      stage_rotated_row(stage, tid, tmem + lane_base + kColDK, key, P.scale, P.theta);
       __syncthreads();
       flush_rows<kHeadDimQK>(stage, nk, P.dk + (static_cast<size_t>(s_b + k0) * P.hkv + g) * kHeadDimQK,
                              static_cast<size_t>(P.hkv) * kHeadDimQK, warp, tid & 31);

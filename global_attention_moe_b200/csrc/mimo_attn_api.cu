@@ -34,6 +34,7 @@ using namespace mimo;
 namespace {
 
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s bound on any single wait
+constexpr int kBwdHeadsPerCta = 2;  // tensor-core backward: query heads of one KV group per CTA (a power of 2)
 
 PFN_cuTensorMapEncodeTiled_v12000 tensormap_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -660,8 +661,15 @@ int launch_bwd(const void* q, const void* k, const void* v, const float* sink, c
       bwdtc_prep_kernel<<<info->sms * 8, 256, 0, stream>>>(P);
       if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
       if (st == MIMO_OK && d->max_seqlen > 0) {
-        dim3 grid((unsigned)((d->max_seqlen + 127) / 128), (unsigned)d->num_seqs, (unsigned)d->num_q_heads);
-        attn_bwd_tc_kernel<<<grid, bwdtc::kThreads, bwdtc::kSmemBytes, stream>>>(tq, tk, tv, to, P,
+        // query heads per CTA: the most, up to kBwdHeadsPerCta, that divide the KV group
+        int hpc = 1;
+        for (int c = kBwdHeadsPerCta; c > 1; c /= 2)
+          if (P.group % c == 0) {
+            hpc = c;
+            break;
+          }
+        dim3 grid((unsigned)((d->max_seqlen + 127) / 128), (unsigned)d->num_seqs, (unsigned)(d->num_q_heads / hpc));
+        attn_bwd_tc_kernel<<<grid, bwdtc::kThreads, bwdtc::kSmemBytes, stream>>>(tq, tk, tv, to, P, hpc,
                                                                                  kDefaultWaitLimitNs);
         if (cudaGetLastError() != cudaSuccess) st = MIMO_ERR_CUDA;
       }

@@ -123,6 +123,8 @@ PLANTED = [
     ("backward dQ reads dS without its MN-major flag", "attn_bwd_tc.cuh",
      "kIdescDQ = make_idesc_f32acc(1, 1, 128, 192) | (1u << 15);", "kIdescDQ = make_idesc_f32acc(1, 1, 128, 192);",
      "bwd_tensor"),
+    ("backward: dK / dV restarted for every head a CTA takes", "attn_bwd_tc.cuh", "first = h == h0;", "first = 1;",
+     "bwd_tensor"),
     ("packed kernel: score columns mapped to keys one ring slot off", "attn_fwd_swa_packed.cuh",
      "const int c0 = (base + klo) % S::kN;", "const int c0 = (base + klo + kBlk) % S::kN;", "fwd_packed_g8"),
     ("packed kernel: K rotated at the next key's position", "attn_fwd_swa_packed.cuh",
