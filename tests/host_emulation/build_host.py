@@ -105,7 +105,7 @@ def generate() -> str:
     errs = sm100[a:sm100.index("};", a) + 2]
     validate = api[api.index("bool aligned16(const void* p)"):api.index("void fill_params(")]
     validate += api[api.index("// Query rows per KV head (q_len x Hq/Hkv)"):api.index("int launch_decode(")]
-    lines = [ln for ln in api.splitlines() if ln.startswith(("constexpr uint64_t kDefaultWaitLimitNs",
+    lines = [ln for ln in api.splitlines() if ln.startswith(("constexpr uint64_t kDefaultWaitLimitNs", "constexpr int kBwdHeadsPerCta",
                                                              "std::atomic<int> g_decode_choice", "size_t align256(",
                                                              "std::atomic<int> g_bwd_choice"))]
     assert len(lines) >= 3, lines
