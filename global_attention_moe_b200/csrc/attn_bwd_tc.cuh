@@ -18,8 +18,8 @@
 //   at the end v_scale dV and R(-pos) scale dK~ of the key rows are added to dv / dk the same way
 //   (the query heads of a KV group add to the same rows).
 // The rotated Q / K dims enter the MMAs as BF16 (one rounding of the rotation), P and dS as BF16.
-// bwdtc_prep_kernel: D - dLSE per (token, head) and the sink gradient (dq, dk, dv, dsink zeroed by
-// the host before).  The work is serialised inside a CTA (load, MMA, softmax-side math, MMA);
+// bwdtc_prep_kernel: D - dLSE per (token, head) and the sink gradient; it also zeroes dq, dk, dv
+// (dsink is zeroed by the host before).  The work is serialised inside a CTA (load, MMA, softmax-side math, MMA);
 // overlap comes from the CTAs resident on other SMs.
 #pragma once
 
@@ -167,6 +167,14 @@ __global__ void __launch_bounds__(256) bwdtc_prep_kernel(const __grid_constant__
   const int lane = threadIdx.x & 31;
   const long long classes = nwarps / P.hq > 0 ? nwarps / P.hq : 1;  // token stride classes per head
   const bool sink = P.sink != nullptr && P.dsink != nullptr;
+  {  // dq, dk, dv zeroed (16-byte aligned, whole rows of 4-float groups); the main kernel adds into them
+    const long long i0 = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x, n = static_cast<long long>(gridDim.x) * 256;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    const long long nq = T * P.hq * (kHeadDimQK / 4), nk = T * P.hkv * (kHeadDimQK / 4), nv = T * P.hkv * (kHeadDimV / 4);
+    for (long long i = i0; i < nq; i += n) reinterpret_cast<float4*>(P.dq)[i] = z;
+    for (long long i = i0; i < nk; i += n) reinterpret_cast<float4*>(P.dk)[i] = z;
+    for (long long i = i0; i < nv; i += n) reinterpret_cast<float4*>(P.dv)[i] = z;
+  }
   for (long long item = warp; item < classes * P.hq; item += nwarps) {
     const int h = static_cast<int>(item / classes);
     float ds = 0.f;

@@ -650,10 +650,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const float* sink, c
   if (g_bwd_choice.load() != 1) {  // tensor cores: dq / dk / dv / dsink accumulate with atomics
     const size_t T = (size_t)d->total_tokens;
     CUtensorMap tq, tk, tv, to;
-    if (cudaMemsetAsync(dq, 0, T * P.hq * kHeadDimQK * 4, stream) != cudaSuccess ||
-        cudaMemsetAsync(dk, 0, T * P.hkv * kHeadDimQK * 4, stream) != cudaSuccess ||
-        cudaMemsetAsync(dv, 0, T * P.hkv * kHeadDimV * 4, stream) != cudaSuccess ||
-        (dsink && cudaMemsetAsync(dsink, 0, P.hq * 4, stream) != cudaSuccess) ||
+    // dq / dk / dv are zeroed by the prep kernel, dsink here
+    if ((dsink && cudaMemsetAsync(dsink, 0, P.hq * 4, stream) != cudaSuccess) ||
         !encode_2d(&tq, q, (uint64_t)P.hq * kHeadDimQK, T) || !encode_2d(&tk, k, (uint64_t)P.hkv * kHeadDimQK, T) ||
         !encode_2d(&tv, v, (uint64_t)P.hkv * kHeadDimV, T) || !encode_2d(&to, dout, (uint64_t)P.hq * kHeadDimV, T)) {
       st = MIMO_ERR_CUDA;
