@@ -945,8 +945,12 @@ int mimo_moe_route(const float* logits, const float* bias, int64_t tokens, int n
   if (top_k <= 16) {  // two tokens per warp
     const long long pairs = (tokens + 1) / 2;
     const unsigned grid = (unsigned)std::min<long long>((pairs + warps_per_cta - 1) / warps_per_cta, 16LL * info->sms);
-    nb::route_pair_kernel<16><<<grid, nb::kThreads, nb::kRoutePairSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-        logits, bias, ids, weights, tokens, num_experts, top_k, normalize ? 1 : 0);
+    if (num_experts == 256)
+      nb::route_pair_kernel<16, true><<<grid, nb::kThreads, nb::kRoutePairSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+          logits, bias, ids, weights, tokens, num_experts, top_k, normalize ? 1 : 0);
+    else
+      nb::route_pair_kernel<16, false><<<grid, nb::kThreads, nb::kRoutePairSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+          logits, bias, ids, weights, tokens, num_experts, top_k, normalize ? 1 : 0);
   } else {
     const unsigned grid =
         (unsigned)std::min<long long>((tokens + warps_per_cta - 1) / warps_per_cta, 16LL * info->sms);

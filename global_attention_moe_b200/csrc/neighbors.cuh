@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
 // bit mask; a scan over the half gives each lane its slot, and the candidates' logits are read again
 // (from L1) by the lanes that evaluate them.  A token with more than 16 candidates, fewer than k, or
 // a NaN among their keys takes the exact loop over all its experts, run by the whole warp.
-template <int kMaxPerLane>
+template <int kMaxPerLane, bool kFull>  // kFull: E == 16 kMaxPerLane, every lane holds kMaxPerLane experts
 __global__ void __launch_bounds__(kThreads) route_pair_kernel(const float* __restrict__ logits,
                                                               const float* __restrict__ bias,
                                                               int32_t* __restrict__ ids, float* __restrict__ weights,
@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(kThreads) route_pair_kernel(const float* __res
   int* c_id = reinterpret_cast<int*>(sm) + (threadIdx.x >> 5) * 96 + 3 * hbase;
   // a candidate's (key, expert) as one integer that orders like (key descending, expert ascending)
   unsigned long long* c_ord = reinterpret_cast<unsigned long long*>(c_id + 16);
-  const int per_lane = E / 16;
+  const int per_lane = kFull ? kMaxPerLane : E / 16;
   const int64_t pair_step = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
   float xn[kMaxPerLane];  // the next token's logits
   int64_t pr = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;  // warp-uniform

@@ -62,7 +62,7 @@ def _launches(s):
         parts = _split_top(m.group(2))
         smem = parts[2] if len(parts) > 2 else "0"
         return f"g_launch_ok = hemu::launch(dim3({parts[0]}), dim3({parts[1]}), {smem}, [&] {{ {m.group(1)}({m.group(3)}); }});"
-    return re.subn(r"([\w:]+(?:<\d+>)?)<<<(.*?)>>>\((.*?)\);", rep, s, flags=re.S)
+    return re.subn(r"([\w:]+(?:<[\w, ]+>)?)<<<(.*?)>>>\((.*?)\);", rep, s, flags=re.S)
 
 
 HOST_FORMS = [
