@@ -249,7 +249,7 @@ CASES = {
                           dequant(H, (45, 160), (16, 40)), dequant(H, (20, 64), (3, 8)),
                           dequant(H, (64, 256), (4, 16), ties=True), dequant(H, (40, 96), (1, 1), ties=True),
                           dequant(H, (5, 4352), (2, 128)), dequant(H, (3, 8224), (1, 48), ties=True)),
-    "split": lambda H: (split(H, 64, 8, 33), split(H, 6, 2, 9), split(H, 8, 8, 3)),
+    "split": lambda H: (split(H, 64, 8, 33), split(H, 6, 2, 9), split(H, 8, 8, 3), split(H, 64, 4, 17)),
     "route": lambda H: (route(H, 256, 8, 200), route(H, 64, 8, 33), route(H, 32, 1, 7),
                         route(H, 256, 8, 64, normalize=False), route(H, 96, 32, 40, ties=True),
                         route(H, 32, 8, 12, ties=True), route(H, 256, 8, 50, pairs=True),
