@@ -54,8 +54,8 @@ PLANTED = [
      "    for (int e = tid; e < kChunk * (kRopeDims / 2); e += kThreads) {", "bwd_window0"),
     ("window mask one key short", "pos - kpos <= P.window", "pos - kpos < P.window", "bwd_window31_mqa"),
     ("router ties to the higher expert", "(ok == bk && oe < be)", "(ok == bk && oe > be)", "route"),
-    ("QKV split writes V eight elements off", "dst = vr + g * 128 + (o - group * 192 - 192);",
-     "dst = vr + g * 128 + (o - group * 192 - 184);", "split"),
+    ("QKV split writes V eight elements off", "dst = v + (t * hkv + g) * 128 + (o - group * 192 - 192);",
+     "dst = v + (t * hkv + g) * 128 + (o - group * 192 - 184);", "split"),
     ("two-token router: the halves' candidate buffers overlap", "(threadIdx.x >> 5) * 96 + 3 * hbase;",
      "(threadIdx.x >> 5) * 96 + hbase;", "route"),
     ("two-token router: slot scan skips one lane's count", "if (hl >= o) scan += y;", "if (hl > o) scan += y;",
