@@ -204,7 +204,8 @@ CASES = {
     # the backward on the tensor cores (BF16 operands: 1e-2) and on the CUDA cores (FP32: 1e-4)
     "bwd_tensor": lambda H: [bwd(H, *c, "tensor", 1e-2) for c in (
         ([300, 129, 17, 1], 8, 2, W.LAYER_SWA, 128, 1e4, True, 41), ([200, 70], 4, 2, W.LAYER_SWA, 0, 1e4, False, 42),
-        ([333, 64, 5], 8, 2, W.LAYER_GLOBAL, -1, 1e7, False, 43), ([150, 40], 6, 2, W.LAYER_SWA, 128, 1e4, True, 44))],
+        ([333, 64, 5], 8, 2, W.LAYER_GLOBAL, -1, 1e7, False, 43), ([150, 40], 6, 2, W.LAYER_SWA, 128, 1e4, True, 44),
+        ([90, 30], 2, 2, W.LAYER_GLOBAL, -1, 1e7, False, 45))],
     "bwd_cuda_cores": lambda H: bwd(H, [300, 129, 17, 1], 8, 2, W.LAYER_SWA, 128, 1e4, True, 41, "cuda_cores", 1e-4),
     # the packed window kernel (query heads of a KV group in the tile's rows): 32 tokens x 4 heads on the
     # small config; 16 tokens x 8 heads across ragged and empty sequences, windows 0 .. 128 (run with few
